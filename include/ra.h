@@ -1,0 +1,172 @@
+/* ra.h -- C ABI of the Ring Attention exact-forward library for NVIDIA B200 (sm_100a).
+ *
+ * The operation (all five pages on Ring Attention agree on it): exact softmax attention
+ *     out = softmax(Q K^T / sqrt(D)) V
+ * over one long sequence whose tokens are split into n_ring shards.  Shard i keeps its queries;
+ * at ring step s it meets the key/value block of shard j = (i - s) mod n_ring
+ * (ultralytics.com "Ring Attention", section "how ring attention works"; jisaku.com
+ * "Ring Attention", 処理フロー), scores it, and merges the partial result into running
+ * statistics with the online-softmax identities m' = max(m_p, m_n),
+ * l' = e^{m_p - m'} l_p + e^{m_n - m'} l_n (troisinh.com "Ring Attention", "Tai sao no hoat
+ * dong"), so that after n_ring steps the result equals full attention.  Here the ring is
+ * virtual: every shard lives on the one GPU, and "the next block arrives" means "the next key/value
+ * tile address".
+ *
+ * Conventions shared by every entry point
+ *   - Tensors q, k, v, out are [B, S, H, D] row-major (D fastest) in NATURAL token order, the
+ *     (batch, seq, heads, head_dim) order of the ring-flash-attn example on jisaku.com.
+ *   - lse is [B, H, S] fp32 in natural token order: the natural-log log-sum-exp of the scaled
+ *     scores of each query row (lse = m + ln l).
+ *   - scale = 1/sqrt(D) (the toy on ultralytics.com divides by dim**0.5).
+ *   - causal != 0 masks key position g_k > query position g_q, on ORIGINAL token positions, the
+ *     diagonal included, whatever the layout.
+ *   - layout chooses which tokens shard i owns (S_loc = S / n_ring):
+ *       RA_LAYOUT_CONTIGUOUS: local token a is global token i*S_loc + a (aiunderstanding.org:
+ *                             each GPU owns a contiguous chunk);
+ *       RA_LAYOUT_STRIPED:    local token a is global token a*n_ring + i (ultralytics.com: tokens
+ *                             spread evenly over the sequence);
+ *       RA_LAYOUT_ZIGZAG:     with C = S/(2 n_ring), local token a < C is global i*C + a and
+ *                             a >= C is global (2 n_ring - 1 - i)*C + (a - C) (aiunderstanding.org
+ *                             names zigzag; this two-chunk form is the reading adopted).
+ *     The result does not depend on the layout (exactness); the layout only changes how the
+ *     causal work is spread over shards and steps.
+ *   - dtype: RA_DTYPE_FP32 (exact fp32 arithmetic) or RA_DTYPE_BF16 (bf16 inputs, fp32
+ *     accumulation, bf16 output rounded to nearest even).  q, k, v, out share the dtype.
+ *   - All device pointers are CUDA device addresses on the current device; the caller owns every
+ *     buffer (including any workspace) and the library keeps no pointer past the call.
+ *   - stream is a cudaStream_t (NULL = legacy default stream).  Work is enqueued on it and the
+ *     call returns after enqueueing; nothing synchronises the device.
+ *   - Return value: RA_OK (0) or a negative RA_ERR_* code; no exception crosses the ABI.
+ *     Arguments are validated before anything is enqueued; a validation error enqueues nothing.
+ */
+#ifndef RA_H
+#define RA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define RA_API __attribute__((visibility("default")))
+#else
+#define RA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+enum ra_layout { RA_LAYOUT_CONTIGUOUS = 0, RA_LAYOUT_STRIPED = 1, RA_LAYOUT_ZIGZAG = 2 };
+enum ra_dtype { RA_DTYPE_FP32 = 0, RA_DTYPE_BF16 = 1 };
+
+/* Kernel path for ra_forward_ex.
+ *   RA_VARIANT_FUSED:    one persistent launch walks all n_ring steps per query tile and keeps the
+ *                        running (m, l, O) on chip (ultralytics.com toy loop structure).
+ *   RA_VARIANT_PER_STEP: one attention launch per ring step writes a partial (O_s, lse_s); an
+ *                        HBM-bound merge launch folds it into the running (O, lse) with the
+ *                        log-sum-exp form of the merge identities.
+ *   RA_VARIANT_AUTO:     FUSED. */
+enum ra_variant { RA_VARIANT_AUTO = 0, RA_VARIANT_FUSED = 1, RA_VARIANT_PER_STEP = 2 };
+
+/* Kernel family for ra_forward_ex.
+ *   RA_KERNEL_AUTO:    tcgen05 tensor-core kernel for bf16 with D in {64, 128}; SIMT otherwise.
+ *   RA_KERNEL_TC:      require the tensor-core kernel (RA_ERR_UNSUPPORTED if it cannot apply).
+ *   RA_KERNEL_SIMT:    CUDA-core kernel with fp32 arithmetic (any dtype, D <= 256). */
+enum ra_kernel { RA_KERNEL_AUTO = 0, RA_KERNEL_TC = 1, RA_KERNEL_SIMT = 2 };
+
+enum ra_status {
+    RA_OK = 0,
+    RA_ERR_INVALID_ARG = -1,     /* null pointer, bad enum, negative size */
+    RA_ERR_SHAPE = -2,           /* S % n_ring != 0, zigzag S % (2 n_ring) != 0, D unsupported */
+    RA_ERR_ALIGN = -3,           /* a tensor pointer is not 16-byte aligned */
+    RA_ERR_UNSUPPORTED = -4,     /* no sm_100 device, or RA_KERNEL_TC cannot apply */
+    RA_ERR_NO_WORKSPACE = -5,    /* caller workspace smaller than ra_workspace_size */
+    RA_ERR_CUDA = -6,            /* a CUDA runtime/driver call failed (see ra_last_error_string) */
+    RA_ERR_DEVICE_TIMEOUT = -7   /* a bounded in-kernel wait expired (from ra_get_device_status) */
+};
+
+/* Debug knobs (ra_options.debug).  RA_DEBUG_STALL_LOADS makes the tensor-core kernel's load warp
+ * issue no copies, so every consumer wait runs out: a test of the bounded-wait give-up path. */
+enum ra_debug { RA_DEBUG_NONE = 0, RA_DEBUG_STALL_LOADS = 1 };
+
+typedef struct ra_options {
+    int variant;             /* enum ra_variant */
+    int kernel;              /* enum ra_kernel */
+    void* workspace;         /* device buffer of >= ra_workspace_size bytes, 256-byte aligned;
+                                NULL: the call allocates stream-ordered (cudaMallocAsync) and frees
+                                it the same way on `stream` */
+    size_t workspace_bytes;
+    uint64_t timeout_ns;     /* limit for every in-kernel wait; 0 = 2 s */
+    int debug;               /* enum ra_debug */
+    void* attn_events[2];    /* optional cudaEvent_t pair recorded on `stream` right before the
+                                first and right after the last attention-kernel launch */
+} ra_options;
+
+/* ra_forward: exact attention as described above, with the defaults of ra_options (variant AUTO,
+ * kernel AUTO, stream-ordered workspace).  q, k, v: [B, S, H, D] in dtype; out: [B, S, H, D] in
+ * dtype; lse: [B, H, S] fp32.  Requires B, H >= 1, S >= 1, 1 <= D <= 256, n_ring >= 1 dividing S
+ * (2 n_ring dividing S for zigzag), 16-byte aligned pointers. */
+RA_API int ra_forward(const void* q, const void* k, const void* v, void* out, float* lse, int64_t B,
+               int64_t H, int64_t S, int64_t D, int n_ring, int causal, int layout, int dtype,
+               void* stream);
+
+/* ra_forward_ex: ra_forward with explicit options (opt may be NULL for the defaults). */
+RA_API int ra_forward_ex(const void* q, const void* k, const void* v, void* out, float* lse, int64_t B,
+                  int64_t H, int64_t S, int64_t D, int n_ring, int causal, int layout, int dtype,
+                  void* stream, const ra_options* opt);
+
+/* ra_workspace_size: bytes of caller workspace ra_forward_ex needs for these arguments and the
+ * given variant/kernel (enum values as in ra_options), written to *bytes.  Host only. */
+RA_API int ra_workspace_size(int64_t B, int64_t H, int64_t S, int64_t D, int n_ring, int causal,
+                      int layout, int dtype, int variant, int kernel, size_t* bytes);
+
+/* ra_permute: gather x [B, S, H, D] (natural order) into shard-major y [B, n_ring, S_loc, H, D]
+ * where y[b, i, a] = x[b, g(i, a)] under `layout` (the per-shard chunks of the pages' sequence
+ * sharding).  ra_unpermute scatters back: y[b, g(i, a)] = x[b, i, a].  x and y must not overlap.
+ * dtype selects the element size (fp32 or bf16).  Asynchronous on `stream`. */
+RA_API int ra_permute(const void* x, void* y, int64_t B, int64_t S, int64_t H, int64_t D, int n_ring,
+               int layout, int dtype, void* stream);
+RA_API int ra_unpermute(const void* x, void* y, int64_t B, int64_t S, int64_t H, int64_t D, int n_ring,
+                 int layout, int dtype, void* stream);
+
+/* ra_merge_partials: fold one ring step's partial result into the running result, in place:
+ *   lse' = ln(e^{lse_run} + e^{lse_step}),  O' = e^{lse_run - lse'} O_run + e^{lse_step - lse'} O_step
+ * (the merge identities in log-sum-exp form, with each O normalised by its own l).  O_* are fp32
+ * [rows, D], lse_* fp32 [rows]; a row with lse = -inf is empty and contributes nothing.
+ * Exported for callers that drive the per-step path themselves and for tests. */
+RA_API int ra_merge_partials(float* O_run, float* lse_run, const float* O_step, const float* lse_step,
+                      int64_t rows, int64_t D, void* stream);
+
+/* ra_layout_positions (host only): pos[i * S_loc + a] = global position of local token a of
+ * shard i under `layout`.  pos has S entries. */
+RA_API int ra_layout_positions(int64_t S, int n_ring, int layout, int64_t* pos);
+
+/* ra_plan_tiles (host only): classify every (query tile, key/value tile) pair of every
+ * (shard i, ring step s) under the causal mask, as the block-skip scheduler does.
+ * cls has n_ring * n_ring * nqt * nkt entries, nqt = nkt = ceil(S_loc / tile), at index
+ * ((i * n_ring + s) * nqt + qt) * nkt + kt; values 0 = EMPTY (skipped), 1 = FULL (no mask),
+ * 2 = PARTIAL (element mask).  Without causal every pair inside the shard is FULL, except a
+ * ragged last key tile, which is PARTIAL. */
+RA_API int ra_plan_tiles(int64_t S, int n_ring, int layout, int causal, int tile, int8_t* cls);
+
+/* ra_plan_items (host only): the fused kernel's work list, heaviest first (LPT).  Each item is
+ * four int32 (b, h, shard i, query-tile pair p) followed by its cost in live key/value tiles
+ * (int32), 5 entries per item.  Writes at most cap items; *n_items receives the full count. */
+RA_API int ra_plan_items(int64_t B, int64_t H, int64_t S, int n_ring, int causal, int layout,
+                  int32_t* items, int64_t cap, int64_t* n_items);
+
+/* ra_status_string: static description of a status code. */
+RA_API const char* ra_status_string(int status);
+
+/* ra_last_error_string: description of the last RA_ERR_CUDA on the calling host thread. */
+RA_API const char* ra_last_error_string(void);
+
+/* ra_get_device_status: read and clear the status word that the kernels of this library set on
+ * the current device (RA_OK, or RA_ERR_DEVICE_TIMEOUT after a bounded wait ran out).  Call it
+ * after synchronising the stream; it synchronises the device itself. */
+RA_API int ra_get_device_status(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* RA_H */

@@ -1,1 +1,246 @@
-"""Ring Attention exact forward on B200 (placeholder; the binding is added with the library)."""
+"""Ring Attention exact forward on NVIDIA B200 (sm_100a).
+
+A thin ctypes binding over the C ABI of ``include/ra.h`` (``libra_b200.so``, built in-tree by
+``python -m long_context_exact_forward_b200._build``).  Every step of the computation runs in the
+library's CUDA kernels; this module only checks tensor properties and marshals pointers.  PyTorch
+provides device memory and streams.  There is no fallback: if the library is missing or the
+device is not a CUDA device the calls raise.
+
+Entry points (same names as the C ABI):
+    forward(q, k, v, n_ring, causal, layout, ...)   -> (out, lse)      ra_forward_ex
+    workspace_size(...)                              -> int             ra_workspace_size
+    permute(x, n_ring, layout) / unpermute(...)      -> tensor          ra_permute / ra_unpermute
+    merge_partials(O_run, lse_run, O_step, lse_step)                     ra_merge_partials
+    layout_positions(S, n_ring, layout)              -> np.ndarray      ra_layout_positions
+    plan_tiles(S, n_ring, layout, causal, tile)      -> np.ndarray      ra_plan_tiles
+    plan_items(B, H, S, n_ring, causal, layout)      -> np.ndarray      ra_plan_items
+    get_device_status()                              -> int             ra_get_device_status
+"""
+import ctypes
+import os
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libra_b200.so")
+
+LAYOUTS = {"contiguous": 0, "striped": 1, "zigzag": 2}
+VARIANTS = {"auto": 0, "fused": 1, "per_step": 2}
+KERNELS = {"auto": 0, "tc": 1, "simt": 2}
+DEBUG_STALL_LOADS = 1
+
+RA_OK = 0
+STATUS = {
+    0: "RA_OK", -1: "RA_ERR_INVALID_ARG", -2: "RA_ERR_SHAPE", -3: "RA_ERR_ALIGN",
+    -4: "RA_ERR_UNSUPPORTED", -5: "RA_ERR_NO_WORKSPACE", -6: "RA_ERR_CUDA",
+    -7: "RA_ERR_DEVICE_TIMEOUT",
+}
+
+
+class RAError(RuntimeError):
+    def __init__(self, code, where, detail=""):
+        self.code = code
+        name = STATUS.get(code, str(code))
+        super().__init__(f"{where} failed: {name}" + (f" ({detail})" if detail else ""))
+
+
+class Options(ctypes.Structure):
+    _fields_ = [
+        ("variant", ctypes.c_int),
+        ("kernel", ctypes.c_int),
+        ("workspace", ctypes.c_void_p),
+        ("workspace_bytes", ctypes.c_size_t),
+        ("timeout_ns", ctypes.c_uint64),
+        ("debug", ctypes.c_int),
+        ("attn_events", ctypes.c_void_p * 2),
+    ]
+
+
+_lib = None
+
+
+def lib():
+    """The loaded C library (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(
+                f"{LIB_PATH} is missing: build it with `python -m long_context_exact_forward_b200._build`")
+        L = ctypes.CDLL(LIB_PATH)
+        i64, vp, ci = ctypes.c_int64, ctypes.c_void_p, ctypes.c_int
+        L.ra_forward.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i64, ci, ci, ci, ci, vp]
+        L.ra_forward_ex.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i64, ci, ci, ci, ci, vp,
+                                    ctypes.POINTER(Options)]
+        L.ra_workspace_size.argtypes = [i64, i64, i64, i64, ci, ci, ci, ci, ci, ci,
+                                        ctypes.POINTER(ctypes.c_size_t)]
+        L.ra_permute.argtypes = [vp, vp, i64, i64, i64, i64, ci, ci, ci, vp]
+        L.ra_unpermute.argtypes = [vp, vp, i64, i64, i64, i64, ci, ci, ci, vp]
+        L.ra_merge_partials.argtypes = [vp, vp, vp, vp, i64, i64, vp]
+        L.ra_layout_positions.argtypes = [i64, ci, ci, vp]
+        L.ra_plan_tiles.argtypes = [i64, ci, ci, ci, ci, vp]
+        L.ra_plan_items.argtypes = [i64, i64, i64, ci, ci, ci, vp, i64, ctypes.POINTER(ctypes.c_int64)]
+        L.ra_status_string.restype = ctypes.c_char_p
+        L.ra_status_string.argtypes = [ci]
+        L.ra_last_error_string.restype = ctypes.c_char_p
+        L.ra_last_error_string.argtypes = []
+        L.ra_get_device_status.argtypes = []
+        for name in ("ra_forward", "ra_forward_ex", "ra_workspace_size", "ra_permute",
+                     "ra_unpermute", "ra_merge_partials", "ra_layout_positions", "ra_plan_tiles",
+                     "ra_plan_items", "ra_get_device_status"):
+            getattr(L, name).restype = ctypes.c_int
+        _lib = L
+    return _lib
+
+
+def _check(rc, where):
+    if rc != RA_OK:
+        detail = lib().ra_last_error_string().decode() if rc == -6 else ""
+        raise RAError(rc, where, detail)
+
+
+def _torch():
+    import torch
+    return torch
+
+
+def _dtype_code(t):
+    torch = _torch()
+    if t.dtype == torch.float32:
+        return 0
+    if t.dtype == torch.bfloat16:
+        return 1
+    raise TypeError(f"dtype {t.dtype} not supported (float32 or bfloat16)")
+
+
+def _stream_handle(stream):
+    torch = _torch()
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _check_cuda(*ts):
+    for t in ts:
+        if not t.is_cuda:
+            raise ValueError("tensors must live on a CUDA device")
+        if not t.is_contiguous():
+            raise ValueError("tensors must be contiguous")
+
+
+def workspace_size(B, H, S, D, n_ring, causal, layout, dtype_code, variant="auto", kernel="auto"):
+    n = ctypes.c_size_t(0)
+    _check(lib().ra_workspace_size(B, H, S, D, n_ring, int(bool(causal)), LAYOUTS[layout],
+                                   dtype_code, VARIANTS[variant], KERNELS[kernel], ctypes.byref(n)),
+           "ra_workspace_size")
+    return n.value
+
+
+def forward(q, k, v, n_ring, causal=True, layout="contiguous", *, variant="auto", kernel="auto",
+            out=None, lse=None, workspace=None, stream=None, events=None, timeout_ns=0, debug=0):
+    """Exact attention of q, k, v ([B, S, H, D], CUDA, fp32 or bf16) over an n_ring virtual ring.
+
+    Returns (out [B, S, H, D] in q's dtype, lse [B, H, S] fp32).  `workspace` is an optional
+    uint8 CUDA tensor of at least workspace_size(...) bytes (otherwise the library allocates
+    stream-ordered); `events` an optional pair of torch.cuda.Event recorded around the attention
+    kernel launches on `stream`.
+    """
+    torch = _torch()
+    _check_cuda(q, k, v)
+    if q.dim() != 4 or q.shape != k.shape or q.shape != v.shape:
+        raise ValueError("q, k, v must all be [B, S, H, D]")
+    if not (q.dtype == k.dtype == v.dtype):
+        raise TypeError("q, k, v must share a dtype")
+    B, S, H, D = q.shape
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, H, S), dtype=torch.float32, device=q.device)
+    _check_cuda(out, lse)
+    opt = Options()
+    opt.variant = VARIANTS[variant]
+    opt.kernel = KERNELS[kernel]
+    if workspace is not None:
+        _check_cuda(workspace)
+        opt.workspace = workspace.data_ptr()
+        opt.workspace_bytes = workspace.numel() * workspace.element_size()
+    opt.timeout_ns = int(timeout_ns)
+    opt.debug = int(debug)
+    if events is not None:
+        opt.attn_events[0] = events[0].cuda_event
+        opt.attn_events[1] = events[1].cuda_event
+    with torch.cuda.device(q.device):
+        rc = lib().ra_forward_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                                 lse.data_ptr(), B, H, S, D, int(n_ring), int(bool(causal)),
+                                 LAYOUTS[layout], _dtype_code(q), _stream_handle(stream),
+                                 ctypes.byref(opt))
+    _check(rc, "ra_forward_ex")
+    return out, lse
+
+
+def permute(x, n_ring, layout, out=None, stream=None, inverse=False):
+    """Natural order [B, S, H, D] -> shard-major [B, n_ring, S/n_ring, H, D] (or back)."""
+    torch = _torch()
+    _check_cuda(x)
+    B, S, H, D = (x.shape[0], x.shape[1] * x.shape[2], x.shape[3], x.shape[4]) if inverse else x.shape
+    if out is None:
+        out = (torch.empty((B, S, H, D), dtype=x.dtype, device=x.device) if inverse else
+               torch.empty((B, n_ring, S // n_ring, H, D), dtype=x.dtype, device=x.device))
+    fn = lib().ra_unpermute if inverse else lib().ra_permute
+    with torch.cuda.device(x.device):
+        rc = fn(x.data_ptr(), out.data_ptr(), B, S, H, D, int(n_ring), LAYOUTS[layout],
+                _dtype_code(x), _stream_handle(stream))
+    _check(rc, "ra_unpermute" if inverse else "ra_permute")
+    return out
+
+
+def unpermute(x, n_ring, layout, out=None, stream=None):
+    return permute(x, n_ring, layout, out=out, stream=stream, inverse=True)
+
+
+def merge_partials(O_run, lse_run, O_step, lse_step, stream=None):
+    """In-place merge of a step's normalised partial (O_step, lse_step) into (O_run, lse_run)."""
+    torch = _torch()
+    _check_cuda(O_run, lse_run, O_step, lse_step)
+    for t in (O_run, lse_run, O_step, lse_step):
+        if t.dtype != torch.float32:
+            raise TypeError("merge_partials works on fp32 tensors")
+    D = O_run.shape[-1]
+    rows = O_run.numel() // D
+    with torch.cuda.device(O_run.device):
+        rc = lib().ra_merge_partials(O_run.data_ptr(), lse_run.data_ptr(), O_step.data_ptr(),
+                                     lse_step.data_ptr(), rows, D, _stream_handle(stream))
+    _check(rc, "ra_merge_partials")
+    return O_run, lse_run
+
+
+def layout_positions(S, n_ring, layout):
+    pos = np.empty(S, dtype=np.int64)
+    _check(lib().ra_layout_positions(S, n_ring, LAYOUTS[layout], pos.ctypes.data),
+           "ra_layout_positions")
+    return pos.reshape(n_ring, S // n_ring)
+
+
+def plan_tiles(S, n_ring, layout, causal, tile):
+    nt = -(-(S // n_ring) // tile)
+    cls = np.empty((n_ring, n_ring, nt, nt), dtype=np.int8)
+    _check(lib().ra_plan_tiles(S, n_ring, LAYOUTS[layout], int(bool(causal)), tile,
+                               cls.ctypes.data), "ra_plan_tiles")
+    return cls
+
+
+def plan_items(B, H, S, n_ring, causal, layout):
+    n = ctypes.c_int64(0)
+    _check(lib().ra_plan_items(B, H, S, n_ring, int(bool(causal)), LAYOUTS[layout], None, 0,
+                               ctypes.byref(n)), "ra_plan_items")
+    items = np.empty((n.value, 5), dtype=np.int32)
+    _check(lib().ra_plan_items(B, H, S, n_ring, int(bool(causal)), LAYOUTS[layout],
+                               items.ctypes.data, n.value, ctypes.byref(n)), "ra_plan_items")
+    return items
+
+
+def get_device_status():
+    return lib().ra_get_device_status()
+
+
+def status_string(code):
+    return lib().ra_status_string(code).decode()

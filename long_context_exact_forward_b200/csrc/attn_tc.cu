@@ -1,0 +1,545 @@
+// attn_tc.cu -- ring-order blockwise attention on the sm_100a tensor cores (tcgen05 + TMEM + TMA).
+//
+// What it computes.  For each work item (batch b, head h, shard i, a pair of 128-row query tiles)
+// the kernel walks the ring steps s in [s_begin, s_end); at step s it meets the key/value block of
+// shard j = (i - s) mod N (ultralytics.com "Ring Attention" toy loop; jisaku.com 処理フロー) and
+// for every live 128-key tile of that block it computes
+//     S = Q_i K_j^T                         (tcgen05.mma, bf16 x bf16 -> fp32 in TMEM)
+//     m' = max(m, rowmax(S) / sqrt(D));  P = exp(S / sqrt(D) - m')     (softmax warps)
+//     l  = e^{m - m'} l + rowsum(P);     O = e^{m - m'} O + P V_j      (tcgen05.mma, P from TMEM)
+// i.e. the online-softmax identities of troisinh.com "Ring Attention" ("Tai sao no hoat dong"),
+// applied tile by tile and step by step, so that the merge across ring steps (the in-kernel form
+// of the pages' per-device accumulation) never leaves the chip.  At the end O / l and
+// lse = m + ln l are written, either as the final result in natural token order or as one ring
+// step's partial result (per-step variant).
+//
+// The causal mask is applied on original token positions.  Because every layout keeps positions
+// increasing within a shard, a query row sees a prefix of each key block; key tiles past the
+// longest prefix of the query tile are never loaded (block skip), tiles inside every row's prefix
+// run unmasked, and only the tile holding a row's prefix end is masked.
+//
+// Layout of one CTA (384 threads, one CTA per SM, persistent over a static slice of the work list):
+//   warps 0-3  softmax for query tile 0 (thread t owns row t = TMEM lane t)
+//   warps 4-7  softmax for query tile 1
+//   warp  8    TMA producer: Q tiles, then K and V tiles into a ring of 4 shared-memory slots
+//   warp  9    MMA issuer (one thread) and TMEM owner
+//   warps 10-11 idle
+// TMEM (512 columns): S0 [0,128), S1 [128,256), O0 [256,256+D), O1 [384,384+D).  P (bf16) is
+// written over the first 64 columns of its S tile and read from there by the P V MMA.
+// The MMA order per key tile t is  P0V(t), S0(t+1), P1V(t), S1(t+1), so each query tile's softmax
+// overlaps the other tile's MMAs.  Because S0(t+1) is issued after P0V(t), the completion of
+// S0(t+1) also proves P0V(t) is done, which lets the softmax warps rescale O in place.
+// Rescaling of O is lazy: it happens only when a row's max grows by more than 2^8.
+//
+// Every wait is bounded (timeout_ns); on give-up the CTA records RA_ERR_DEVICE_TIMEOUT in the
+// status word, lets its own copies and MMAs drain (again bounded), frees TMEM and exits.
+#include <cuda_bf16.h>
+
+#include "ra.h"
+#include "ra_internal.cuh"
+#include "sm100.cuh"
+
+namespace ra {
+namespace {
+using namespace sm100;
+
+constexpr int kM = 128;           // query rows per tile
+constexpr int kN = 128;           // keys per tile
+constexpr int kSlots = 4;         // K/V tile slots
+constexpr int kThreads = 384;
+constexpr int kLoadWarp = 8;
+constexpr int kMmaWarp = 9;
+constexpr uint32_t kTmemCols = 512;
+constexpr float kRescaleLog2 = 8.0f;  // lazy-rescale threshold (log2 units)
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+constexpr uint32_t kNegInfBits = 0xff800000u;
+constexpr int kColBlockBytes = 128 * 128;  // one 128-row x 64-element bf16 block (128-B rows)
+
+template <int kD>
+struct TcSmem {
+    static constexpr int kTileBytes = kM * kD * 2;
+    uint8_t q[2][kTileBytes];         // each tile: kD/64 column blocks of 128 rows x 128 B
+    uint8_t kv[kSlots][kTileBytes];
+    uint64_t q_full, q_empty, drain;
+    uint64_t slot_full[kSlots], slot_empty[kSlots];
+    uint64_t s_full[2], p_full[2], o_final[2], o_free[2];
+    uint32_t tmem_base;
+    int abort;
+};
+
+__device__ __forceinline__ uint32_t s_col(int q) { return (uint32_t)q * 128u; }
+template <int kD>
+__device__ __forceinline__ uint32_t o_col(int q) { return 256u + (uint32_t)q * 128u; }
+
+struct ItemGeom {
+    int64_t b, h, i;
+    int64_t a0[2];    // first local row of each query tile
+    int64_t last[2];  // last valid local row of each query tile (clamped to the shard)
+};
+
+__device__ __forceinline__ ItemGeom item_geom(const AttnArgs& A, int4 it) {
+    ItemGeom G;
+    G.b = it.x;
+    G.h = it.y;
+    G.i = it.z;
+    for (int q = 0; q < 2; ++q) {
+        G.a0[q] = (int64_t)it.w * 2 * kM + q * kM;
+        const int64_t e = G.a0[q] + kM - 1;
+        G.last[q] = e < A.L.S_loc - 1 ? e : A.L.S_loc - 1;
+    }
+    return G;
+}
+
+// Live key tiles of block j for query tile q (0 if the tile lies past the shard end).
+__device__ __forceinline__ int tiles_for(const AttnArgs& A, const ItemGeom& G, int q, int64_t j) {
+    if (G.a0[q] >= A.L.S_loc) return 0;
+    const int64_t n = visible_keys(A.L, A.causal, G.i, G.last[q], j);
+    return (int)((n + kN - 1) / kN);
+}
+
+// Flat sequence of (step, key tile) pairs of one item, skipping dead steps.
+struct TileIter {
+    int s, s_end, kt, nt0, nt1;
+    int64_t j;
+    bool valid;
+    __device__ __forceinline__ void load_step(const AttnArgs& A, const ItemGeom& G) {
+        for (; s < s_end; ++s) {
+            j = ring_block(G.i, s, A.L.N);
+            nt0 = tiles_for(A, G, 0, j);
+            nt1 = tiles_for(A, G, 1, j);
+            if (nt0 > 0 || nt1 > 0) {
+                valid = true;
+                return;
+            }
+        }
+        valid = false;
+    }
+    __device__ __forceinline__ void init(const AttnArgs& A, const ItemGeom& G) {
+        s = A.s_begin;
+        s_end = A.s_end;
+        kt = 0;
+        load_step(A, G);
+    }
+    __device__ __forceinline__ void next(const AttnArgs& A, const ItemGeom& G) {
+        if (++kt >= (nt0 > nt1 ? nt0 : nt1)) {
+            kt = 0;
+            ++s;
+            load_step(A, G);
+        }
+    }
+    __device__ __forceinline__ bool act(int q) const { return kt < (q ? nt1 : nt0); }
+};
+
+__device__ __forceinline__ void give_up(volatile int* abort, int* status) {
+    *abort = 1;
+    atomicExch(status, RA_ERR_DEVICE_TIMEOUT);
+}
+
+// Order uses of r[] after the asynchronous TMEM load has landed.
+__device__ __forceinline__ void tmem_wait_ld_regs(uint32_t (&r)[32]) {
+    asm volatile("tcgen05.wait::ld.sync.aligned;"
+                 : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]),
+                   "+r"(r[6]), "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]),
+                   "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15]), "+r"(r[16]), "+r"(r[17]),
+                   "+r"(r[18]), "+r"(r[19]), "+r"(r[20]), "+r"(r[21]), "+r"(r[22]), "+r"(r[23]),
+                   "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]), "+r"(r[29]),
+                   "+r"(r[30]), "+r"(r[31])
+                 :
+                 : "memory");
+}
+
+template <int kD>
+struct Roles {
+    TcSmem<kD>& sm;
+    const AttnArgs& A;
+    const int4* __restrict__ items;
+    int n_items;
+    uint64_t timeout;
+    int* status;
+    volatile int* abort;
+    uint32_t tmem;
+
+    // ------------------------------------------------------------ TMA producer (one thread)
+    __device__ void producer(const CUtensorMap* tm_q, const CUtensorMap* tm_k,
+                             const CUtensorMap* tm_v, int debug) {
+        uint32_t slot_it = 0, q_it = 0;
+        bool ok = true;
+        for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
+            const ItemGeom G = item_geom(A, items[it]);
+            TileIter t;
+            t.init(A, G);
+            if (!t.valid) continue;
+            if (debug == RA_DEBUG_STALL_LOADS) continue;  // consumers must time out
+            if (!mbar_wait(&sm.q_empty, (q_it & 1) ^ 1, timeout, abort)) { ok = false; break; }
+            mbar_arrive_expect_tx(&sm.q_full, 2 * TcSmem<kD>::kTileBytes);
+            for (int q = 0; q < 2; ++q)
+                for (int cb = 0; cb < kD / 64; ++cb)
+                    tma_load_5d(sm.q[q] + cb * kColBlockBytes, tm_q, &sm.q_full, cb * 64, (int)G.h,
+                                (int)G.a0[q], (int)G.i, (int)G.b);
+            ++q_it;
+            for (; t.valid && ok; t.next(A, G)) {
+                for (int w = 0; w < 2; ++w) {  // K then V of this tile
+                    const uint32_t slot = slot_it % kSlots;
+                    if (!mbar_wait(&sm.slot_empty[slot], ((slot_it / kSlots) & 1) ^ 1, timeout, abort)) {
+                        ok = false;
+                        break;
+                    }
+                    mbar_arrive_expect_tx(&sm.slot_full[slot], TcSmem<kD>::kTileBytes);
+                    for (int cb = 0; cb < kD / 64; ++cb)
+                        tma_load_5d(sm.kv[slot] + cb * kColBlockBytes, w ? tm_v : tm_k,
+                                    &sm.slot_full[slot], cb * 64, (int)G.h, t.kt * kN, (int)t.j,
+                                    (int)G.b);
+                    ++slot_it;
+                }
+            }
+        }
+        if (!ok) {
+            give_up(abort, status);
+            // let the copies already issued land before the CTA can exit
+            const uint32_t first = slot_it > kSlots ? slot_it - kSlots : 0;
+            for (uint32_t x = first; x < slot_it; ++x)
+                mbar_wait(&sm.slot_full[x % kSlots], (x / kSlots) & 1, timeout, nullptr);
+            if (q_it > 0) mbar_wait(&sm.q_full, (q_it - 1) & 1, timeout, nullptr);
+        }
+    }
+
+    // ------------------------------------------------------------ MMA issuer (one thread)
+    __device__ void issue_s(int q, uint32_t kslot) {
+        constexpr uint32_t idesc = idesc_bf16_f32(kM, kN, 0, 0);
+        const uint32_t qa = smem_addr(sm.q[q]), ka = smem_addr(sm.kv[kslot]);
+#pragma unroll
+        for (int kk = 0; kk < kD / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * kColBlockBytes + (kk & 3) * 32;
+            mma_ss(tmem + s_col(q), smem_desc_sw128(qa + off, 16, 1024),
+                   smem_desc_sw128(ka + off, 16, 1024), idesc, kk > 0);
+        }
+        mma_commit(&sm.s_full[q]);
+    }
+
+    __device__ void issue_pv(int q, uint32_t vslot, bool accumulate) {
+        constexpr uint32_t idesc = idesc_bf16_f32(kM, kD, 0, 1);  // V is MN-major (D fastest)
+        const uint32_t va = smem_addr(sm.kv[vslot]);
+#pragma unroll
+        for (int kk = 0; kk < kN / 16; ++kk) {
+            // 16 keys = 16 rows of 128 B of every column block; P: 16 bf16 = 8 TMEM columns
+            mma_ts(tmem + o_col<kD>(q), tmem + s_col(q) + kk * 8,
+                   smem_desc_sw128(va + kk * 16 * 128, kColBlockBytes, 1024), idesc,
+                   (kk > 0 || accumulate) ? 1u : 0u);
+        }
+    }
+
+    __device__ void mma() {
+        uint32_t cons_it = 0, q_it = 0, p_cnt[2] = {0, 0}, act_items[2] = {0, 0};
+        bool ok = true;
+        auto wait = [&](uint64_t* bar, uint32_t parity) {
+            if (!ok) return false;
+            ok = mbar_wait(bar, parity, timeout, abort);
+            if (ok) tc_fence_after();
+            return ok;
+        };
+        for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
+            const ItemGeom G = item_geom(A, items[it]);
+            TileIter cur;
+            cur.init(A, G);
+            if (!cur.valid) continue;
+            if (!wait(&sm.q_full, q_it & 1)) break;
+            ++q_it;
+            bool first_pv[2] = {true, true}, any_act[2] = {false, false};
+            uint32_t kslot = cons_it % kSlots;
+            if (!wait(&sm.slot_full[kslot], (cons_it / kSlots) & 1)) break;
+            ++cons_it;
+            for (int q = 0; q < 2; ++q)
+                if (cur.act(q)) {
+                    issue_s(q, kslot);
+                    any_act[q] = true;
+                }
+            mma_commit(&sm.slot_empty[kslot]);
+            TileIter nxt = cur;
+            nxt.next(A, G);
+            if (!nxt.valid) mma_commit(&sm.q_empty);
+            for (;;) {
+                const uint32_t vslot = cons_it % kSlots;
+                if (!wait(&sm.slot_full[vslot], (cons_it / kSlots) & 1)) break;
+                ++cons_it;
+                for (int q = 0; q < 2; ++q) {
+                    if (cur.act(q)) {
+                        if (!wait(&sm.p_full[q], p_cnt[q] & 1)) break;
+                        ++p_cnt[q];
+                        if (first_pv[q] && act_items[q] > 0 &&
+                            !wait(&sm.o_free[q], (act_items[q] - 1) & 1))
+                            break;
+                        issue_pv(q, vslot, !first_pv[q]);
+                        first_pv[q] = false;
+                    }
+                    if (q == 0 && nxt.valid) {
+                        kslot = cons_it % kSlots;
+                        if (!wait(&sm.slot_full[kslot], (cons_it / kSlots) & 1)) break;
+                        ++cons_it;
+                        if (nxt.act(0)) {
+                            issue_s(0, kslot);
+                            any_act[0] = true;
+                        }
+                    }
+                }
+                if (!ok) break;
+                mma_commit(&sm.slot_empty[vslot]);
+                if (!nxt.valid) break;
+                if (nxt.act(1)) {
+                    issue_s(1, kslot);
+                    any_act[1] = true;
+                }
+                mma_commit(&sm.slot_empty[kslot]);
+                cur = nxt;
+                nxt.next(A, G);
+                if (!nxt.valid) mma_commit(&sm.q_empty);
+            }
+            if (!ok) break;
+            for (int q = 0; q < 2; ++q)
+                if (any_act[q]) {
+                    mma_commit(&sm.o_final[q]);
+                    ++act_items[q];
+                }
+        }
+        if (!ok) {
+            give_up(abort, status);
+            mma_commit(&sm.drain);  // every MMA issued so far has finished once this arrives
+            mbar_wait(&sm.drain, 0, timeout, nullptr);
+        }
+    }
+
+    // ------------------------------------------------------------ softmax + epilogue (128 threads per tile)
+    __device__ void softmax(int q, int warp, int row) {
+        const uint32_t lane_base = tmem + ((uint32_t)((warp & 3) * 32) << 16);
+        const uint32_t tS = lane_base + s_col(q), tO = lane_base + o_col<kD>(q);
+        const float sl2 = A.scale * kLog2e;
+        uint32_t s_cnt = 0, items_act = 0;
+        bool ok = true;
+        auto wait_all = [&](uint64_t* bar, uint32_t parity) {
+            bool w = mbar_wait(bar, parity, timeout, abort);
+            ok = __all_sync(0xffffffffu, w);
+            if (ok) tc_fence_after();
+            return ok;
+        };
+        for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
+            const ItemGeom G = item_geom(A, items[it]);
+            const int64_t a = G.a0[q] + row;
+            float m_run = -INFINITY, l = 0.f;
+            int n_act = 0;
+            for (int s = A.s_begin; s < A.s_end && ok; ++s) {
+                const int64_t j = ring_block(G.i, s, A.L.N);
+                const int nt = tiles_for(A, G, q, j);
+                if (nt == 0) continue;
+                const int64_t cnt = visible_keys(A.L, A.causal, G.i, a, j);
+                for (int kt = 0; kt < nt; ++kt) {
+                    if (!wait_all(&sm.s_full[q], s_cnt & 1)) break;
+                    ++s_cnt;
+                    uint32_t r[128];
+#pragma unroll
+                    for (int c = 0; c < 4; ++c)
+                        tmem_ld32(tS + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&r[c * 32]));
+#pragma unroll
+                    for (int c = 0; c < 4; ++c)
+                        tmem_wait_ld_regs(*reinterpret_cast<uint32_t(*)[32]>(&r[c * 32]));
+                    const int64_t valid = cnt - (int64_t)kt * kN;
+                    if (valid < kN) {
+#pragma unroll
+                        for (int c = 0; c < kN; ++c)
+                            if (c >= valid) r[c] = kNegInfBits;
+                    }
+                    float mx0 = -INFINITY, mx1 = -INFINITY;
+#pragma unroll
+                    for (int c = 0; c < kN; c += 2) {
+                        mx0 = fmaxf(mx0, __uint_as_float(r[c]));
+                        mx1 = fmaxf(mx1, __uint_as_float(r[c + 1]));
+                    }
+                    const float m_new = fmaxf(m_run, fmaxf(mx0, mx1) * sl2);
+                    bool rescale = false;
+                    float alpha = 1.f;
+                    if (n_act == 0) {
+                        m_run = m_new;
+                    } else if (m_new > m_run + kRescaleLog2) {
+                        alpha = ex2(m_run - m_new);
+                        rescale = true;
+                        l *= alpha;
+                        m_run = m_new;
+                    }
+                    const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
+                    float l0 = 0.f, l1 = 0.f;
+#pragma unroll
+                    for (int c4 = 0; c4 < 4; ++c4) {
+                        uint32_t pk[16];
+#pragma unroll
+                        for (int x = 0; x < 16; ++x) {
+                            const float p0 = ex2(fmaf(__uint_as_float(r[c4 * 32 + 2 * x]), sl2, -m_use));
+                            const float p1 = ex2(fmaf(__uint_as_float(r[c4 * 32 + 2 * x + 1]), sl2, -m_use));
+                            l0 += p0;
+                            l1 += p1;
+                            pk[x] = pack_bf16x2(p0, p1);
+                        }
+                        tmem_st16(tS + c4 * 16, pk);
+                    }
+                    l += l0 + l1;
+                    if (__any_sync(0xffffffffu, rescale)) {
+#pragma unroll 1
+                        for (int c = 0; c < kD / 32; ++c) {
+                            uint32_t o[32];
+                            tmem_ld32(tO + c * 32, o);
+                            tmem_wait_ld_regs(o);
+#pragma unroll
+                            for (int x = 0; x < 32; ++x) o[x] = __float_as_uint(__uint_as_float(o[x]) * alpha);
+                            tmem_st32(tO + c * 32, o);
+                        }
+                    }
+                    tmem_wait_st();
+                    tc_fence_before();
+                    mbar_arrive(&sm.p_full[q]);
+                    ++n_act;
+                }
+            }
+            if (!ok) break;
+            epilogue(q, G, a, n_act, m_run, l, tO, ok, wait_all, items_act);
+        }
+        if (!ok) give_up(abort, status);
+    }
+
+    template <typename Wait>
+    __device__ void epilogue(int q, const ItemGeom& G, int64_t a, int n_act, float m_run, float l,
+                             uint32_t tO, bool& ok, Wait& wait_all, uint32_t& items_act) {
+        const bool row_ok = a < A.L.S_loc;
+        const float inv_l = l > 0.f ? 1.f / l : 0.f;
+        const float lse = l > 0.f ? (m_run + log2f(l)) * kLn2 : -INFINITY;
+        const int64_t H = A.H, S = A.L.S;
+        float* lse_dst;
+        uint8_t* row_dst;
+        if (A.out_mode == kOutFinal) {
+            const int64_t g = row_ok ? global_position(A.L, G.i, a) : 0;
+            row_dst = static_cast<uint8_t*>(A.out) + (((G.b * S + g) * H + G.h) * kD) * 2;
+            lse_dst = A.lse + (G.b * H + G.h) * S + g;
+        } else {
+            const int64_t rr = ((G.b * A.L.N + G.i) * A.L.S_loc + a) * H + G.h;
+            row_dst = static_cast<uint8_t*>(A.out) + rr * kD * 4;
+            lse_dst = A.lse + rr;
+        }
+        if (n_act > 0) {
+            if (!wait_all(&sm.o_final[q], items_act & 1)) return;
+            ++items_act;
+#pragma unroll 1
+            for (int c = 0; c < kD / 32; ++c) {
+                uint32_t o[32];
+                tmem_ld32(tO + c * 32, o);
+                tmem_wait_ld_regs(o);
+                if (row_ok) store_chunk(row_dst, c, o, inv_l);
+            }
+            tc_fence_before();
+            mbar_arrive(&sm.o_free[q]);
+        } else if (row_ok) {
+            uint32_t o[32];
+#pragma unroll
+            for (int x = 0; x < 32; ++x) o[x] = 0u;
+            for (int c = 0; c < kD / 32; ++c) store_chunk(row_dst, c, o, 0.f);
+        }
+        if (row_ok) *lse_dst = lse;
+    }
+
+    __device__ __forceinline__ void store_chunk(uint8_t* row_dst, int c, const uint32_t (&o)[32],
+                                                float inv_l) {
+        if (A.out_mode == kOutFinal) {  // bf16, 32 values = 64 bytes
+            uint4* dst = reinterpret_cast<uint4*>(row_dst + c * 64);
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {
+                uint4 u;
+                u.x = pack_bf16x2(__uint_as_float(o[8 * v + 0]) * inv_l, __uint_as_float(o[8 * v + 1]) * inv_l);
+                u.y = pack_bf16x2(__uint_as_float(o[8 * v + 2]) * inv_l, __uint_as_float(o[8 * v + 3]) * inv_l);
+                u.z = pack_bf16x2(__uint_as_float(o[8 * v + 4]) * inv_l, __uint_as_float(o[8 * v + 5]) * inv_l);
+                u.w = pack_bf16x2(__uint_as_float(o[8 * v + 6]) * inv_l, __uint_as_float(o[8 * v + 7]) * inv_l);
+                dst[v] = u;
+            }
+        } else {  // fp32, 32 values = 128 bytes
+            float4* dst = reinterpret_cast<float4*>(row_dst + c * 128);
+#pragma unroll
+            for (int v = 0; v < 8; ++v)
+                dst[v] = make_float4(__uint_as_float(o[4 * v + 0]) * inv_l, __uint_as_float(o[4 * v + 1]) * inv_l,
+                                     __uint_as_float(o[4 * v + 2]) * inv_l, __uint_as_float(o[4 * v + 3]) * inv_l);
+        }
+    }
+};
+
+template <int kD>
+__global__ void __launch_bounds__(kThreads, 1)
+    attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                   const __grid_constant__ CUtensorMap tm_v, const AttnArgs A,
+                   const int4* __restrict__ items, int n_items, uint64_t timeout_ns, int debug,
+                   int* status) {
+    extern __shared__ uint8_t smem_raw[];
+    TcSmem<kD>& sm = *reinterpret_cast<TcSmem<kD>*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        mbar_init(&sm.q_full, 1);
+        mbar_init(&sm.q_empty, 1);
+        mbar_init(&sm.drain, 1);
+        for (int k = 0; k < kSlots; ++k) {
+            mbar_init(&sm.slot_full[k], 1);
+            mbar_init(&sm.slot_empty[k], 1);
+        }
+        for (int q = 0; q < 2; ++q) {
+            mbar_init(&sm.s_full[q], 1);
+            mbar_init(&sm.p_full[q], kM);
+            mbar_init(&sm.o_final[q], 1);
+            mbar_init(&sm.o_free[q], kM);
+        }
+        sm.abort = 0;
+        fence_barrier_init();
+    }
+    if (warp == kLoadWarp && lane == 0) {
+        tma_prefetch_desc(&tm_q);
+        tma_prefetch_desc(&tm_k);
+        tma_prefetch_desc(&tm_v);
+    }
+    if (warp == kMmaWarp) {
+        tmem_alloc(&sm.tmem_base, kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+
+    Roles<kD> roles{sm, A, items, n_items, timeout_ns, status, &sm.abort, sm.tmem_base};
+    if (warp == kLoadWarp) {
+        if (lane == 0) roles.producer(&tm_q, &tm_k, &tm_v, debug);
+        __syncwarp();
+    } else if (warp == kMmaWarp) {
+        if (lane == 0) roles.mma();
+        __syncwarp();
+    } else if (warp < 8) {
+        roles.softmax(warp >> 2, warp, threadIdx.x & 127);
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == kMmaWarp) {
+        tc_fence_after();
+        tmem_dealloc(sm.tmem_base, kTmemCols);
+    }
+}
+
+}  // namespace
+
+size_t tc_smem_bytes(int64_t D) {
+    return (D == 64 ? sizeof(TcSmem<64>) : sizeof(TcSmem<128>)) + 1024;
+}
+
+cudaError_t launch_attn_tc(const AttnArgs& a, const TcLaunch& t, cudaStream_t stream) {
+    if (t.n_items == 0) return cudaSuccess;
+    const size_t smem = tc_smem_bytes(a.D);
+    auto kern = (a.D == 64) ? attn_tc_kernel<64> : attn_tc_kernel<128>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    kern<<<t.grid, kThreads, smem, stream>>>(t.tm_q, t.tm_k, t.tm_v, a, t.items, t.n_items,
+                                             t.timeout_ns, t.debug, t.status);
+    return cudaGetLastError();
+}
+
+}  // namespace ra

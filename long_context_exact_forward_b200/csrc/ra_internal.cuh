@@ -1,0 +1,59 @@
+// ra_internal.cuh -- parameter blocks and launcher declarations shared by the library's .cu files.
+#pragma once
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "layout.cuh"
+
+namespace ra {
+
+// Where an attention launch puts its result.
+//   kOutFinal:   normalised O in the input dtype at natural position g(i, a), lse natural [B, H, S].
+//   kOutPartial: normalised O_s fp32 and lse_s fp32, both in shard-major row order
+//                row = ((b * N + i) * S_loc + a) * H + h  (O_s [rows, D], lse_s [rows]).
+enum OutMode { kOutFinal = 0, kOutPartial = 1 };
+
+struct AttnArgs {
+    Layout L;
+    int64_t B, H, D;
+    int causal;
+    int dtype;            // RA_DTYPE_*
+    int s_begin, s_end;   // ring steps walked: s in [s_begin, s_end), block j = (i - s) mod N
+    int out_mode;         // OutMode
+    void* out;            // kOutFinal: [B, S, H, D] dtype; kOutPartial: fp32 [rows, D]
+    float* lse;           // kOutFinal: [B, H, S]; kOutPartial: [rows]
+    float scale;          // 1 / sqrt(D)
+};
+
+// permute.cu
+cudaError_t launch_permute(const void* const* src, void* const* dst, int n_tensors, int64_t B,
+                           const Layout& L, int64_t H, int64_t D, int esize, bool inverse,
+                           cudaStream_t stream);
+
+// merge.cu: fold (O_s, lse_s) into (O_r, lse_r) in place, or (final) write the merged result
+// to out (natural order, dtype) and lse natural [B, H, S].
+cudaError_t launch_merge_inplace(float* O_r, float* lse_r, const float* O_s, const float* lse_s,
+                                 int64_t rows, int64_t D, cudaStream_t stream);
+cudaError_t launch_merge_final(const float* O_r, const float* lse_r, const float* O_s,
+                               const float* lse_s, void* out, float* lse, int dtype, int64_t B,
+                               const Layout& L, int64_t H, int64_t D, cudaStream_t stream);
+
+// attn_simt.cu: CUDA-core attention over natural-order q, k, v (any layout, D <= 256).
+cudaError_t launch_attn_simt(const void* q, const void* k, const void* v, const AttnArgs& a,
+                             cudaStream_t stream);
+
+// attn_tc.cu: tcgen05 attention over shard-major bf16 q, k, v (D in {64, 128}).
+struct TcLaunch {
+    CUtensorMap tm_q, tm_k, tm_v;
+    const int4* items;     // work list (b, h, i, pair), heaviest first
+    int n_items;
+    int grid;
+    uint64_t timeout_ns;
+    int debug;
+    int* status;           // device status word, set to RA_ERR_DEVICE_TIMEOUT on a give-up
+};
+size_t tc_smem_bytes(int64_t D);
+cudaError_t launch_attn_tc(const AttnArgs& a, const TcLaunch& t, cudaStream_t stream);
+
+}  // namespace ra

@@ -1,0 +1,79 @@
+"""C-ABI checks that need no GPU: the library loads, exports what include/ra.h declares, and
+rejects bad arguments before touching the device."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import long_context_exact_forward_b200 as ra
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "ra.h")
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"RA_API\s+[\w\s\*]+?\b(ra_\w+)\s*\(", text)))
+
+
+def test_library_exports_every_declared_symbol():
+    names = declared_symbols()
+    assert "ra_forward" in names and "ra_forward_ex" in names and len(names) >= 12
+    lib = ctypes.CDLL(ra.LIB_PATH)
+    for n in names:
+        assert hasattr(lib, n), f"{n} declared in ra.h but not exported"
+
+
+def test_status_strings():
+    for code in (0, -1, -2, -3, -4, -5, -6, -7):
+        assert ra.status_string(code) and ra.status_string(code) != "unknown status"
+    assert ra.status_string(12345) == "unknown status"
+
+
+FAKE = 0x100000  # 16-byte aligned, never dereferenced: validation fails first
+
+
+def call(B=1, H=2, S=64, D=16, n_ring=4, causal=1, layout=0, dtype=0, q=FAKE, k=FAKE, v=FAKE,
+         out=FAKE, lse=FAKE, variant=0, kernel=0):
+    opt = ra.Options()
+    opt.variant = variant
+    opt.kernel = kernel
+    return ra.lib().ra_forward_ex(q, k, v, out, lse, B, H, S, D, n_ring, causal, layout, dtype,
+                                  None, ctypes.byref(opt))
+
+
+@pytest.mark.parametrize("kw, code", [
+    (dict(S=63), -2),                    # S % n_ring
+    (dict(S=68, layout=2), -2),          # zigzag needs S % 2N
+    (dict(D=300), -2),                   # head dim above 256
+    (dict(D=0), -1),
+    (dict(B=0), -1),
+    (dict(n_ring=0), -1),
+    (dict(layout=3), -1),
+    (dict(dtype=5), -1),
+    (dict(q=0), -1),
+    (dict(lse=0), -1),
+    (dict(k=FAKE + 8), -3),              # misaligned tensor
+    (dict(variant=7), -1),
+])
+def test_validation_rejects_before_any_cuda_call(kw, code):
+    assert call(**kw) == code
+
+
+def test_workspace_size_grows_with_per_step_and_permute():
+    args = dict(B=1, H=4, S=4096, D=128, n_ring=4, causal=True, dtype_code=1)
+    fused_contig = ra.workspace_size(layout="contiguous", variant="fused", **args)
+    fused_striped = ra.workspace_size(layout="striped", variant="fused", **args)
+    per_step = ra.workspace_size(layout="contiguous", variant="per_step", **args)
+    elems = 1 * 4096 * 4 * 128
+    assert fused_striped >= fused_contig + 3 * elems * 2          # permuted q, k, v
+    assert per_step >= fused_contig + 2 * elems * 4               # running and step partials
+    simt = ra.workspace_size(layout="striped", variant="fused", kernel="simt", **args)
+    assert simt <= fused_contig                                   # SIMT reads natural order
+
+
+def test_workspace_size_rejects_bad_shape():
+    with pytest.raises(ra.RAError):
+        ra.workspace_size(1, 1, 10, 16, 3, False, "contiguous", 0)

@@ -1,0 +1,101 @@
+"""The host-side planner (layout maps, causal block-skip tile classes, LPT work list) checked on
+the CPU against brute force over the oracle's independent layout positions."""
+import numpy as np
+import pytest
+
+import long_context_exact_forward_b200 as ra
+import oracle
+
+LAYOUT_CASES = [(48, 4, "contiguous"), (48, 4, "striped"), (48, 4, "zigzag"), (40, 5, "contiguous"),
+                (40, 5, "striped"), (60, 3, "zigzag"), (7, 1, "contiguous"), (1024, 8, "zigzag")]
+
+
+@pytest.mark.parametrize("S, N, layout", LAYOUT_CASES)
+def test_layout_positions_match_oracle(S, N, layout):
+    np.testing.assert_array_equal(ra.layout_positions(S, N, layout), oracle.layout_positions(S, N, layout))
+
+
+@pytest.mark.parametrize("S, N, layout", LAYOUT_CASES)
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("tile", [1, 3, 4, 8, 64])
+def test_tile_classes_are_exact(S, N, layout, causal, tile):
+    if S > 100 and tile < 8:
+        pytest.skip("large case runs with wide tiles only")
+    pos = oracle.layout_positions(S, N, layout)
+    S_loc = S // N
+    nt = -(-S_loc // tile)
+    cls = ra.plan_tiles(S, N, layout, causal, tile)
+    assert cls.shape == (N, N, nt, nt)
+    covered = np.zeros((S, S), dtype=np.int64)
+    for i in range(N):
+        for s in range(N):
+            j = (i - s) % N
+            for qt in range(nt):
+                qa = np.arange(qt * tile, min((qt + 1) * tile, S_loc))
+                for kt in range(nt):
+                    ka = np.arange(kt * tile, (kt + 1) * tile)
+                    inside = ka < S_loc
+                    gq = pos[i, qa][:, None]
+                    gk = np.where(inside, pos[j, np.minimum(ka, S_loc - 1)], S + 1)[None, :]
+                    allowed = (gk <= gq) if causal else np.broadcast_to(inside[None, :], (qa.size, ka.size))
+                    allowed = allowed & inside[None, :]
+                    c = cls[i, s, qt, kt]
+                    if c == 0:
+                        assert not allowed.any(), "EMPTY tile holds an allowed pair"
+                    elif c == 1:
+                        assert allowed.all(), "FULL tile holds a masked pair"
+                    else:
+                        assert c == 2 and allowed.any() and not allowed.all()
+                    gqs = np.broadcast_to(gq, allowed.shape)[allowed]
+                    gks = np.broadcast_to(gk, allowed.shape)[allowed]
+                    np.add.at(covered, (gqs, gks), 1)
+    want = np.tril(np.ones((S, S), dtype=np.int64)) if causal else np.ones((S, S), dtype=np.int64)
+    np.testing.assert_array_equal(covered, want)  # every allowed pair exactly once
+
+
+@pytest.mark.parametrize("layout", ["contiguous", "striped", "zigzag"])
+@pytest.mark.parametrize("causal", [False, True])
+def test_work_list_covers_every_item_once_heaviest_first(layout, causal):
+    B, H, N, S_loc = 2, 3, 4, 640  # 640 = 2.5 pairs of 256 rows: a ragged last pair
+    S = N * S_loc
+    items = ra.plan_items(B, H, S, N, causal, layout)
+    pairs = -(-S_loc // 256)
+    assert items.shape == (B * H * N * pairs, 5)
+    keys = {tuple(r[:4]) for r in items.tolist()}
+    assert keys == {(b, h, i, p) for b in range(B) for h in range(H) for i in range(N) for p in range(pairs)}
+    # (b, h) major, heaviest first inside a head
+    bh = items[:, 0] * H + items[:, 1]
+    assert (np.diff(bh) >= 0).all()
+    for g in range(B * H):
+        cost = items[bh == g, 4]
+        assert (np.diff(cost) <= 0).all()
+    # cost = live (128-row query tile, 128-key tile) pairs, from the oracle's positions
+    pos = oracle.layout_positions(S, N, layout)
+    for b, h, i, p, cost in items[:N * pairs].tolist():
+        want = 0
+        for q in range(2):
+            a0 = p * 256 + q * 128
+            if a0 >= S_loc:
+                continue
+            last = min(a0 + 127, S_loc - 1)
+            for s in range(N):
+                j = (i - s) % N
+                n_vis = int((pos[j] <= pos[i, last]).sum()) if causal else S_loc
+                want += -(-n_vis // 128)
+        assert cost == want
+
+
+def test_causal_work_totals_match_closed_form():
+    # striped spreads the causal triangle evenly: every shard's items cost about the same
+    S, N = 8192, 16
+    for layout, spread_max in (("striped", 1.10), ("zigzag", 1.25)):
+        items = ra.plan_items(1, 1, S, N, True, layout)
+        per_shard = np.zeros(N)
+        for _, _, i, _, cost in items.tolist():
+            per_shard[i] += cost
+        assert per_shard.max() / per_shard.min() < spread_max
+    items = ra.plan_items(1, 1, S, N, True, "contiguous")
+    per_shard = np.zeros(N)
+    for _, _, i, _, cost in items.tolist():
+        per_shard[i] += cost
+    assert per_shard[-1] / per_shard[0] > 10  # the last shard sees every earlier block
