@@ -1,0 +1,334 @@
+#!/usr/bin/env python
+"""Throughput of the exact ring-attention forward on B200: attention TFLOP/s (causal counted as
+half) on the s128k workload -- batch 1, 32 heads, head dim 128, 131072 tokens in 16 shards of
+8192, bf16, causal, striped layout -- with synthetic seeded inputs resident in HBM.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Prints one JSON line (rank 0).  `value` is device-timed (CUDA events around K back-to-back calls,
+max over ranks); `e2e` repeats the measurement through the public API with the inputs copied from
+pinned host memory and the result copied back inside the timed region; `roofline` is the
+attention kernel alone, timed with the library's event hook; `cpu_baseline` is the fp64 oracle on
+a bounded sample of the same workload on the host cores.  `--impl reference` times that oracle
+as the reference arm.  Inputs (3.2 GB) exceed the 126 MB L2, so no flush is needed.
+Under torchrun with N > 1 every rank runs its own replica (the virtual ring lives on one GPU;
+there is no data-path collective) and `value` sums the ranks' work over the slowest rank's time.
+"""
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from long_context_exact_forward_b200 import inputs  # noqa: E402
+
+METRIC = "ring-attn fwd TFLOP/s (bf16, causal) and % of B200 dense BF16 tensor peak"
+UNIT = "TFLOP/s"
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def attention_flops(B, H, S, D, causal):
+    """4 * B * H * S^2 * D, halved when causal (the convention of the target metric)."""
+    f = 4.0 * B * H * S * S * D
+    return f / 2 if causal else f
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return p, "measured"
+    except OSError:
+        return PEAKS_FALLBACK, "fallback"
+
+
+# ------------------------------------------------------------------ clocks during the timed region
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+
+    def __init__(self, device):
+        self.lines = []
+        self.proc = None
+        try:
+            uuid = "GPU-" + str(torch.cuda.get_device_properties(device).uuid)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", uuid, f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except (OSError, AttributeError):
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.thread.join(timeout=2)
+        sm, mx, power, reasons = [], [], [], set()
+        for line in self.lines:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx.append(float(parts[2]))
+                power.append(float(parts[3]))
+            except ValueError:
+                continue
+            for name, val in zip(self.REASONS, parts[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(name)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        # samples under load: power within 60% of the run's peak draw
+        pmax = max(power)
+        loaded = [s for s, p in zip(sm, power) if p >= 0.6 * pmax] or sm
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm), "power_w_max": pmax}
+
+
+# ------------------------------------------------------------------ distributed plumbing
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def max_over_ranks(x, world):
+    if world == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return t.item()
+
+
+def barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+
+
+# ------------------------------------------------------------------ oracle on the host cores
+def oracle_sample(q, k, v, causal, rows_per_head, seed_base=7000):
+    """Time the oracle on `rows_per_head` uniformly drawn query rows of every head."""
+    import oracle  # test-side fp64 reference: only this CPU-baseline leg runs it
+    B, S, H, D = q.shape
+    rows = np.stack([np.sort(np.random.default_rng(seed_base + h).choice(S, rows_per_head, replace=False))
+                     for h in range(H)])
+    threads = os.cpu_count() or 1
+    flops = B * sum(4.0 * D * ((r + 1) if causal else S) for r in rows.ravel())
+    t0 = time.perf_counter()
+    oracle.attention(q, k, v, causal, rows=rows, threads=threads)
+    dt = time.perf_counter() - t0
+    return flops, dt, threads, rows.size
+
+
+def run_reference(args, w):
+    """Reference arm: the fp64 oracle, as it stands, on the host cores (rank 0 only)."""
+    world, rank, _ = dist_env()
+    if rank != 0:
+        return
+    q, k, v = inputs.make_qkv(w.B, w.S, w.H, w.D, torch.bfloat16, "cpu", w.seed)
+    rows_per_head = args.ref_rows
+    for _ in range(args.warmup):
+        oracle_sample(q, k, v, True, rows_per_head)
+    tot_f, tot_t = 0.0, 0.0
+    for _ in range(args.steps):
+        f, dt, threads, n = oracle_sample(q, k, v, True, rows_per_head)
+        tot_f += f
+        tot_t += dt
+    value = tot_f / tot_t / 1e12
+    sample = (f"{rows_per_head} query rows per head x {w.H} heads of {w.name} (causal), "
+              f"{tot_f / args.steps:.3e} flops per step")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": tot_t / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": config_dict(w, args),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def config_dict(w, args):
+    return {
+        "workload": f"{w.name}: batch {w.B}, {w.H} heads, head dim {w.D}, {w.S} tokens in {w.n_ring} "
+                    f"shards of {w.S_loc}, bf16, causal, {args.layout} layout",
+        "B": w.B, "H": w.H, "S": w.S, "D": w.D, "n_ring": w.n_ring, "causal": True,
+        "layout": args.layout, "variant": args.variant,
+        "l2": "inputs (3 x B*S*H*D bf16) larger than the 126 MB L2; no flush",
+    }
+
+
+# ------------------------------------------------------------------ our arm
+def run_ours(args, w):
+    import long_context_exact_forward_b200 as ra
+    world, rank, local = dist_env()
+    if world > 1:
+        torch.cuda.set_device(local)
+        torch.distributed.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120))
+    dev = torch.device("cuda", torch.cuda.current_device())
+    stream = torch.cuda.current_stream()
+    B, H, S, D, N = w.B, w.H, w.S, w.D, w.n_ring
+    q, k, v = inputs.make_qkv(B, S, H, D, torch.bfloat16, dev, w.seed + rank)
+    out = torch.empty_like(q)
+    lse = torch.empty((B, H, S), dtype=torch.float32, device=dev)
+    ws = torch.empty(ra.workspace_size(B, H, S, D, N, True, args.layout, 1, variant=args.variant),
+                     dtype=torch.uint8, device=dev)
+    flops = attention_flops(B, H, S, D, True)
+
+    def step(ev=None):
+        ra.forward(q, k, v, N, True, args.layout, variant=args.variant, out=out, lse=lse,
+                   workspace=ws, stream=stream, events=ev)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    assert ra.get_device_status() == 0
+
+    # ---- device-timed region: K calls back to back, inputs resident in HBM
+    kev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    clocks = ClockSampler(dev)
+    start.record(stream)
+    for s in range(args.steps):
+        step(kev[s])
+    end.record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    barrier(world)
+    ms = max_over_ranks(start.elapsed_time(end), world)
+    kernel_ms = [a.elapsed_time(b) for a, b in kev]
+    status = ra.get_device_status()
+    ms_per_step = ms / args.steps
+    value = world * flops / (ms_per_step / 1e3) / 1e12
+
+    # ---- end to end through the public API: pinned host inputs in, result back to the host
+    e2e = None
+    if not args.no_e2e:
+        qh, kh, vh = (t.cpu().pin_memory() for t in (q, k, v))
+        oh = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+        lh = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+        qd, kd, vd = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+
+        def e2e_step():
+            qd.copy_(qh, non_blocking=True)
+            kd.copy_(kh, non_blocking=True)
+            vd.copy_(vh, non_blocking=True)
+            ra.forward(qd, kd, vd, N, True, args.layout, variant=args.variant, out=out, lse=lse,
+                       workspace=ws, stream=stream)
+            oh.copy_(out, non_blocking=True)
+            lh.copy_(lse, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        barrier(world)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ems = max_over_ranks(e0.elapsed_time(e1), world) / args.steps
+        bi = 3 * q.numel() * q.element_size()
+        bo = out.numel() * out.element_size() + lse.numel() * lse.element_size()
+        e2e = {"value": world * flops / (ems / 1e3) / 1e12, "unit": UNIT, "h2d_bytes_per_step": bi,
+               "d2h_bytes_per_step": bo, "ms_per_step": ems}
+        del qh, kh, vh, oh, lh, qd, kd, vd
+
+    # ---- roofline of the dominant kernel (the attention kernel)
+    peaks, peak_src = load_peaks()
+    k_ms = statistics.mean(kernel_ms)
+    achieved = flops / (k_ms / 1e3) / 1e12
+    peak = peaks["bf16_tflops_sustained"]
+    roofline = {
+        "bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+        "traffic": args.traffic_bytes,
+        "peak_kind": f"bf16 dense cuBLAS, sustained ({peak_src})",
+        "frac_of_burst_peak": achieved / peaks["bf16_tflops"],
+        "kernel": "attn_tc_kernel<128> (fused ring, tcgen05)", "kernel_ms": k_ms,
+        "algorithmic_flops_per_launch": flops,
+    }
+
+    # ---- CPU baseline: the oracle on a bounded sample (rank 0, N = 1 only)
+    cpu = None
+    if not args.no_cpu_baseline and world == 1 and rank == 0:
+        qc, kc, vc = q.cpu(), k.cpu(), v.cpu()
+        f, dt, threads, n = oracle_sample(qc, kc, vc, True, args.cpu_rows)
+        cpu = {"value": f / dt / 1e12, "unit": UNIT, "cores": threads, "kind": "oracle",
+               "sample": f"{args.cpu_rows} query rows per head x {H} heads of {w.name} (causal), "
+                         f"{f:.3e} flops in {dt:.1f} s"}
+
+    launches_per_step = (1 if args.layout != "contiguous" else 0) + (
+        1 if args.variant in ("fused", "auto") else 2 * N - 1)
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": config_dict(w, args),
+        "pct_of_bf16_peak": {"burst_measured": value / world / peaks["bf16_tflops"],
+                             "sustained_measured": value / world / peaks["bf16_tflops_sustained"],
+                             "nvidia_dense_spec_2250": value / world / 2250.0},
+        "clocks": clk, "e2e": e2e, "roofline": roofline, "cpu_baseline": cpu,
+        "gpu_launches": launches_per_step * args.steps, "device_status": status,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="s128k", choices=sorted(inputs.WORKLOADS))
+    ap.add_argument("--layout", default="striped", choices=["contiguous", "striped", "zigzag"])
+    ap.add_argument("--variant", default="fused", choices=["fused", "per_step"])
+    ap.add_argument("--heads", type=int, default=0, help="override the head count (profiling runs)")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-rows", type=int, default=256, help="oracle rows per head for cpu_baseline")
+    ap.add_argument("--ref-rows", type=int, default=64, help="oracle rows per head per reference step")
+    ap.add_argument("--traffic-bytes", type=float, default=None,
+                    help="DRAM bytes per attention launch from an ncu capture of this kernel")
+    args = ap.parse_args()
+    w = inputs.WORKLOADS[args.workload]
+    if args.heads:
+        from dataclasses import replace
+        w = replace(w, H=args.heads)
+    if args.impl == "reference":
+        run_reference(args, w)
+    else:
+        run_ours(args, w)
+
+
+if __name__ == "__main__":
+    main()

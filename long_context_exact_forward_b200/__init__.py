@@ -166,6 +166,9 @@ def forward(q, k, v, n_ring, causal=True, layout="contiguous", *, variant="auto"
     opt.timeout_ns = int(timeout_ns)
     opt.debug = int(debug)
     if events is not None:
+        for ev in events:  # torch creates the CUDA event lazily, on first record
+            if ev.cuda_event == 0:
+                ev.record(stream if stream is not None else torch.cuda.current_stream())
         opt.attn_events[0] = events[0].cuda_event
         opt.attn_events[1] = events[1].cuda_event
     with torch.cuda.device(q.device):
