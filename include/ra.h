@@ -154,6 +154,30 @@ RA_API int ra_plan_tiles(int64_t S, int n_ring, int layout, int causal, int tile
 RA_API int ra_plan_items(int64_t B, int64_t H, int64_t S, int n_ring, int causal, int layout,
                   int32_t* items, int64_t cap, int64_t* n_items);
 
+/* RA_NOALLOC_SCRATCH_BYTES: size of the fixed device array that ra_forward_noalloc uses as
+ * scratch.  Every GPU that loads the library holds this much device memory until the process
+ * exits. */
+#define RA_NOALLOC_SCRATCH_BYTES (64u << 20)
+
+/* ra_forward_noalloc: the pages have no counterpart to this call; it exists for callers that
+ * cannot let a library allocate GPU memory -- code recording a CUDA graph, engines that manage
+ * every byte of device memory through their own allocator, loops where an allocation could stall.
+ * It computes what ra_forward computes for bf16 q, k, v with D in {64, 128} on sm_100 (the fused
+ * tensor-core ring), but takes its scratch (work list; shard-major copies of q, k, v for the
+ * striped and zigzag layouts) from one fixed device array of RA_NOALLOC_SCRATCH_BYTES instead of
+ * allocating.  Arguments as for ra_forward (dtype is bf16 implicitly).
+ *   - The first call on a device looks up the array's address with that device current; make it
+ *     before any stream capture.
+ *   - All calls on a device share the array and leave their data in it; calls whose GPU work
+ *     overlaps (other streams, other host threads) race on it.
+ *   - A problem whose scratch does not fit (B*H*n_ring*ceil(S_loc/256) work items of 16 bytes,
+ *     plus 3*B*S*H*D*2 bytes for striped/zigzag, at most 12288 items per head) is rejected with
+ *     RA_ERR_NO_WORKSPACE and a message in ra_last_error_string; nothing is enqueued.
+ *   - Other dtypes or head dims return RA_ERR_UNSUPPORTED. */
+RA_API int ra_forward_noalloc(const void* q, const void* k, const void* v, void* out, float* lse,
+                              int64_t B, int64_t H, int64_t S, int64_t D, int n_ring, int causal,
+                              int layout, void* stream);
+
 /* ra_status_string: static description of a status code. */
 RA_API const char* ra_status_string(int status);
 

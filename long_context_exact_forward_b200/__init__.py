@@ -76,6 +76,7 @@ def lib():
         L.ra_permute.argtypes = [vp, vp, i64, i64, i64, i64, ci, ci, ci, vp]
         L.ra_unpermute.argtypes = [vp, vp, i64, i64, i64, i64, ci, ci, ci, vp]
         L.ra_merge_partials.argtypes = [vp, vp, vp, vp, i64, i64, vp]
+        L.ra_forward_noalloc.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i64, ci, ci, ci, vp]
         L.ra_layout_positions.argtypes = [i64, ci, ci, vp]
         L.ra_plan_tiles.argtypes = [i64, ci, ci, ci, ci, vp]
         L.ra_plan_items.argtypes = [i64, i64, i64, ci, ci, ci, vp, i64, ctypes.POINTER(ctypes.c_int64)]
@@ -84,7 +85,7 @@ def lib():
         L.ra_last_error_string.restype = ctypes.c_char_p
         L.ra_last_error_string.argtypes = []
         L.ra_get_device_status.argtypes = []
-        for name in ("ra_forward", "ra_forward_ex", "ra_workspace_size", "ra_permute",
+        for name in ("ra_forward", "ra_forward_ex", "ra_forward_noalloc", "ra_workspace_size", "ra_permute",
                      "ra_unpermute", "ra_merge_partials", "ra_layout_positions", "ra_plan_tiles",
                      "ra_plan_items", "ra_get_device_status"):
             getattr(L, name).restype = ctypes.c_int
@@ -177,6 +178,28 @@ def forward(q, k, v, n_ring, causal=True, layout="contiguous", *, variant="auto"
                                  LAYOUTS[layout], _dtype_code(q), _stream_handle(stream),
                                  ctypes.byref(opt))
     _check(rc, "ra_forward_ex")
+    return out, lse
+
+
+def forward_noalloc(q, k, v, n_ring, causal=True, layout="contiguous", *, out=None, lse=None,
+                    stream=None):
+    """ra_forward_noalloc: like forward() for bf16 inputs, but the library allocates nothing --
+    its scratch is a fixed device array shared by all calls on the device (see include/ra.h)."""
+    torch = _torch()
+    _check_cuda(q, k, v)
+    if q.dtype != torch.bfloat16 or k.dtype != q.dtype or v.dtype != q.dtype:
+        raise TypeError("forward_noalloc takes bf16 q, k, v")
+    B, S, H, D = q.shape
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, H, S), dtype=torch.float32, device=q.device)
+    _check_cuda(out, lse)
+    with torch.cuda.device(q.device):
+        rc = lib().ra_forward_noalloc(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                                      lse.data_ptr(), B, H, S, D, int(n_ring), int(bool(causal)),
+                                      LAYOUTS[layout], _stream_handle(stream))
+    _check(rc, "ra_forward_noalloc")
     return out, lse
 
 

@@ -445,6 +445,27 @@ ra_options default_options() {
 
 }  // namespace
 
+// Helpers shared with other entry points of the library (declared in ra_internal.cuh).
+namespace ra {
+int host_check_shape(int64_t B, int64_t H, int64_t S, int64_t D, int n_ring, int layout, int dtype) {
+    return check_shape(B, H, S, D, n_ring, layout, dtype);
+}
+int host_device_facts(int* sms, bool* sm100, int** status) {
+    DeviceInfo d;
+    const int rc = device_info(&d);
+    if (rc != RA_OK) return rc;
+    *sms = d.sms;
+    *sm100 = d.sm100;
+    *status = d.status;
+    return RA_OK;
+}
+int host_encode_qkv_map(CUtensorMap* map, const void* base, int64_t B, const Layout& L, int64_t H, int64_t D) {
+    return encode_qkv_map(map, base, B, L, H, D);
+}
+int host_cuda_fail(cudaError_t e, const char* what) { return cuda_fail(e, what); }
+void host_set_error(const char* msg) { snprintf(g_last_error, sizeof g_last_error, "%s", msg); }
+}  // namespace ra
+
 extern "C" {
 
 int ra_forward(const void* q, const void* k, const void* v, void* out, float* lse, int64_t B,

@@ -1,0 +1,60 @@
+"""ra_forward_noalloc: the forward pass for callers that cannot let the library allocate GPU
+memory (graph capture, engines that own all device memory, allocation-free hot loops).  Its
+scratch is one fixed device array shared by all calls on a device.
+
+The entry point is called through the C ABI and checked against ra_forward (the allocating entry
+point) within the bf16 tolerances of the other GPU tests, on two calls in a row with different
+problems so that the second call reuses scratch the first one left behind.  This file is named to
+be collected last.
+"""
+import ctypes
+
+import pytest
+import torch
+
+import long_context_exact_forward_b200 as ra
+from long_context_exact_forward_b200 import inputs
+
+pytestmark = pytest.mark.gpu
+
+CASES = [  # B, H, S, D, n_ring, causal, layout
+    (1, 4, 4 * 1024, 128, 4, True, "striped"),
+    (1, 3, 2 * 1000, 128, 2, True, "contiguous"),
+    (2, 2, 8 * 256, 64, 8, False, "zigzag"),
+]
+
+
+def call_noalloc(q, k, v, n_ring, causal, layout):
+    B, S, H, D = q.shape
+    out = torch.empty_like(q)
+    lse = torch.empty((B, H, S), dtype=torch.float32, device=q.device)
+    stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    rc = ra.lib().ra_forward_noalloc(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                                     lse.data_ptr(), B, H, S, D, n_ring, int(causal),
+                                     ra.LAYOUTS[layout], stream)
+    return rc, out, lse
+
+
+def test_noalloc_matches_allocating_entry_point_twice_in_a_row():
+    for rep in range(2):
+        for n, (B, H, S, D, N, causal, layout) in enumerate(CASES):
+            q, k, v = inputs.make_qkv(B, S, H, D, torch.bfloat16, "cuda", seed=100 * rep + n)
+            rc, out, lse = call_noalloc(q, k, v, N, causal, layout)
+            assert rc == 0, ra.status_string(rc)
+            ref, ref_lse = ra.forward(q, k, v, N, causal, layout)
+            torch.cuda.synchronize()
+            assert ra.get_device_status() == 0
+            d = (out.float() - ref.float()).abs()
+            assert d.max().item() <= 2e-2 and d.mean().item() <= 2e-3
+            assert (lse - ref_lse).abs().max().item() <= 1e-3
+
+
+def test_noalloc_rejects_problems_beyond_its_scratch():
+    # striped needs 3 shard-major copies: 3 x 1 x 65536 x 4 x 128 x 2 B = 192 MiB > 64 MiB
+    q, k, v = inputs.make_qkv(1, 65536, 4, 128, torch.bfloat16, "cuda", seed=1)
+    rc, _, _ = call_noalloc(q, k, v, 8, True, "striped")
+    assert rc == -5  # RA_ERR_NO_WORKSPACE
+    assert b"RA_NOALLOC_SCRATCH_BYTES" in ra.lib().ra_last_error_string()
+    q2, k2, v2 = inputs.make_qkv(1, 256, 1, 96, torch.bfloat16, "cuda", seed=2)
+    rc, _, _ = call_noalloc(q2, k2, v2, 2, True, "contiguous")
+    assert rc == -4  # RA_ERR_UNSUPPORTED: head dim outside the tensor-core kernel
