@@ -22,7 +22,9 @@ import os
 import numpy as np
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libra_b200.so")
+# RA_LIB may name another build of the same library (for example one compiled with different
+# tuning constants); by default the in-tree build is used.
+LIB_PATH = os.environ.get("RA_LIB") or os.path.join(_HERE, "libra_b200.so")
 
 LAYOUTS = {"contiguous": 0, "striped": 1, "zigzag": 2}
 VARIANTS = {"auto": 0, "fused": 1, "per_step": 2}

@@ -56,6 +56,42 @@ constexpr float kLn2 = 0.6931471805599453f;
 constexpr uint32_t kNegInfBits = 0xff800000u;
 constexpr int kColBlockBytes = 128 * 128;  // one 128-row x 64-element bf16 block (128-B rows)
 
+// Every kExp2PolyEvery-th pair of P columns can be exponentiated on the FMA pipe instead of the
+// MUFU unit (16 384 exponentials per 128x128 tile, as many cycles as the tile's MMAs).  Measured
+// on s128k: 0 (all on MUFU) is fastest, 4 costs 4.5 % and 2 costs 8 %: the softmax warps are bound
+// by issue latency, not by the MUFU pipe, so the default is 0.
+#ifndef RA_EXP2_POLY_EVERY
+#define RA_EXP2_POLY_EVERY 0
+#endif
+constexpr int kExp2PolyEvery = RA_EXP2_POLY_EVERY;
+
+// 2^x for a pair of floats on the FMA pipe (Cody-Waite style range reduction):
+//   x is clamped to >= -127, t = x + 1.5*2^23 rounded toward -inf puts floor(x) in t's low
+//   mantissa bits, f = x - floor(x) in [0, 1), 2^f ~ 1 + f(c1 + f(c2 + f c3)), and floor(x) is added
+//   to the exponent field (t's bits shifted left by 23 equal floor(x) << 23 modulo 2^32).
+//   c1..c3 minimise the maximum relative error of the cubic on [0, 1) with p(0) = 1 fixed (a
+//   linear program on 4001 points): 8.6e-5, far below the 2^-9 rounding of P to bf16.  At
+//   x = -127 the result is exactly +0 (f = 0, p = 1, exponent field 0), so masked scores vanish.
+__device__ __forceinline__ uint64_t exp2_poly_f32x2(uint64_t x2) {
+    constexpr float kShift = 12582912.0f;  // 1.5 * 2^23
+    float x0, x1;
+    split_f32x2(x2, x0, x1);
+    const uint64_t xc = f32x2(fmaxf(x0, -127.f), fmaxf(x1, -127.f));
+    const uint64_t t = add_rm_f32x2(xc, f32x2(kShift, kShift));
+    const uint64_t fl = sub_f32x2(t, f32x2(kShift, kShift));
+    const uint64_t fr = sub_f32x2(xc, fl);
+    uint64_t p = fma_f32x2(fr, f32x2(0.07706724107265472f, 0.07706724107265472f),
+                           f32x2(0.22764497995376587f, 0.22764497995376587f));
+    p = fma_f32x2(p, fr, f32x2(0.6951166391372681f, 0.6951166391372681f));
+    p = fma_f32x2(p, fr, f32x2(1.f, 1.f));
+    float t0, t1, p0, p1;
+    split_f32x2(t, t0, t1);
+    split_f32x2(p, p0, p1);
+    const uint32_t r0 = __float_as_uint(p0) + (__float_as_uint(t0) << 23);
+    const uint32_t r1 = __float_as_uint(p1) + (__float_as_uint(t1) << 23);
+    return f32x2(__uint_as_float(r0), __uint_as_float(r1));
+}
+
 template <int kD>
 struct TcSmem {
     static constexpr int kTileBytes = kM * kD * 2;
@@ -73,41 +109,39 @@ template <int kD>
 __device__ __forceinline__ uint32_t o_col(int q) { return 256u + (uint32_t)q * 128u; }
 
 struct ItemGeom {
-    int64_t b, h, i;
-    int64_t a0[2];    // first local row of each query tile
-    int64_t last[2];  // last valid local row of each query tile (clamped to the shard)
+    int b, h, i;
+    int a0[2];    // first local row of each query tile
+    int last[2];  // last valid local row of each query tile (clamped to the shard)
 };
 
-__device__ __forceinline__ ItemGeom item_geom(const AttnArgs& A, int4 it) {
+__device__ __forceinline__ ItemGeom item_geom(const Layout32& L, int4 it) {
     ItemGeom G;
     G.b = it.x;
     G.h = it.y;
     G.i = it.z;
     for (int q = 0; q < 2; ++q) {
-        G.a0[q] = (int64_t)it.w * 2 * kM + q * kM;
-        const int64_t e = G.a0[q] + kM - 1;
-        G.last[q] = e < A.L.S_loc - 1 ? e : A.L.S_loc - 1;
+        G.a0[q] = it.w * 2 * kM + q * kM;
+        const int e = G.a0[q] + kM - 1;
+        G.last[q] = e < L.S_loc - 1 ? e : L.S_loc - 1;
     }
     return G;
 }
 
 // Live key tiles of block j for query tile q (0 if the tile lies past the shard end).
-__device__ __forceinline__ int tiles_for(const AttnArgs& A, const ItemGeom& G, int q, int64_t j) {
-    if (G.a0[q] >= A.L.S_loc) return 0;
-    const int64_t n = visible_keys(A.L, A.causal, G.i, G.last[q], j);
-    return (int)((n + kN - 1) / kN);
+__device__ __forceinline__ int tiles_for(const Layout32& L, int causal, const ItemGeom& G, int q, int j) {
+    if (G.a0[q] >= L.S_loc) return 0;
+    return (visible_keys(L, causal, G.i, G.last[q], j) + kN - 1) / kN;
 }
 
 // Flat sequence of (step, key tile) pairs of one item, skipping dead steps.
 struct TileIter {
-    int s, s_end, kt, nt0, nt1;
-    int64_t j;
+    int s, s_end, kt, nt0, nt1, j;
     bool valid;
-    __device__ __forceinline__ void load_step(const AttnArgs& A, const ItemGeom& G) {
+    __device__ __forceinline__ void load_step(const Layout32& L, int causal, const ItemGeom& G) {
         for (; s < s_end; ++s) {
-            j = ring_block(G.i, s, A.L.N);
-            nt0 = tiles_for(A, G, 0, j);
-            nt1 = tiles_for(A, G, 1, j);
+            j = ring_block32(G.i, s, L.N);
+            nt0 = tiles_for(L, causal, G, 0, j);
+            nt1 = tiles_for(L, causal, G, 1, j);
             if (nt0 > 0 || nt1 > 0) {
                 valid = true;
                 return;
@@ -115,17 +149,17 @@ struct TileIter {
         }
         valid = false;
     }
-    __device__ __forceinline__ void init(const AttnArgs& A, const ItemGeom& G) {
+    __device__ __forceinline__ void init(const AttnArgs& A, const Layout32& L, const ItemGeom& G) {
         s = A.s_begin;
         s_end = A.s_end;
         kt = 0;
-        load_step(A, G);
+        load_step(L, A.causal, G);
     }
-    __device__ __forceinline__ void next(const AttnArgs& A, const ItemGeom& G) {
+    __device__ __forceinline__ void next(const Layout32& L, int causal, const ItemGeom& G) {
         if (++kt >= (nt0 > nt1 ? nt0 : nt1)) {
             kt = 0;
             ++s;
-            load_step(A, G);
+            load_step(L, causal, G);
         }
     }
     __device__ __forceinline__ bool act(int q) const { return kt < (q ? nt1 : nt0); }
@@ -159,6 +193,7 @@ struct Roles {
     int* status;
     volatile int* abort;
     uint32_t tmem;
+    Layout32 L;
 
     // ------------------------------------------------------------ TMA producer (one thread)
     __device__ void producer(const CUtensorMap* tm_q, const CUtensorMap* tm_k,
@@ -166,9 +201,9 @@ struct Roles {
         uint32_t slot_it = 0, q_it = 0;
         bool ok = true;
         for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
-            const ItemGeom G = item_geom(A, items[it]);
+            const ItemGeom G = item_geom(L, items[it]);
             TileIter t;
-            t.init(A, G);
+            t.init(A, L, G);
             if (!t.valid) continue;
             if (debug == RA_DEBUG_STALL_LOADS) continue;  // consumers must time out
             if (!mbar_wait(&sm.q_empty, (q_it & 1) ^ 1, timeout, abort)) { ok = false; break; }
@@ -178,7 +213,7 @@ struct Roles {
                     tma_load_5d(sm.q[q] + cb * kColBlockBytes, tm_q, &sm.q_full, cb * 64, (int)G.h,
                                 (int)G.a0[q], (int)G.i, (int)G.b);
             ++q_it;
-            for (; t.valid && ok; t.next(A, G)) {
+            for (; t.valid && ok; t.next(L, A.causal, G)) {
                 for (int w = 0; w < 2; ++w) {  // K then V of this tile
                     const uint32_t slot = slot_it % kSlots;
                     if (!mbar_wait(&sm.slot_empty[slot], ((slot_it / kSlots) & 1) ^ 1, timeout, abort)) {
@@ -239,9 +274,9 @@ struct Roles {
             return ok;
         };
         for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
-            const ItemGeom G = item_geom(A, items[it]);
+            const ItemGeom G = item_geom(L, items[it]);
             TileIter cur;
-            cur.init(A, G);
+            cur.init(A, L, G);
             if (!cur.valid) continue;
             if (!wait(&sm.q_full, q_it & 1)) break;
             ++q_it;
@@ -256,7 +291,7 @@ struct Roles {
                 }
             mma_commit(&sm.slot_empty[kslot]);
             TileIter nxt = cur;
-            nxt.next(A, G);
+            nxt.next(L, A.causal, G);
             if (!nxt.valid) mma_commit(&sm.q_empty);
             for (;;) {
                 const uint32_t vslot = cons_it % kSlots;
@@ -291,7 +326,7 @@ struct Roles {
                 }
                 mma_commit(&sm.slot_empty[kslot]);
                 cur = nxt;
-                nxt.next(A, G);
+                nxt.next(L, A.causal, G);
                 if (!nxt.valid) mma_commit(&sm.q_empty);
             }
             if (!ok) break;
@@ -322,15 +357,15 @@ struct Roles {
             return ok;
         };
         for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
-            const ItemGeom G = item_geom(A, items[it]);
-            const int64_t a = G.a0[q] + row;
+            const ItemGeom G = item_geom(L, items[it]);
+            const int a = G.a0[q] + row;
             float m_run = -INFINITY, l = 0.f;
             int n_act = 0;
             for (int s = A.s_begin; s < A.s_end && ok; ++s) {
-                const int64_t j = ring_block(G.i, s, A.L.N);
-                const int nt = tiles_for(A, G, q, j);
+                const int j = ring_block32(G.i, s, L.N);
+                const int nt = tiles_for(L, A.causal, G, q, j);
                 if (nt == 0) continue;
-                const int64_t cnt = visible_keys(A.L, A.causal, G.i, a, j);
+                const int cnt = visible_keys(L, A.causal, G.i, a, j);
                 for (int kt = 0; kt < nt; ++kt) {
                     if (!wait_all(&sm.s_full[q], s_cnt & 1)) break;
                     ++s_cnt;
@@ -341,19 +376,26 @@ struct Roles {
 #pragma unroll
                     for (int c = 0; c < 4; ++c)
                         tmem_wait_ld_regs(*reinterpret_cast<uint32_t(*)[32]>(&r[c * 32]));
-                    const int64_t valid = cnt - (int64_t)kt * kN;
+                    const int valid = cnt - kt * kN;
                     if (valid < kN) {
 #pragma unroll
                         for (int c = 0; c < kN; ++c)
                             if (c >= valid) r[c] = kNegInfBits;
                     }
-                    float mx0 = -INFINITY, mx1 = -INFINITY;
+#define SF(c) __uint_as_float(r[(c)])
+                    // row max: 8 independent chains of three-input max
+                    float mc[8];
 #pragma unroll
-                    for (int c = 0; c < kN; c += 2) {
-                        mx0 = fmaxf(mx0, __uint_as_float(r[c]));
-                        mx1 = fmaxf(mx1, __uint_as_float(r[c + 1]));
-                    }
-                    const float m_new = fmaxf(m_run, fmaxf(mx0, mx1) * sl2);
+                    for (int k = 0; k < 8; ++k) mc[k] = fmax3(SF(k), SF(k + 8), SF(k + 16));
+#pragma unroll
+                    for (int c = 24; c < 120; c += 16)
+#pragma unroll
+                        for (int k = 0; k < 8; ++k) mc[k] = fmax3(mc[k], SF(c + k), SF(c + k + 8));
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) mc[k] = fmaxf(mc[k], SF(120 + k));
+                    const float mx = fmax3(fmax3(mc[0], mc[1], mc[2]), fmax3(mc[3], mc[4], mc[5]),
+                                           fmaxf(mc[6], mc[7]));
+                    const float m_new = fmaxf(m_run, mx * sl2);
                     bool rescale = false;
                     float alpha = 1.f;
                     if (n_act == 0) {
@@ -365,29 +407,54 @@ struct Roles {
                         m_run = m_new;
                     }
                     const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
-                    float l0 = 0.f, l1 = 0.f;
+                    // P = 2^(S * scale * log2 e - m), two columns per packed op; every
+                    // kExp2PolyEvery-th pair on the FMA pipe, the rest on MUFU
+                    const uint64_t scale2 = f32x2(sl2, sl2), neg_m2 = f32x2(-m_use, -m_use);
+                    uint64_t lsum[4] = {0, 0, 0, 0};
 #pragma unroll
                     for (int c4 = 0; c4 < 4; ++c4) {
                         uint32_t pk[16];
 #pragma unroll
                         for (int x = 0; x < 16; ++x) {
-                            const float p0 = ex2(fmaf(__uint_as_float(r[c4 * 32 + 2 * x]), sl2, -m_use));
-                            const float p1 = ex2(fmaf(__uint_as_float(r[c4 * 32 + 2 * x + 1]), sl2, -m_use));
-                            l0 += p0;
-                            l1 += p1;
+                            const int c = c4 * 32 + 2 * x;
+                            const uint64_t t2 = fma_f32x2(f32x2(SF(c), SF(c + 1)), scale2, neg_m2);
+                            uint64_t p2;
+                            if (kExp2PolyEvery > 0 && (x % kExp2PolyEvery) == kExp2PolyEvery - 1) {
+                                p2 = exp2_poly_f32x2(t2);
+                            } else {
+                                float t0, t1;
+                                split_f32x2(t2, t0, t1);
+                                p2 = f32x2(ex2(t0), ex2(t1));
+                            }
+                            lsum[x & 3] = add_f32x2(lsum[x & 3], p2);
+                            float p0, p1;
+                            split_f32x2(p2, p0, p1);
                             pk[x] = pack_bf16x2(p0, p1);
                         }
                         tmem_st16(tS + c4 * 16, pk);
                     }
-                    l += l0 + l1;
+                    {
+                        float a0, a1, b0, b1;
+                        split_f32x2(add_f32x2(add_f32x2(lsum[0], lsum[1]), add_f32x2(lsum[2], lsum[3])), a0, a1);
+                        (void)b0;
+                        (void)b1;
+                        l += a0 + a1;
+                    }
+#undef SF
                     if (__any_sync(0xffffffffu, rescale)) {
+                        const uint64_t alpha2 = f32x2(alpha, alpha);
 #pragma unroll 1
                         for (int c = 0; c < kD / 32; ++c) {
                             uint32_t o[32];
                             tmem_ld32(tO + c * 32, o);
                             tmem_wait_ld_regs(o);
 #pragma unroll
-                            for (int x = 0; x < 32; ++x) o[x] = __float_as_uint(__uint_as_float(o[x]) * alpha);
+                            for (int x = 0; x < 16; ++x) {
+                                float v0, v1;
+                                split_f32x2(mul_f32x2(f32x2(__uint_as_float(o[2 * x]), __uint_as_float(o[2 * x + 1])), alpha2), v0, v1);
+                                o[2 * x] = __float_as_uint(v0);
+                                o[2 * x + 1] = __float_as_uint(v1);
+                            }
                             tmem_st32(tO + c * 32, o);
                         }
                     }
@@ -404,20 +471,20 @@ struct Roles {
     }
 
     template <typename Wait>
-    __device__ void epilogue(int q, const ItemGeom& G, int64_t a, int n_act, float m_run, float l,
+    __device__ void epilogue(int q, const ItemGeom& G, int a, int n_act, float m_run, float l,
                              uint32_t tO, bool& ok, Wait& wait_all, uint32_t& items_act) {
-        const bool row_ok = a < A.L.S_loc;
+        const bool row_ok = a < L.S_loc;
         const float inv_l = l > 0.f ? 1.f / l : 0.f;
         const float lse = l > 0.f ? (m_run + log2f(l)) * kLn2 : -INFINITY;
         const int64_t H = A.H, S = A.L.S;
         float* lse_dst;
         uint8_t* row_dst;
         if (A.out_mode == kOutFinal) {
-            const int64_t g = row_ok ? global_position(A.L, G.i, a) : 0;
+            const int64_t g = row_ok ? global_position(L, G.i, a) : 0;
             row_dst = static_cast<uint8_t*>(A.out) + (((G.b * S + g) * H + G.h) * kD) * 2;
             lse_dst = A.lse + (G.b * H + G.h) * S + g;
         } else {
-            const int64_t rr = ((G.b * A.L.N + G.i) * A.L.S_loc + a) * H + G.h;
+            const int64_t rr = (((int64_t)G.b * L.N + G.i) * L.S_loc + a) * H + G.h;
             row_dst = static_cast<uint8_t*>(A.out) + rr * kD * 4;
             lse_dst = A.lse + rr;
         }
@@ -506,14 +573,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     tc_fence_after();
 
-    Roles<kD> roles{sm, A, items, n_items, timeout_ns, status, &sm.abort, sm.tmem_base};
-    if (warp == kLoadWarp) {
-        if (lane == 0) roles.producer(&tm_q, &tm_k, &tm_v, debug);
-        __syncwarp();
-    } else if (warp == kMmaWarp) {
-        if (lane == 0) roles.mma();
-        __syncwarp();
-    } else if (warp < 8) {
+    Roles<kD> roles{sm, A, items, n_items, timeout_ns, status, &sm.abort, sm.tmem_base, narrow(A.L)};
+    // register split: 256 softmax threads x 208 + 128 producer/MMA threads x 80 = 63488 <= 384 x 168
+    if (warp >= 8) {
+        setmaxnreg_dec80();
+        if (warp == kLoadWarp) {
+            if (lane == 0) roles.producer(&tm_q, &tm_k, &tm_v, debug);
+            __syncwarp();
+        } else if (warp == kMmaWarp) {
+            if (lane == 0) roles.mma();
+            __syncwarp();
+        }
+    } else {
+        setmaxnreg_inc208();
         roles.softmax(warp >> 2, warp, threadIdx.x & 127);
     }
 

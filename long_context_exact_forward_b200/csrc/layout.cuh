@@ -58,4 +58,36 @@ RA_HD int64_t visible_keys(const Layout& L, int causal, int64_t i, int64_t a, in
 // (ultralytics.com "Ring Attention" toy loop; jisaku.com 処理フロー t = 0 .. N-1).
 RA_HD int64_t ring_block(int64_t i, int64_t s, int64_t N) { return ((i - s) % N + N) % N; }
 
+// 32-bit forms of the same maps for device code (the host rejects S >= 2^31, so every position,
+// count and index of a shard fits in 32 bits; 32-bit division is far cheaper on the GPU).
+struct Layout32 {
+    int S, N, S_loc, kind;
+};
+
+RA_HD Layout32 narrow(const Layout& L) { return Layout32{(int)L.S, (int)L.N, (int)L.S_loc, L.kind}; }
+
+RA_HD int clamp32(int x, int lo, int hi) { return x < lo ? lo : (x > hi ? hi : x); }
+
+RA_HD int global_position(const Layout32& L, int i, int a) {
+    if (L.kind == 0) return i * L.S_loc + a;
+    if (L.kind == 1) return a * L.N + i;
+    const int C = L.S_loc >> 1;
+    return a < C ? i * C + a : (2 * L.N - 1 - i) * C + (a - C);
+}
+
+RA_HD int key_count(const Layout32& L, int j, int gq) {
+    if (L.kind == 0) return clamp32(gq - j * L.S_loc + 1, 0, L.S_loc);
+    if (L.kind == 1) return gq < j ? 0 : clamp32((gq - j) / L.N + 1, 0, L.S_loc);
+    const int C = L.S_loc >> 1;
+    return clamp32(gq - j * C + 1, 0, C) + clamp32(gq - (2 * L.N - 1 - j) * C + 1, 0, C);
+}
+
+RA_HD int visible_keys(const Layout32& L, int causal, int i, int a, int j) {
+    if (!causal) return L.S_loc;
+    if (a >= L.S_loc) a = L.S_loc - 1;
+    return key_count(L, j, global_position(L, i, a));
+}
+
+RA_HD int ring_block32(int i, int s, int N) { return ((i - s) % N + N) % N; }
+
 }  // namespace ra
