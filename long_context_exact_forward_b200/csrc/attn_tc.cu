@@ -98,7 +98,8 @@ struct TcSmem {
     uint8_t q[2][kTileBytes];         // each tile: kD/64 column blocks of 128 rows x 128 B
     uint8_t kv[kSlots][kTileBytes];
     uint64_t q_full, q_empty, drain;
-    uint64_t slot_full[kSlots], slot_empty[kSlots];
+    uint64_t kv_full[2];              // K and V of key tile n have landed (barrier n % 2)
+    uint64_t slot_empty[kSlots];      // key tile n uses slots 2n and 2n+1 (mod kSlots)
     uint64_t s_full[2], p_full[2], o_final[2], o_free[2];
     uint32_t tmem_base;
     int abort;
@@ -198,7 +199,7 @@ struct Roles {
     // ------------------------------------------------------------ TMA producer (one thread)
     __device__ void producer(const CUtensorMap* tm_q, const CUtensorMap* tm_k,
                              const CUtensorMap* tm_v, int debug) {
-        uint32_t slot_it = 0, q_it = 0;
+        uint32_t tile_it = 0, q_it = 0;
         bool ok = true;
         for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
             const ItemGeom G = item_geom(L, items[it]);
@@ -210,31 +211,32 @@ struct Roles {
             mbar_arrive_expect_tx(&sm.q_full, 2 * TcSmem<kD>::kTileBytes);
             for (int q = 0; q < 2; ++q)
                 for (int cb = 0; cb < kD / 64; ++cb)
-                    tma_load_5d(sm.q[q] + cb * kColBlockBytes, tm_q, &sm.q_full, cb * 64, (int)G.h,
-                                (int)G.a0[q], (int)G.i, (int)G.b);
+                    tma_load_5d(sm.q[q] + cb * kColBlockBytes, tm_q, &sm.q_full, cb * 64, G.h,
+                                G.a0[q], G.i, G.b);
             ++q_it;
             for (; t.valid && ok; t.next(L, A.causal, G)) {
-                for (int w = 0; w < 2; ++w) {  // K then V of this tile
-                    const uint32_t slot = slot_it % kSlots;
-                    if (!mbar_wait(&sm.slot_empty[slot], ((slot_it / kSlots) & 1) ^ 1, timeout, abort)) {
+                uint64_t* full = &sm.kv_full[tile_it & 1];
+                for (int w = 0; w < 2; ++w) {  // K then V of this tile, each as soon as its slot frees
+                    const uint32_t use = 2 * tile_it + w;
+                    const uint32_t slot = use % kSlots;
+                    if (!mbar_wait(&sm.slot_empty[slot], ((use / kSlots) & 1) ^ 1, timeout, abort)) {
                         ok = false;
                         break;
                     }
-                    mbar_arrive_expect_tx(&sm.slot_full[slot], TcSmem<kD>::kTileBytes);
+                    if (w == 0) mbar_arrive_expect_tx(full, 2 * TcSmem<kD>::kTileBytes);
                     for (int cb = 0; cb < kD / 64; ++cb)
-                        tma_load_5d(sm.kv[slot] + cb * kColBlockBytes, w ? tm_v : tm_k,
-                                    &sm.slot_full[slot], cb * 64, (int)G.h, t.kt * kN, (int)t.j,
-                                    (int)G.b);
-                    ++slot_it;
+                        tma_load_5d(sm.kv[slot] + cb * kColBlockBytes, w ? tm_v : tm_k, full, cb * 64,
+                                    G.h, t.kt * kN, t.j, G.b);
                 }
+                if (ok) ++tile_it;
             }
         }
         if (!ok) {
             give_up(abort, status);
-            // let the copies already issued land before the CTA can exit
-            const uint32_t first = slot_it > kSlots ? slot_it - kSlots : 0;
-            for (uint32_t x = first; x < slot_it; ++x)
-                mbar_wait(&sm.slot_full[x % kSlots], (x / kSlots) & 1, timeout, nullptr);
+            // let the copies already issued land before the CTA can exit (if the last tile's V
+            // copy was never issued, its wait runs out after the K copy has landed)
+            if (tile_it > 0) mbar_wait(&sm.kv_full[(tile_it - 1) & 1], ((tile_it - 1) >> 1) & 1, timeout, nullptr);
+            mbar_wait(&sm.kv_full[tile_it & 1], (tile_it >> 1) & 1, timeout, nullptr);
             if (q_it > 0) mbar_wait(&sm.q_full, (q_it - 1) & 1, timeout, nullptr);
         }
     }
@@ -265,7 +267,7 @@ struct Roles {
     }
 
     __device__ void mma() {
-        uint32_t cons_it = 0, q_it = 0, p_cnt[2] = {0, 0}, act_items[2] = {0, 0};
+        uint32_t tile_it = 0, q_it = 0, p_cnt[2] = {0, 0}, act_items[2] = {0, 0};
         bool ok = true;
         auto wait = [&](uint64_t* bar, uint32_t parity) {
             if (!ok) return false;
@@ -273,17 +275,18 @@ struct Roles {
             if (ok) tc_fence_after();
             return ok;
         };
+        auto& wait_tma = wait;  // K/V/Q tiles landed (TMA)
         for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
             const ItemGeom G = item_geom(L, items[it]);
             TileIter cur;
             cur.init(A, L, G);
             if (!cur.valid) continue;
-            if (!wait(&sm.q_full, q_it & 1)) break;
+            if (!wait_tma(&sm.q_full, q_it & 1)) break;
             ++q_it;
             bool first_pv[2] = {true, true}, any_act[2] = {false, false};
-            uint32_t kslot = cons_it % kSlots;
-            if (!wait(&sm.slot_full[kslot], (cons_it / kSlots) & 1)) break;
-            ++cons_it;
+            // one wait per key tile: K and V of tile n complete the same barrier
+            if (!wait_tma(&sm.kv_full[tile_it & 1], (tile_it >> 1) & 1)) break;
+            uint32_t kslot = (2 * tile_it) % kSlots;
             for (int q = 0; q < 2; ++q)
                 if (cur.act(q)) {
                     issue_s(q, kslot);
@@ -294,9 +297,7 @@ struct Roles {
             nxt.next(L, A.causal, G);
             if (!nxt.valid) mma_commit(&sm.q_empty);
             for (;;) {
-                const uint32_t vslot = cons_it % kSlots;
-                if (!wait(&sm.slot_full[vslot], (cons_it / kSlots) & 1)) break;
-                ++cons_it;
+                const uint32_t vslot = (2 * tile_it + 1) % kSlots;  // landed with K of this tile
                 for (int q = 0; q < 2; ++q) {
                     if (cur.act(q)) {
                         if (!wait(&sm.p_full[q], p_cnt[q] & 1)) break;
@@ -308,9 +309,8 @@ struct Roles {
                         first_pv[q] = false;
                     }
                     if (q == 0 && nxt.valid) {
-                        kslot = cons_it % kSlots;
-                        if (!wait(&sm.slot_full[kslot], (cons_it / kSlots) & 1)) break;
-                        ++cons_it;
+                        if (!wait_tma(&sm.kv_full[(tile_it + 1) & 1], ((tile_it + 1) >> 1) & 1)) break;
+                        kslot = (2 * (tile_it + 1)) % kSlots;
                         if (nxt.act(0)) {
                             issue_s(0, kslot);
                             any_act[0] = true;
@@ -326,10 +326,12 @@ struct Roles {
                 }
                 mma_commit(&sm.slot_empty[kslot]);
                 cur = nxt;
+                ++tile_it;
                 nxt.next(L, A.causal, G);
                 if (!nxt.valid) mma_commit(&sm.q_empty);
             }
             if (!ok) break;
+            ++tile_it;  // past the item's last key tile
             for (int q = 0; q < 2; ++q)
                 if (any_act[q]) {
                     mma_commit(&sm.o_final[q]);
@@ -547,10 +549,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_init(&sm.q_full, 1);
         mbar_init(&sm.q_empty, 1);
         mbar_init(&sm.drain, 1);
-        for (int k = 0; k < kSlots; ++k) {
-            mbar_init(&sm.slot_full[k], 1);
-            mbar_init(&sm.slot_empty[k], 1);
-        }
+        mbar_init(&sm.kv_full[0], 1);
+        mbar_init(&sm.kv_full[1], 1);
+        for (int k = 0; k < kSlots; ++k) mbar_init(&sm.slot_empty[k], 1);
         for (int q = 0; q < 2; ++q) {
             mbar_init(&sm.s_full[q], 1);
             mbar_init(&sm.p_full[q], kM);
@@ -574,9 +575,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
 
     Roles<kD> roles{sm, A, items, n_items, timeout_ns, status, &sm.abort, sm.tmem_base, narrow(A.L)};
-    // register split: 256 softmax threads x 208 + 128 producer/MMA threads x 80 = 63488 <= 384 x 168
+    // register split: 256 softmax threads x 184 + 128 producer/MMA threads x 112 = 61440 <= 384 x 168
     if (warp >= 8) {
-        setmaxnreg_dec80();
+        setmaxnreg_dec112();
         if (warp == kLoadWarp) {
             if (lane == 0) roles.producer(&tm_q, &tm_k, &tm_v, debug);
             __syncwarp();
@@ -585,7 +586,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             __syncwarp();
         }
     } else {
-        setmaxnreg_inc208();
+        setmaxnreg_inc184();
         roles.softmax(warp >> 2, warp, threadIdx.x & 127);
     }
 

@@ -59,6 +59,19 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
     return ok != 0;
 }
 
+// Non-blocking probe: has the phase with the given parity completed?
+__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_addr(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
 // Wait for the phase with the given parity to complete, giving up after timeout_ns or as soon as
 // *abort is set by another role.  Returns false on give-up (the caller unwinds).
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint64_t timeout_ns,
@@ -264,8 +277,8 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
     return d;
 }
 
-__device__ __forceinline__ void setmaxnreg_inc208() { asm volatile("setmaxnreg.inc.sync.aligned.u32 208;"); }
-__device__ __forceinline__ void setmaxnreg_dec80() { asm volatile("setmaxnreg.dec.sync.aligned.u32 80;"); }
+__device__ __forceinline__ void setmaxnreg_inc184() { asm volatile("setmaxnreg.inc.sync.aligned.u32 184;"); }
+__device__ __forceinline__ void setmaxnreg_dec112() { asm volatile("setmaxnreg.dec.sync.aligned.u32 112;"); }
 
 }  // namespace sm100
 }  // namespace ra
