@@ -462,7 +462,8 @@ struct Roles {
                     }
                     tmem_wait_st();
                     tc_fence_before();
-                    mbar_arrive(&sm.p_full[q]);
+                    __syncwarp();
+                    if ((threadIdx.x & 31) == 0) mbar_arrive(&sm.p_full[q]);
                     ++n_act;
                 }
             }
@@ -501,7 +502,8 @@ struct Roles {
                 if (row_ok) store_chunk(row_dst, c, o, inv_l);
             }
             tc_fence_before();
-            mbar_arrive(&sm.o_free[q]);
+            __syncwarp();
+            if ((threadIdx.x & 31) == 0) mbar_arrive(&sm.o_free[q]);
         } else if (row_ok) {
             uint32_t o[32];
 #pragma unroll
@@ -554,9 +556,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int k = 0; k < kSlots; ++k) mbar_init(&sm.slot_empty[k], 1);
         for (int q = 0; q < 2; ++q) {
             mbar_init(&sm.s_full[q], 1);
-            mbar_init(&sm.p_full[q], kM);
+            mbar_init(&sm.p_full[q], 4);  // one arrival per softmax warp
             mbar_init(&sm.o_final[q], 1);
-            mbar_init(&sm.o_free[q], kM);
+            mbar_init(&sm.o_free[q], 4);
         }
         sm.abort = 0;
         fence_barrier_init();
