@@ -35,6 +35,24 @@ METRIC = "ring-attn fwd TFLOP/s (bf16, causal) and % of B200 dense BF16 tensor p
 UNIT = "TFLOP/s"
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
+# DRAM bytes (read + write) per attention launch on s128k, from an ncu capture of the 4-head case
+# scaled by heads (profiles/attn_tc_fused_s128k_striped.md); valid only for the kernel source whose
+# sha256 starts with the recorded prefix -- any other source reports traffic as null.
+TRAFFIC_RECORD = {"attn_tc_sha256_prefix": "cd8e775b99814d1c", "bytes_per_launch": 8.50e9 * 8}
+
+
+def recorded_traffic(args):
+    import hashlib
+    src = os.path.join(ROOT, "long_context_exact_forward_b200", "csrc", "attn_tc.cu")
+    try:
+        digest = hashlib.sha256(open(src, "rb").read()).hexdigest()
+    except OSError:
+        return None
+    default_run = args.workload == "s128k" and args.layout == "striped" and args.heads in (0, 32)
+    if default_run and digest.startswith(TRAFFIC_RECORD["attn_tc_sha256_prefix"]):
+        return TRAFFIC_RECORD["bytes_per_launch"]
+    return None
+
 
 def attention_flops(B, H, S, D, causal):
     """4 * B * H * S^2 * D, halved when causal (the convention of the target metric)."""
@@ -116,12 +134,18 @@ def dist_env():
     return world, rank, local
 
 
-def max_over_ranks(x, world):
+def max_over_ranks(x, world, device="cuda"):
+    """The slowest rank's value (timings are reported as the max over ranks)."""
     if world == 1:
         return x
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    t = torch.tensor([x], dtype=torch.float64, device=device)
     torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
     return t.item()
+
+
+def job_throughput(flops_per_rank, world, ms_per_step):
+    """Whole-job TFLOP/s: every rank's work over the slowest rank's time (weak scaling)."""
+    return world * flops_per_rank / (ms_per_step / 1e3) / 1e12
 
 
 def barrier(world):
@@ -182,6 +206,48 @@ def config_dict(w, args):
     }
 
 
+def hbm_kernels(ra, q, n_ring, layout, stream, reps=10):
+    """Achieved DRAM bandwidth of the permute and merge kernels against the measured copy peak.
+
+    permute: q [B, S, H, D] bf16 -> shard-major copy; algorithmic bytes = read + write of q.
+    merge:   one ring step's partial folded into the running result (fp32 [B*S*H, D] and
+             lse [B*S*H]); algorithmic bytes = 12 per output element + 12 per row.
+    """
+    peaks, src = load_peaks()
+    res = {"peak_gbs": peaks["hbm_gbs"], "peak_kind": f"copy ({src})"}
+    y = torch.empty((q.shape[0], n_ring, q.shape[1] // n_ring, q.shape[2], q.shape[3]), dtype=q.dtype,
+                    device=q.device)
+    lay = layout if layout != "contiguous" else "striped"
+
+    def timed(fn):
+        fn()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(reps):
+            fn()
+        b.record(stream)
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) / reps
+
+    ms = timed(lambda: ra.permute(q, n_ring, lay, out=y, stream=stream))
+    byts = 2.0 * q.numel() * q.element_size()
+    res["permute"] = {"layout": lay, "ms": ms, "bytes": byts, "achieved_gbs": byts / ms / 1e6,
+                      "frac": byts / ms / 1e6 / peaks["hbm_gbs"]}
+    del y
+    rows, D = q.numel() // q.shape[-1], q.shape[-1]
+    g = torch.Generator(device=q.device).manual_seed(0)
+    O_r = torch.randn(rows, D, device=q.device, generator=g)
+    O_s = torch.randn(rows, D, device=q.device, generator=g)
+    l_r = torch.randn(rows, device=q.device, generator=g)
+    l_s = torch.randn(rows, device=q.device, generator=g)
+    ms = timed(lambda: ra.merge_partials(O_r, l_r, O_s, l_s, stream=stream))
+    byts = 12.0 * rows * D + 12.0 * rows
+    res["merge"] = {"rows": rows, "D": D, "ms": ms, "bytes": byts, "achieved_gbs": byts / ms / 1e6,
+                    "frac": byts / ms / 1e6 / peaks["hbm_gbs"]}
+    return res
+
+
 # ------------------------------------------------------------------ our arm
 def run_ours(args, w):
     import long_context_exact_forward_b200 as ra
@@ -226,7 +292,7 @@ def run_ours(args, w):
     kernel_ms = [a.elapsed_time(b) for a, b in kev]
     status = ra.get_device_status()
     ms_per_step = ms / args.steps
-    value = world * flops / (ms_per_step / 1e3) / 1e12
+    value = job_throughput(flops, world, ms_per_step)
 
     # ---- end to end through the public API: pinned host inputs in, result back to the host
     e2e = None
@@ -257,9 +323,15 @@ def run_ours(args, w):
         ems = max_over_ranks(e0.elapsed_time(e1), world) / args.steps
         bi = 3 * q.numel() * q.element_size()
         bo = out.numel() * out.element_size() + lse.numel() * lse.element_size()
-        e2e = {"value": world * flops / (ems / 1e3) / 1e12, "unit": UNIT, "h2d_bytes_per_step": bi,
+        e2e = {"value": job_throughput(flops, world, ems), "unit": UNIT, "h2d_bytes_per_step": bi,
                "d2h_bytes_per_step": bo, "ms_per_step": ems}
         del qh, kh, vh, oh, lh, qd, kd, vd
+
+    # ---- the HBM-bound kernels (permute of q into shard-major order; one per-step merge),
+    #      timed alone on this workload's sizes, outside the timed region
+    hbm = None
+    if not args.no_hbm_kernels:
+        hbm = hbm_kernels(ra, q, N, args.layout, stream)
 
     # ---- roofline of the dominant kernel (the attention kernel)
     peaks, peak_src = load_peaks()
@@ -268,7 +340,7 @@ def run_ours(args, w):
     peak = peaks["bf16_tflops_sustained"]
     roofline = {
         "bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
-        "traffic": args.traffic_bytes,
+        "traffic": args.traffic_bytes if args.traffic_bytes is not None else recorded_traffic(args),
         "peak_kind": f"bf16 dense cuBLAS, sustained ({peak_src})",
         "frac_of_burst_peak": achieved / peaks["bf16_tflops"],
         "kernel": "attn_tc_kernel<128> (fused ring, tcgen05)", "kernel_ms": k_ms,
@@ -294,7 +366,7 @@ def run_ours(args, w):
         "pct_of_bf16_peak": {"burst_measured": value / world / peaks["bf16_tflops"],
                              "sustained_measured": value / world / peaks["bf16_tflops_sustained"],
                              "nvidia_dense_spec_2250": value / world / 2250.0},
-        "clocks": clk, "e2e": e2e, "roofline": roofline, "cpu_baseline": cpu,
+        "clocks": clk, "e2e": e2e, "roofline": roofline, "cpu_baseline": cpu, "hbm_kernels": hbm,
         "gpu_launches": launches_per_step * args.steps, "device_status": status,
     }
     if rank == 0:
@@ -315,6 +387,7 @@ def main():
     ap.add_argument("--heads", type=int, default=0, help="override the head count (profiling runs)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-hbm-kernels", action="store_true")
     ap.add_argument("--cpu-rows", type=int, default=256, help="oracle rows per head for cpu_baseline")
     ap.add_argument("--ref-rows", type=int, default=64, help="oracle rows per head per reference step")
     ap.add_argument("--traffic-bytes", type=float, default=None,
