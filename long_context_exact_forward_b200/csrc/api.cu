@@ -207,6 +207,7 @@ int flat_items(int64_t B, int64_t H, const Layout& L, int causal, bool per_step,
 enum Kernel { kTC, kSIMT };
 
 struct Workspace {
+    size_t counters = 0, n_counters = 0;  // one work counter per attention launch (zeroed per call)
     size_t items = 0, n_items_total = 0;
     size_t qp = 0, kp = 0, vp = 0;  // permuted q, k, v
     size_t O_run = 0, lse_run = 0, O_step = 0, lse_step = 0;
@@ -227,6 +228,9 @@ Workspace carve(int64_t B, int64_t H, const Layout& L, int64_t D, int causal, in
         } else {
             w.n_items_total = plan_items(B, H, L, causal, 0, (int)L.N).size();
         }
+        w.counters = off;
+        w.n_counters = w.per_step ? (size_t)L.N : 1;
+        off = align_up(off + w.n_counters * sizeof(int));
         w.items = off;
         off = align_up(off + w.n_items_total * sizeof(int4));
         w.permute = (L.kind != RA_LAYOUT_CONTIGUOUS);
@@ -387,6 +391,8 @@ int run_forward(const Call& c, const ra_options& opt) {
             (e = cudaMemcpyAsync(ws + w.items, fl->data, fl->count * sizeof(int4),
                                  cudaMemcpyHostToDevice, c.stream)) != cudaSuccess)
             return finish(cuda_fail(e, "work list upload"));
+        if ((e = cudaMemsetAsync(ws + w.counters, 0, w.n_counters * sizeof(int), c.stream)) != cudaSuccess)
+            return finish(cuda_fail(e, "work counter reset"));
         tc.timeout_ns = opt.timeout_ns ? opt.timeout_ns : 2000000000ull;
         tc.debug = opt.debug;
         tc.status = dev.status;
@@ -405,6 +411,7 @@ int run_forward(const Call& c, const ra_options& opt) {
             t.items = reinterpret_cast<const int4*>(ws + w.items) + step_item_offset[list];
             t.n_items = step_item_offset[list + 1] - step_item_offset[list];
             t.grid = std::max(1, std::min(t.n_items, dev.sms));
+            t.counter = reinterpret_cast<int*>(ws + w.counters) + list;
             return ra::launch_attn_tc(a, t, c.stream);
         }
         return ra::launch_attn_simt(q, k, v, a, c.stream);

@@ -18,7 +18,8 @@
 // longest prefix of the query tile are never loaded (block skip), tiles inside every row's prefix
 // run unmasked, and only the tile holding a row's prefix end is masked.
 //
-// Layout of one CTA (384 threads, one CTA per SM, persistent over a static slice of the work list):
+// Layout of one CTA (384 threads, one CTA per SM, persistent; items are taken from a launch-wide
+// counter, heaviest first):
 //   warps 0-3  softmax for query tile 0 (thread t owns row t = TMEM lane t)
 //   warps 4-7  softmax for query tile 1
 //   warp  8    TMA producer: Q tiles, then K and V tiles into a ring of 4 shared-memory slots
@@ -101,6 +102,8 @@ struct TcSmem {
     uint64_t kv_full[2];              // K and V of key tile n have landed (barrier n % 2)
     uint64_t slot_empty[kSlots];      // key tile n uses slots 2n and 2n+1 (mod kSlots)
     uint64_t s_full[2], p_full[2], o_final[2], o_free[2];
+    uint64_t item_full[2], item_empty[2];  // ring of work-item indices handed out by the load warp
+    int item_idx[2];
     uint32_t tmem_base;
     int abort;
 };
@@ -195,14 +198,24 @@ struct Roles {
     volatile int* abort;
     uint32_t tmem;
     Layout32 L;
+    int* counter;  // next work item of this launch (zeroed by the host before the launch)
 
     // ------------------------------------------------------------ TMA producer (one thread)
     __device__ void producer(const CUtensorMap* tm_q, const CUtensorMap* tm_k,
                              const CUtensorMap* tm_v, int debug) {
-        uint32_t tile_it = 0, q_it = 0;
+        uint32_t tile_it = 0, q_it = 0, armed = 0;
         bool ok = true;
-        for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
-            const ItemGeom G = item_geom(L, items[it]);
+        // Dynamic schedule: take the next item from the launch-wide counter and publish its index
+        // to the other roles through a two-entry ring (index -1 ends the loop).
+        for (uint32_t k = 0; ok; ++k) {
+            const uint32_t b = k & 1;
+            if (!mbar_wait(&sm.item_empty[b], ((k >> 1) & 1) ^ 1, timeout, abort)) { ok = false; break; }
+            int idx = atomicAdd(counter, 1);
+            if (idx >= n_items) idx = -1;
+            sm.item_idx[b] = idx;
+            mbar_arrive(&sm.item_full[b]);
+            if (idx < 0) break;
+            const ItemGeom G = item_geom(L, items[idx]);
             TileIter t;
             t.init(A, L, G);
             if (!t.valid) continue;
@@ -223,7 +236,10 @@ struct Roles {
                         ok = false;
                         break;
                     }
-                    if (w == 0) mbar_arrive_expect_tx(full, 2 * TcSmem<kD>::kTileBytes);
+                    if (w == 0) {
+                        mbar_arrive_expect_tx(full, 2 * TcSmem<kD>::kTileBytes);
+                        armed = tile_it + 1;
+                    }
                     for (int cb = 0; cb < kD / 64; ++cb)
                         tma_load_5d(sm.kv[slot] + cb * kColBlockBytes, w ? tm_v : tm_k, full, cb * 64,
                                     G.h, t.kt * kN, t.j, G.b);
@@ -236,7 +252,7 @@ struct Roles {
             // let the copies already issued land before the CTA can exit (if the last tile's V
             // copy was never issued, its wait runs out after the K copy has landed)
             if (tile_it > 0) mbar_wait(&sm.kv_full[(tile_it - 1) & 1], ((tile_it - 1) >> 1) & 1, timeout, nullptr);
-            mbar_wait(&sm.kv_full[tile_it & 1], (tile_it >> 1) & 1, timeout, nullptr);
+            if (armed > tile_it) mbar_wait(&sm.kv_full[tile_it & 1], (tile_it >> 1) & 1, timeout, nullptr);
             if (q_it > 0) mbar_wait(&sm.q_full, (q_it - 1) & 1, timeout, nullptr);
         }
     }
@@ -276,8 +292,13 @@ struct Roles {
             return ok;
         };
         auto& wait_tma = wait;  // K/V/Q tiles landed (TMA)
-        for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
-            const ItemGeom G = item_geom(L, items[it]);
+        for (uint32_t k = 0; ok; ++k) {
+            const uint32_t b = k & 1;
+            if (!wait(&sm.item_full[b], (k >> 1) & 1)) break;
+            const int idx = sm.item_idx[b];
+            mbar_arrive(&sm.item_empty[b]);
+            if (idx < 0) break;
+            const ItemGeom G = item_geom(L, items[idx]);
             TileIter cur;
             cur.init(A, L, G);
             if (!cur.valid) continue;
@@ -358,8 +379,14 @@ struct Roles {
             if (ok) tc_fence_after();
             return ok;
         };
-        for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
-            const ItemGeom G = item_geom(L, items[it]);
+        for (uint32_t k = 0; ok; ++k) {
+            const uint32_t b = k & 1;
+            if (!wait_all(&sm.item_full[b], (k >> 1) & 1)) break;
+            const int idx = sm.item_idx[b];
+            __syncwarp();
+            if ((threadIdx.x & 31) == 0) mbar_arrive(&sm.item_empty[b]);
+            if (idx < 0) break;
+            const ItemGeom G = item_geom(L, items[idx]);
             const int a = G.a0[q] + row;
             float m_run = -INFINITY, l = 0.f;
             int n_act = 0;
@@ -540,8 +567,8 @@ template <int kD>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const AttnArgs A,
-                   const int4* __restrict__ items, int n_items, uint64_t timeout_ns, int debug,
-                   int* status) {
+                   const int4* __restrict__ items, int n_items, int* counter, uint64_t timeout_ns,
+                   int debug, int* status) {
     extern __shared__ uint8_t smem_raw[];
     TcSmem<kD>& sm = *reinterpret_cast<TcSmem<kD>*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -554,6 +581,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_init(&sm.kv_full[0], 1);
         mbar_init(&sm.kv_full[1], 1);
         for (int k = 0; k < kSlots; ++k) mbar_init(&sm.slot_empty[k], 1);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&sm.item_full[b], 1);
+            mbar_init(&sm.item_empty[b], 9);  // the MMA thread + one lane of each softmax warp
+        }
         for (int q = 0; q < 2; ++q) {
             mbar_init(&sm.s_full[q], 1);
             mbar_init(&sm.p_full[q], 4);  // one arrival per softmax warp
@@ -576,7 +607,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     tc_fence_after();
 
-    Roles<kD> roles{sm, A, items, n_items, timeout_ns, status, &sm.abort, sm.tmem_base, narrow(A.L)};
+    Roles<kD> roles{sm, A, items, n_items, timeout_ns, status, &sm.abort, sm.tmem_base, narrow(A.L), counter};
     // register split: 256 softmax threads x 184 + 128 producer/MMA threads x 112 = 61440 <= 384 x 168
     if (warp >= 8) {
         setmaxnreg_dec112();
@@ -612,7 +643,7 @@ cudaError_t launch_attn_tc(const AttnArgs& a, const TcLaunch& t, cudaStream_t st
     auto kern = (a.D == 64) ? attn_tc_kernel<64> : attn_tc_kernel<128>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    kern<<<t.grid, kThreads, smem, stream>>>(t.tm_q, t.tm_k, t.tm_v, a, t.items, t.n_items,
+    kern<<<t.grid, kThreads, smem, stream>>>(t.tm_q, t.tm_k, t.tm_v, a, t.items, t.n_items, t.counter,
                                              t.timeout_ns, t.debug, t.status);
     return cudaGetLastError();
 }

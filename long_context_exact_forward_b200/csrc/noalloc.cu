@@ -13,9 +13,10 @@
 // Rules of use.
 //   * The first call on a device looks up the array's device address (cudaGetSymbolAddress) with
 //     that device current; make that first call before any stream capture.
-//   * Every call on a device shares the one array and leaves its contents behind.  Nothing in it
-//     has to start at zero: each call rewrites the parts it reads.  Calls whose GPU work overlaps
-//     (different streams, or concurrent host threads) race on the array and corrupt each other.
+//   * Every call on a device shares the one array and leaves its contents behind.  The one part
+//     that must start at zero, the kernel's work counter, is cleared by each call on its stream
+//     (cudaMemsetAsync, no allocation); everything else is rewritten before it is read.  Calls
+//     whose GPU work overlaps (different streams, or concurrent host threads) race on the array.
 //   * Problems whose scratch exceeds the array are rejected with RA_ERR_NO_WORKSPACE (message in
 //     ra_last_error_string); nothing is enqueued then.
 #include <cuda.h>
@@ -120,8 +121,9 @@ extern "C" int ra_forward_noalloc(const void* q, const void* k, const void* v, v
     const int64_t n_items = B * H * per_head;
     const size_t tensor_bytes = (size_t)(B * S * H * D) * 2;
     const bool permute = (layout != RA_LAYOUT_CONTIGUOUS);
+    const size_t counter_bytes = 256;  // the persistent kernel's work counter, zeroed every call
     const size_t items_bytes = align256((size_t)n_items * sizeof(int4));
-    const size_t need = items_bytes + (permute ? 3 * align256(tensor_bytes) : 0);
+    const size_t need = counter_bytes + items_bytes + (permute ? 3 * align256(tensor_bytes) : 0);
     if (per_head > kMaxItemsPerHead || need > kScratchBytes || n_items > INT32_MAX) {
         ra::host_set_error("ra_forward_noalloc: problem needs more scratch than the fixed "
                            "RA_NOALLOC_SCRATCH_BYTES array (or more than 12288 work items per head)");
@@ -131,15 +133,18 @@ extern "C" int ra_forward_noalloc(const void* q, const void* k, const void* v, v
     if ((rc = scratch_address(&scratch)) != RA_OK) return rc;
     cudaStream_t stream = static_cast<cudaStream_t>(stream_handle);
 
-    int4* items = reinterpret_cast<int4*>(scratch);
+    int* counter = reinterpret_cast<int*>(scratch);
+    int4* items = reinterpret_cast<int4*>(scratch + counter_bytes);
+    cudaError_t e = cudaMemsetAsync(counter, 0, sizeof(int), stream);
+    if (e != cudaSuccess) return ra::host_cuda_fail(e, "work counter reset");
     const size_t smem = (size_t)per_head * sizeof(int);
     build_work_list<<<1, 1024, smem, stream>>>(items, B * H, H, L, causal ? 1 : 0, pairs);
-    cudaError_t e = cudaGetLastError();
+    e = cudaGetLastError();
     if (e != cudaSuccess) return ra::host_cuda_fail(e, "work list launch");
 
     const void *qs = q, *ks = k, *vs = v;
     if (permute) {
-        unsigned char* base = scratch + items_bytes;
+        unsigned char* base = scratch + counter_bytes + items_bytes;
         void* dst[3] = {base, base + align256(tensor_bytes), base + 2 * align256(tensor_bytes)};
         const void* src[3] = {q, k, v};
         if ((e = ra::launch_permute(src, dst, 3, B, L, H, D, 2, false, stream)) != cudaSuccess)
@@ -154,6 +159,7 @@ extern "C" int ra_forward_noalloc(const void* q, const void* k, const void* v, v
     if ((rc = ra::host_encode_qkv_map(&t.tm_v, vs, B, L, H, D)) != RA_OK) return rc;
     t.items = items;
     t.n_items = (int)n_items;
+    t.counter = counter;
     t.grid = (int)(n_items < sms ? n_items : sms);
     t.timeout_ns = 2000000000ull;
     t.debug = 0;

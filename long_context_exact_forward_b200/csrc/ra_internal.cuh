@@ -48,6 +48,7 @@ struct TcLaunch {
     CUtensorMap tm_q, tm_k, tm_v;
     const int4* items;     // work list (b, h, i, pair), heaviest first
     int n_items;
+    int* counter;          // zero before the launch; CTAs take items in list order
     int grid;
     uint64_t timeout_ns;
     int debug;
