@@ -38,7 +38,7 @@ PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # DRAM bytes (read + write) per attention launch on s128k, from an ncu capture of the 4-head case
 # scaled by heads (profiles/attn_tc_fused_s128k_striped.md); valid only for the kernel source whose
 # sha256 starts with the recorded prefix -- any other source reports traffic as null.
-TRAFFIC_RECORD = {"attn_tc_sha256_prefix": "cd8e775b99814d1c", "bytes_per_launch": 8.50e9 * 8}
+TRAFFIC_RECORD = {"attn_tc_sha256_prefix": "971a67f661c562ad", "bytes_per_launch": 3.903e9 * 8}
 
 
 def recorded_traffic(args):
