@@ -148,11 +148,14 @@ RA_API int ra_layout_positions(int64_t S, int n_ring, int layout, int64_t* pos);
  * ragged last key tile, which is PARTIAL. */
 RA_API int ra_plan_tiles(int64_t S, int n_ring, int layout, int causal, int tile, int8_t* cls);
 
-/* ra_plan_items (host only): the fused kernel's work list, heaviest first (LPT).  Each item is
- * four int32 (b, h, shard i, query-tile pair p) followed by its cost in live key/value tiles
- * (int32), 5 entries per item.  Writes at most cap items; *n_items receives the full count. */
-RA_API int ra_plan_items(int64_t B, int64_t H, int64_t S, int n_ring, int causal, int layout,
-                  int32_t* items, int64_t cap, int64_t* n_items);
+/* ra_plan_items (host only): the fused kernel's work list, in the order CTAs take it.  Each item
+ * is four int32 (b, h, shard i, query-tile pair p) followed by its cost in live key/value tiles
+ * (int32), 5 entries per item.  Items are (b, h) major; inside a head they are heaviest first
+ * (LPT), except that when one head's keys and values (4*S*D bytes) exceed 96 MB the items of each
+ * shard are grouped (groups heaviest first, LPT inside).  Writes at most cap items; *n_items
+ * receives the full count. */
+RA_API int ra_plan_items(int64_t B, int64_t H, int64_t S, int64_t D, int n_ring, int causal,
+                         int layout, int32_t* items, int64_t cap, int64_t* n_items);
 
 /* RA_NOALLOC_SCRATCH_BYTES: size of the fixed device array that ra_forward_noalloc uses as
  * scratch.  Every GPU that loads the library holds this much device memory until the process
@@ -171,7 +174,8 @@ RA_API int ra_plan_items(int64_t B, int64_t H, int64_t S, int n_ring, int causal
  *   - All calls on a device share the array and leave their data in it; calls whose GPU work
  *     overlaps (other streams, other host threads) race on it.
  *   - A problem whose scratch does not fit (B*H*n_ring*ceil(S_loc/256) work items of 16 bytes,
- *     plus 3*B*S*H*D*2 bytes for striped/zigzag, at most 12288 items per head) is rejected with
+ *     plus 3*B*S*H*D*2 bytes for striped/zigzag and 256 bytes of counter, at most 11264 items per
+ *     head) is rejected with
  *     RA_ERR_NO_WORKSPACE and a message in ra_last_error_string; nothing is enqueued.
  *   - Other dtypes or head dims return RA_ERR_UNSUPPORTED. */
 RA_API int ra_forward_noalloc(const void* q, const void* k, const void* v, void* out, float* lse,

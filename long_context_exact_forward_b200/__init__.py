@@ -13,7 +13,7 @@ Entry points (same names as the C ABI):
     merge_partials(O_run, lse_run, O_step, lse_step)                     ra_merge_partials
     layout_positions(S, n_ring, layout)              -> np.ndarray      ra_layout_positions
     plan_tiles(S, n_ring, layout, causal, tile)      -> np.ndarray      ra_plan_tiles
-    plan_items(B, H, S, n_ring, causal, layout)      -> np.ndarray      ra_plan_items
+    plan_items(B, H, S, n_ring, causal, layout, D)   -> np.ndarray      ra_plan_items
     get_device_status()                              -> int             ra_get_device_status
 """
 import ctypes
@@ -81,7 +81,7 @@ def lib():
         L.ra_forward_noalloc.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i64, ci, ci, ci, vp]
         L.ra_layout_positions.argtypes = [i64, ci, ci, vp]
         L.ra_plan_tiles.argtypes = [i64, ci, ci, ci, ci, vp]
-        L.ra_plan_items.argtypes = [i64, i64, i64, ci, ci, ci, vp, i64, ctypes.POINTER(ctypes.c_int64)]
+        L.ra_plan_items.argtypes = [i64, i64, i64, i64, ci, ci, ci, vp, i64, ctypes.POINTER(ctypes.c_int64)]
         L.ra_status_string.restype = ctypes.c_char_p
         L.ra_status_string.argtypes = [ci]
         L.ra_last_error_string.restype = ctypes.c_char_p
@@ -256,12 +256,12 @@ def plan_tiles(S, n_ring, layout, causal, tile):
     return cls
 
 
-def plan_items(B, H, S, n_ring, causal, layout):
+def plan_items(B, H, S, n_ring, causal, layout, D=128):
     n = ctypes.c_int64(0)
-    _check(lib().ra_plan_items(B, H, S, n_ring, int(bool(causal)), LAYOUTS[layout], None, 0,
+    _check(lib().ra_plan_items(B, H, S, D, n_ring, int(bool(causal)), LAYOUTS[layout], None, 0,
                                ctypes.byref(n)), "ra_plan_items")
     items = np.empty((n.value, 5), dtype=np.int32)
-    _check(lib().ra_plan_items(B, H, S, n_ring, int(bool(causal)), LAYOUTS[layout],
+    _check(lib().ra_plan_items(B, H, S, D, n_ring, int(bool(causal)), LAYOUTS[layout],
                                items.ctypes.data, n.value, ctypes.byref(n)), "ra_plan_items")
     return items
 

@@ -111,9 +111,10 @@ int tc_tiles_for(const Layout& L, int causal, int64_t i, int64_t a0, int64_t j) 
 struct PlanKey {
     int64_t B, H, S;
     int n_ring, causal, layout, s_begin, s_end;
+    int64_t D;
     bool operator<(const PlanKey& o) const {
-        return std::tie(B, H, S, n_ring, causal, layout, s_begin, s_end) <
-               std::tie(o.B, o.H, o.S, o.n_ring, o.causal, o.layout, o.s_begin, o.s_end);
+        return std::tie(B, H, S, n_ring, causal, layout, s_begin, s_end, D) <
+               std::tie(o.B, o.H, o.S, o.n_ring, o.causal, o.layout, o.s_begin, o.s_end, o.D);
     }
 };
 
@@ -124,12 +125,13 @@ struct PlanItem {
 // Work list of the tensor-core kernel for ring steps [s_begin, s_end): one item per
 // (b, h, shard i, pair of 128-row query tiles), cost = live (query tile, key tile) pairs.
 // Order: (b, h) major so that CTAs running at the same time share one head's keys and values in
-// L2; inside a head, heaviest first (LPT) so the short items fill the tail.
-const std::vector<PlanItem>& plan_items(int64_t B, int64_t H, const Layout& L, int causal,
-                                        int s_begin, int s_end) {
+// L2; inside a head, heaviest first (LPT) so the short items fill the tail -- or, when one head's
+// K/V exceeds L2 (plan_groups_by_shard), shard groups heaviest first and LPT inside a group.
+const std::vector<PlanItem>& plan_items(int64_t B, int64_t H, const Layout& L, int64_t D_for_plan,
+                                        int causal, int s_begin, int s_end) {
     static std::mutex mu;
     static std::map<PlanKey, std::vector<PlanItem>> cache;
-    PlanKey key{B, H, L.S, (int)L.N, causal, L.kind, s_begin, s_end};
+    PlanKey key{B, H, L.S, (int)L.N, causal, L.kind, s_begin, s_end, D_for_plan};
     std::lock_guard<std::mutex> lock(mu);
     auto it = cache.find(key);
     if (it != cache.end()) return it->second;
@@ -146,8 +148,22 @@ const std::vector<PlanItem>& plan_items(int64_t B, int64_t H, const Layout& L, i
             }
             head.push_back(PlanItem{0, 0, (int32_t)i, (int32_t)p, (int32_t)std::min<int64_t>(cost, INT32_MAX)});
         }
-    std::stable_sort(head.begin(), head.end(),
-                     [](const PlanItem& x, const PlanItem& y) { return x.cost > y.cost; });
+    if (ra::plan_groups_by_shard(L.S, D_for_plan)) {
+        // one head's K/V does not fit L2: group the items of one shard (they walk the same ring
+        // sequence of key/value blocks, so CTAs running together share tiles in L2), groups
+        // heaviest first, items heaviest first inside a group
+        std::vector<int64_t> group_cost((size_t)L.N, 0);
+        for (const PlanItem& x : head) group_cost[(size_t)x.i] += x.cost;
+        std::stable_sort(head.begin(), head.end(), [&](const PlanItem& x, const PlanItem& y) {
+            if (group_cost[(size_t)x.i] != group_cost[(size_t)y.i])
+                return group_cost[(size_t)x.i] > group_cost[(size_t)y.i];
+            if (x.i != y.i) return x.i < y.i;
+            return x.cost > y.cost;
+        });
+    } else {
+        std::stable_sort(head.begin(), head.end(),
+                         [](const PlanItem& x, const PlanItem& y) { return x.cost > y.cost; });
+    }
     std::vector<PlanItem> all;
     all.reserve(head.size() * (size_t)(B * H));
     for (int64_t b = 0; b < B; ++b)
@@ -169,10 +185,11 @@ struct FlatList {
     std::vector<int> offsets;
 };
 
-int flat_items(int64_t B, int64_t H, const Layout& L, int causal, bool per_step, const FlatList** out) {
+int flat_items(int64_t B, int64_t H, const Layout& L, int64_t D, int causal, bool per_step,
+               const FlatList** out) {
     static std::mutex mu;
     static std::map<std::pair<PlanKey, bool>, FlatList> cache;
-    const PlanKey key{B, H, L.S, (int)L.N, causal, L.kind, 0, (int)L.N};
+    const PlanKey key{B, H, L.S, (int)L.N, causal, L.kind, 0, (int)L.N, D};
     {
         std::lock_guard<std::mutex> lock(mu);
         auto it = cache.find({key, per_step});
@@ -186,7 +203,7 @@ int flat_items(int64_t B, int64_t H, const Layout& L, int causal, bool per_step,
     const int n_lists = per_step ? (int)L.N : 1;
     for (int s = 0; s < n_lists; ++s) {
         f.offsets.push_back((int)flat.size());
-        const auto& items = per_step ? plan_items(B, H, L, causal, s, s + 1) : plan_items(B, H, L, causal, 0, (int)L.N);
+        const auto& items = per_step ? plan_items(B, H, L, D, causal, s, s + 1) : plan_items(B, H, L, D, causal, 0, (int)L.N);
         for (const PlanItem& x : items) flat.push_back(make_int4(x.b, x.h, x.i, x.p));
     }
     f.offsets.push_back((int)flat.size());
@@ -224,9 +241,9 @@ Workspace carve(int64_t B, int64_t H, const Layout& L, int64_t D, int causal, in
     w.per_step = per_step && L.N > 1;
     if (kernel == kTC) {
         if (w.per_step) {
-            for (int s = 0; s < (int)L.N; ++s) w.n_items_total += plan_items(B, H, L, causal, s, s + 1).size();
+            for (int s = 0; s < (int)L.N; ++s) w.n_items_total += plan_items(B, H, L, D, causal, s, s + 1).size();
         } else {
-            w.n_items_total = plan_items(B, H, L, causal, 0, (int)L.N).size();
+            w.n_items_total = plan_items(B, H, L, D, causal, 0, (int)L.N).size();
         }
         w.counters = off;
         w.n_counters = w.per_step ? (size_t)L.N : 1;
@@ -385,7 +402,7 @@ int run_forward(const Call& c, const ra_options& opt) {
         if ((rc = encode_qkv_map(&tc.tm_v, v, c.B, L, c.H, c.D)) != RA_OK) return finish(rc);
         // upload the work list(s) from the cached pinned copy
         const FlatList* fl = nullptr;
-        if ((rc = flat_items(c.B, c.H, L, args.causal, w.per_step, &fl)) != RA_OK) return finish(rc);
+        if ((rc = flat_items(c.B, c.H, L, c.D, args.causal, w.per_step, &fl)) != RA_OK) return finish(rc);
         step_item_offset = fl->offsets;
         if (fl->count > 0 &&
             (e = cudaMemcpyAsync(ws + w.items, fl->data, fl->count * sizeof(int4),
@@ -572,13 +589,13 @@ int ra_plan_tiles(int64_t S, int n_ring, int layout, int causal, int tile, int8_
     return RA_OK;
 }
 
-int ra_plan_items(int64_t B, int64_t H, int64_t S, int n_ring, int causal, int layout,
+int ra_plan_items(int64_t B, int64_t H, int64_t S, int64_t D, int n_ring, int causal, int layout,
                   int32_t* items, int64_t cap, int64_t* n_items) {
     if (!n_items || (cap > 0 && !items)) return RA_ERR_INVALID_ARG;
-    int rc = check_shape(B, H, S, 1, n_ring, layout, RA_DTYPE_FP32);
+    int rc = check_shape(B, H, S, D, n_ring, layout, RA_DTYPE_FP32);
     if (rc != RA_OK) return rc;
     const Layout L = make_layout(S, n_ring, layout);
-    const auto& list = plan_items(B, H, L, causal ? 1 : 0, 0, n_ring);
+    const auto& list = plan_items(B, H, L, D, causal ? 1 : 0, 0, n_ring);
     *n_items = (int64_t)list.size();
     for (int64_t t = 0; t < std::min<int64_t>(cap, (int64_t)list.size()); ++t) {
         const PlanItem& x = list[(size_t)t];

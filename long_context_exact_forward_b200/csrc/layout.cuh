@@ -58,6 +58,11 @@ RA_HD int64_t visible_keys(const Layout& L, int causal, int64_t i, int64_t a, in
 // (ultralytics.com "Ring Attention" toy loop; jisaku.com 処理フロー t = 0 .. N-1).
 RA_HD int64_t ring_block(int64_t i, int64_t s, int64_t N) { return ((i - s) % N + N) % N; }
 
+// Work order of the persistent kernel: when one head's keys and values (4*S*D bytes in bf16) no
+// longer fit comfortably in the 126 MB L2, the items of each shard are grouped together so that CTAs
+// running at the same time walk the same ring sequence of key/value blocks.
+RA_HD bool plan_groups_by_shard(int64_t S, int64_t D) { return S * D * 4 > (int64_t(96) << 20); }
+
 // 32-bit forms of the same maps for device code (the host rejects S >= 2^31, so every position,
 // count and index of a shard fits in 32 bits; 32-bit division is far cheaper on the GPU).
 struct Layout32 {

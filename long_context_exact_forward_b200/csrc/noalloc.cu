@@ -35,7 +35,7 @@ using ra::Layout;
 constexpr size_t kScratchBytes = (size_t)RA_NOALLOC_SCRATCH_BYTES;
 constexpr int kTileRows = 128;
 constexpr int kPairRows = 256;
-constexpr int kMaxItemsPerHead = 12288;  // shared-memory cost table of the list builder (48 KB)
+constexpr int kMaxItemsPerHead = 11264;  // shared-memory tables of the list builder (< 48 KB)
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kScratchBytes];
 
@@ -65,12 +65,15 @@ __device__ int live_tiles(const Layout& L, int causal, int64_t i, int64_t a0, in
     return (int)((ra::visible_keys(L, causal, i, last, j) + kTileRows - 1) / kTileRows);
 }
 
-// One CTA builds the persistent kernel's work list on the device: per head the N * pairs items
-// (shard i, query-tile pair p) sorted by decreasing cost (stable, so ties keep (i, p) order),
-// repeated for every (b, h) in head-major order -- the same list the host planner uploads.
+// One CTA builds the persistent kernel's work list on the device -- the same list, in the same
+// order, as the host planner uploads: per head the N * pairs items (shard i, query-tile pair p),
+// heaviest first (stable, ties keep (i, p) order), or with `by_shard` grouped by shard (groups
+// heaviest first, heaviest first inside), repeated for every (b, h) in head-major order.
 __global__ void build_work_list(int4* __restrict__ items, int64_t BH, int64_t H, Layout L, int causal,
-                                int pairs) {
-    extern __shared__ int cost[];
+                                int pairs, int by_shard) {
+    extern __shared__ int smem_i[];
+    int* cost = smem_i;                      // [N * pairs]
+    int* group = smem_i + L.N * pairs;       // [N]
     const int n = (int)L.N * pairs;
     for (int x = threadIdx.x; x < n; x += blockDim.x) {
         const int64_t i = x / pairs, p = x % pairs;
@@ -82,12 +85,25 @@ __global__ void build_work_list(int4* __restrict__ items, int64_t BH, int64_t H,
         cost[x] = c;
     }
     __syncthreads();
+    for (int g = threadIdx.x; g < (int)L.N; g += blockDim.x) {
+        int t = 0;
+        for (int p = 0; p < pairs; ++p) t += cost[g * pairs + p];
+        group[g] = t;
+    }
+    __syncthreads();
     for (int x = threadIdx.x; x < n; x += blockDim.x) {
-        const int c = cost[x];
+        const int c = cost[x], gx = x / pairs, gc = group[gx];
         int rank = 0;
         for (int y = 0; y < n; ++y) {
             const int cy = cost[y];
-            rank += (cy > c) || (cy == c && y < x);
+            bool before;
+            if (by_shard) {
+                const int gy = y / pairs, gcy = group[gy];
+                before = (gcy > gc) || (gcy == gc && (gy < gx || (gy == gx && (cy > c || (cy == c && y < x)))));
+            } else {
+                before = (cy > c) || (cy == c && y < x);
+            }
+            rank += before;
         }
         const int i = x / pairs, p = x % pairs;
         for (int64_t bh = 0; bh < BH; ++bh)
@@ -126,7 +142,7 @@ extern "C" int ra_forward_noalloc(const void* q, const void* k, const void* v, v
     const size_t need = counter_bytes + items_bytes + (permute ? 3 * align256(tensor_bytes) : 0);
     if (per_head > kMaxItemsPerHead || need > kScratchBytes || n_items > INT32_MAX) {
         ra::host_set_error("ra_forward_noalloc: problem needs more scratch than the fixed "
-                           "RA_NOALLOC_SCRATCH_BYTES array (or more than 12288 work items per head)");
+                           "RA_NOALLOC_SCRATCH_BYTES array (or more than 11264 work items per head)");
         return RA_ERR_NO_WORKSPACE;
     }
     unsigned char* scratch = nullptr;
@@ -137,8 +153,9 @@ extern "C" int ra_forward_noalloc(const void* q, const void* k, const void* v, v
     int4* items = reinterpret_cast<int4*>(scratch + counter_bytes);
     cudaError_t e = cudaMemsetAsync(counter, 0, sizeof(int), stream);
     if (e != cudaSuccess) return ra::host_cuda_fail(e, "work counter reset");
-    const size_t smem = (size_t)per_head * sizeof(int);
-    build_work_list<<<1, 1024, smem, stream>>>(items, B * H, H, L, causal ? 1 : 0, pairs);
+    const size_t smem = (size_t)(per_head + L.N) * sizeof(int);
+    build_work_list<<<1, 1024, smem, stream>>>(items, B * H, H, L, causal ? 1 : 0, pairs,
+                                                ra::plan_groups_by_shard(S, D) ? 1 : 0);
     e = cudaGetLastError();
     if (e != cudaSuccess) return ra::host_cuda_fail(e, "work list launch");
 

@@ -99,3 +99,26 @@ def test_causal_work_totals_match_closed_form():
     for _, _, i, _, cost in items.tolist():
         per_shard[i] += cost
     assert per_shard[-1] / per_shard[0] > 10  # the last shard sees every earlier block
+
+
+def test_work_list_groups_shards_when_a_head_exceeds_l2():
+    # one head's K/V = 4 * S * D bytes = 128 MiB > 96 MiB: items of a shard are kept together
+    B, H, S, D, N = 1, 2, 262144, 128, 16
+    items = ra.plan_items(B, H, S, N, True, "striped", D=D)
+    pairs = (S // N + 255) // 256
+    assert items.shape == (B * H * N * pairs, 5)
+    per_head = N * pairs
+    for h in range(H):
+        blk = items[h * per_head:(h + 1) * per_head]
+        assert (blk[:, 1] == h).all()
+        shards = blk[:, 2]
+        runs = [shards[0]] + [b for a, b in zip(shards[:-1], shards[1:]) if a != b]
+        assert sorted(runs) == list(range(N))  # each shard appears as one contiguous run
+        group_cost = [int(blk[shards == i, 4].sum()) for i in runs]
+        assert group_cost == sorted(group_cost, reverse=True)
+        for i in range(N):
+            c = blk[shards == i, 4]
+            assert (np.diff(c) <= 0).all()
+    # below the threshold the plain heaviest-first order is kept
+    small = ra.plan_items(1, 1, 65536, 16, True, "striped", D=128)
+    assert (np.diff(small[:, 4]) <= 0).all()

@@ -49,6 +49,20 @@ def test_noalloc_matches_allocating_entry_point_twice_in_a_row():
             assert (lse - ref_lse).abs().max().item() <= 1e-3
 
 
+def test_noalloc_shard_grouped_order_matches():
+    """A head whose K/V exceeds L2 makes the device-built work list group items by shard."""
+    q, k, v = inputs.make_qkv(1, 262144, 1, 128, torch.bfloat16, "cuda", seed=7)
+    for rep in range(2):
+        rc, out, lse = call_noalloc(q, k, v, 16, True, "contiguous")
+        assert rc == 0, ra.status_string(rc)
+        ref, ref_lse = ra.forward(q, k, v, 16, True, "contiguous")
+        torch.cuda.synchronize()
+        assert ra.get_device_status() == 0
+        d = (out.float() - ref.float()).abs()
+        assert d.max().item() <= 2e-2 and d.mean().item() <= 2e-3
+        assert (lse - ref_lse).abs().max().item() <= 1e-3
+
+
 def test_noalloc_rejects_problems_beyond_its_scratch():
     # striped needs 3 shard-major copies: 3 x 1 x 65536 x 4 x 128 x 2 B = 192 MiB > 64 MiB
     q, k, v = inputs.make_qkv(1, 65536, 4, 128, torch.bfloat16, "cuda", seed=1)
