@@ -35,21 +35,24 @@ METRIC = "ring-attn fwd TFLOP/s (bf16, causal) and % of B200 dense BF16 tensor p
 UNIT = "TFLOP/s"
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
-# DRAM bytes (read + write) per attention launch on s128k, from an ncu capture of the 4-head case
-# scaled by heads (profiles/attn_tc_fused_s128k_striped.md); valid only for the kernel source whose
-# sha256 starts with the recorded prefix -- any other source reports traffic as null.
-TRAFFIC_RECORD = {"attn_tc_sha256_prefix": "971a67f661c562ad", "bytes_per_launch": 3.903e9 * 8}
+# DRAM bytes (read + write) per attention launch on s128k striped, from an ncu capture of the
+# 4-head case scaled by heads (profiles/attn_tc_fused_s128k_striped.md); valid only while
+# sha256(attn_tc.cu + api.cu) starts with the recorded prefix -- otherwise traffic is null.
+TRAFFIC_RECORD = {"source_sha256_prefix": "unmeasured", "bytes_per_launch": None}
 
 
 def recorded_traffic(args):
+    """DRAM bytes per launch recorded for this exact kernel and host code (which decides the
+    layout the kernel reads), or None."""
     import hashlib
-    src = os.path.join(ROOT, "long_context_exact_forward_b200", "csrc", "attn_tc.cu")
-    try:
-        digest = hashlib.sha256(open(src, "rb").read()).hexdigest()
-    except OSError:
-        return None
+    h = hashlib.sha256()
+    for rel in ("attn_tc.cu", "api.cu"):
+        try:
+            h.update(open(os.path.join(ROOT, "long_context_exact_forward_b200", "csrc", rel), "rb").read())
+        except OSError:
+            return None
     default_run = args.workload == "s128k" and args.layout == "striped" and args.heads in (0, 32)
-    if default_run and digest.startswith(TRAFFIC_RECORD["attn_tc_sha256_prefix"]):
+    if default_run and h.hexdigest().startswith(TRAFFIC_RECORD["source_sha256_prefix"]):
         return TRAFFIC_RECORD["bytes_per_launch"]
     return None
 
@@ -294,38 +297,82 @@ def run_ours(args, w):
     ms_per_step = ms / args.steps
     value = job_throughput(flops, world, ms_per_step)
 
-    # ---- end to end through the public API: pinned host inputs in, result back to the host
+    # ---- end to end through the public API: every step copies its inputs from pinned host memory
+    #      to the device and its result (out, lse) back.  Pipelined: copies run on their own
+    #      streams into double-buffered device tensors, so step s+1's inputs travel while step s
+    #      computes (what a caller streaming many sequences does).  The serial form, where every
+    #      copy waits for the previous call, is reported beside it.
     e2e = None
     if not args.no_e2e:
         qh, kh, vh = (t.cpu().pin_memory() for t in (q, k, v))
-        oh = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-        lh = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
-        qd, kd, vd = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+        oh = [torch.empty(out.shape, dtype=out.dtype).pin_memory() for _ in range(2)]
+        lh = [torch.empty(lse.shape, dtype=lse.dtype).pin_memory() for _ in range(2)]
+        dq = [[torch.empty_like(q) for _ in range(3)] for _ in range(2)]
+        do = [torch.empty_like(q) for _ in range(2)]
+        dl = [torch.empty_like(lse) for _ in range(2)]
+        h2d, d2h = torch.cuda.Stream(), torch.cuda.Stream()
+        ev_in = [torch.cuda.Event() for _ in range(2)]
+        ev_done = [torch.cuda.Event() for _ in range(2)]
+        ev_free_in = [torch.cuda.Event() for _ in range(2)]
+        ev_free_out = [torch.cuda.Event() for _ in range(2)]
 
-        def e2e_step():
-            qd.copy_(qh, non_blocking=True)
-            kd.copy_(kh, non_blocking=True)
-            vd.copy_(vh, non_blocking=True)
-            ra.forward(qd, kd, vd, N, True, args.layout, variant=args.variant, out=out, lse=lse,
-                       workspace=ws, stream=stream)
-            oh.copy_(out, non_blocking=True)
-            lh.copy_(lse, non_blocking=True)
+        def pipelined(n_steps):
+            for st in range(n_steps):
+                b = st % 2
+                with torch.cuda.stream(h2d):
+                    if st >= 2:
+                        h2d.wait_event(ev_free_in[b])
+                    for dst, src in zip(dq[b], (qh, kh, vh)):
+                        dst.copy_(src, non_blocking=True)
+                    ev_in[b].record(h2d)
+                stream.wait_event(ev_in[b])
+                if st >= 2:
+                    stream.wait_event(ev_free_out[b])
+                ra.forward(dq[b][0], dq[b][1], dq[b][2], N, True, args.layout, variant=args.variant,
+                           out=do[b], lse=dl[b], workspace=ws, stream=stream)
+                ev_free_in[b].record(stream)
+                ev_done[b].record(stream)
+                with torch.cuda.stream(d2h):
+                    d2h.wait_event(ev_done[b])
+                    oh[b].copy_(do[b], non_blocking=True)
+                    lh[b].copy_(dl[b], non_blocking=True)
+                    ev_free_out[b].record(d2h)
 
-        e2e_step()
+        pipelined(2)
         torch.cuda.synchronize()
         barrier(world)
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for _ in range(args.steps):
-            e2e_step()
-        e1.record(stream)
+        e0.record(h2d)
+        pipelined(args.steps)
+        e1.record(d2h)
         torch.cuda.synchronize()
         ems = max_over_ranks(e0.elapsed_time(e1), world) / args.steps
+
+        def serial_step():
+            for dst, src in zip(dq[0], (qh, kh, vh)):
+                dst.copy_(src, non_blocking=True)
+            ra.forward(dq[0][0], dq[0][1], dq[0][2], N, True, args.layout, variant=args.variant,
+                       out=do[0], lse=dl[0], workspace=ws, stream=stream)
+            oh[0].copy_(do[0], non_blocking=True)
+            lh[0].copy_(dl[0], non_blocking=True)
+
+        serial_step()
+        torch.cuda.synchronize()
+        barrier(world)
+        s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s0.record(stream)
+        for _ in range(args.steps):
+            serial_step()
+        s1.record(stream)
+        torch.cuda.synchronize()
+        sms = max_over_ranks(s0.elapsed_time(s1), world) / args.steps
         bi = 3 * q.numel() * q.element_size()
         bo = out.numel() * out.element_size() + lse.numel() * lse.element_size()
         e2e = {"value": job_throughput(flops, world, ems), "unit": UNIT, "h2d_bytes_per_step": bi,
-               "d2h_bytes_per_step": bo, "ms_per_step": ems}
-        del qh, kh, vh, oh, lh, qd, kd, vd
+               "d2h_bytes_per_step": bo, "ms_per_step": ems,
+               "form": "copies on their own streams, double-buffered, overlapping the previous step",
+               "serial": {"value": job_throughput(flops, world, sms), "ms_per_step": sms}}
+        del qh, kh, vh, oh, lh, dq, do, dl
 
     # ---- the HBM-bound kernels (permute of q into shard-major order; one per-step merge),
     #      timed alone on this workload's sizes, outside the timed region
@@ -356,8 +403,11 @@ def run_ours(args, w):
                "sample": f"{args.cpu_rows} query rows per head x {H} heads of {w.name} (causal), "
                          f"{f:.3e} flops in {dt:.1f} s"}
 
-    launches_per_step = (1 if args.layout != "contiguous" else 0) + (
-        1 if args.variant in ("fused", "auto") else 2 * N - 1)
+    # our kernels per step: the zigzag permute (striped and contiguous are read in place) and the
+    # attention launch(es) -- per-step: N attention launches and N - 1 merges (2 kernels each,
+    # the last one a single final merge)
+    launches_per_step = (1 if args.layout == "zigzag" else 0) + (
+        1 if args.variant in ("fused", "auto") else N + 2 * (N - 2) + 1)
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,

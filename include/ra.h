@@ -166,15 +166,15 @@ RA_API int ra_plan_items(int64_t B, int64_t H, int64_t S, int64_t D, int n_ring,
  * cannot let a library allocate GPU memory -- code recording a CUDA graph, engines that manage
  * every byte of device memory through their own allocator, loops where an allocation could stall.
  * It computes what ra_forward computes for bf16 q, k, v with D in {64, 128} on sm_100 (the fused
- * tensor-core ring), but takes its scratch (work list; shard-major copies of q, k, v for the
- * striped and zigzag layouts) from one fixed device array of RA_NOALLOC_SCRATCH_BYTES instead of
+ * tensor-core ring), but takes its scratch (work list and counter; shard-major copies of q, k, v
+ * for the zigzag layout) from one fixed device array of RA_NOALLOC_SCRATCH_BYTES instead of
  * allocating.  Arguments as for ra_forward (dtype is bf16 implicitly).
  *   - The first call on a device looks up the array's address with that device current; make it
  *     before any stream capture.
  *   - All calls on a device share the array and leave their data in it; calls whose GPU work
  *     overlaps (other streams, other host threads) race on it.
  *   - A problem whose scratch does not fit (B*H*n_ring*ceil(S_loc/256) work items of 16 bytes,
- *     plus 3*B*S*H*D*2 bytes for striped/zigzag and 256 bytes of counter, at most 11264 items per
+ *     plus 3*B*S*H*D*2 bytes for zigzag and 256 bytes of counter, at most 11264 items per
  *     head) is rejected with
  *     RA_ERR_NO_WORKSPACE and a message in ra_last_error_string; nothing is enqueued.
  *   - Other dtypes or head dims return RA_ERR_UNSUPPORTED. */

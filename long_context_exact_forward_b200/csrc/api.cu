@@ -3,8 +3,8 @@
 //
 // Launch sequence of ra_forward (everything on the caller's stream):
 //   tensor-core kernel (bf16, D in {64, 128}):
-//     1. permute q, k, v into shard-major order (striped / zigzag only; contiguous is already
-//        shard-major, S = N * S_loc)
+//     1. zigzag only: permute q, k, v into shard-major order (contiguous is already shard-major,
+//        S = N * S_loc; striped is read in place through a strided tensor map)
 //     2. fused:    one persistent launch walks all N ring steps and writes out / lse in natural
 //                  order (the unpermute is folded into its epilogue)
 //        per-step: for s = 0 .. N-1 one launch writes the step's partial (O_s, lse_s); an HBM-bound
@@ -250,7 +250,8 @@ Workspace carve(int64_t B, int64_t H, const Layout& L, int64_t D, int causal, in
         off = align_up(off + w.n_counters * sizeof(int));
         w.items = off;
         off = align_up(off + w.n_items_total * sizeof(int4));
-        w.permute = (L.kind != RA_LAYOUT_CONTIGUOUS);
+        // striped is read in place through a strided tensor map; zigzag is gathered shard-major
+        w.permute = (L.kind == RA_LAYOUT_ZIGZAG);
         if (w.permute) {
             w.qp = off;
             off = align_up(off + elems * esize);
@@ -289,17 +290,23 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
     return fn;
 }
 
-// Shard-major bf16 tensor [B, N, S_loc, H, D] viewed as 5-D (D, H, S_loc, N, B); one box is
-// 64 head-dim elements (128 bytes, the 128-byte swizzle span) x 1 head x 128 tokens.
-int encode_qkv_map(CUtensorMap* map, const void* base, int64_t B, const Layout& L, int64_t H, int64_t D) {
+// bf16 q/k/v viewed as 5-D (D, H, a, i, B) -- local token a of shard i -- so that the kernel's
+// TMA coordinates are the same for every source:
+//   shard-major [B, N, S_loc, H, D] (contiguous layout, or a permuted copy): a-stride H*D, i-stride S_loc*H*D;
+//   natural order under the striped layout (token a*N + i):                   a-stride N*H*D, i-stride H*D.
+// One box is 64 head-dim elements (128 bytes, the 128-byte swizzle span) x 1 head x 128 tokens;
+// tokens past the shard end read as zero.
+int encode_qkv_map(CUtensorMap* map, const void* base, int64_t B, const Layout& L, int64_t H, int64_t D,
+                   bool striped_natural) {
     auto fn = encode_fn();
     if (!fn) {
         snprintf(g_last_error, sizeof g_last_error, "cuTensorMapEncodeTiled entry point unavailable");
         return RA_ERR_CUDA;
     }
+    const cuuint64_t row = (cuuint64_t)(H * D * 2);
     const cuuint64_t dims[5] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)L.S_loc, (cuuint64_t)L.N, (cuuint64_t)B};
-    const cuuint64_t strides[4] = {(cuuint64_t)(D * 2), (cuuint64_t)(H * D * 2),
-                                   (cuuint64_t)(L.S_loc * H * D * 2), (cuuint64_t)(L.S * H * D * 2)};
+    const cuuint64_t strides[4] = {(cuuint64_t)(D * 2), striped_natural ? row * (cuuint64_t)L.N : row,
+                                   striped_natural ? row : row * (cuuint64_t)L.S_loc, row * (cuuint64_t)L.S};
     const cuuint32_t box[5] = {64, 1, (cuuint32_t)kTcTileM, 1, 1};
     const cuuint32_t estr[5] = {1, 1, 1, 1, 1};
     CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(base), dims, strides, box,
@@ -397,9 +404,10 @@ int run_forward(const Call& c, const ra_options& opt) {
             k = dst[1];
             v = dst[2];
         }
-        if ((rc = encode_qkv_map(&tc.tm_q, q, c.B, L, c.H, c.D)) != RA_OK) return finish(rc);
-        if ((rc = encode_qkv_map(&tc.tm_k, k, c.B, L, c.H, c.D)) != RA_OK) return finish(rc);
-        if ((rc = encode_qkv_map(&tc.tm_v, v, c.B, L, c.H, c.D)) != RA_OK) return finish(rc);
+        const bool striped_natural = (L.kind == RA_LAYOUT_STRIPED);
+        if ((rc = encode_qkv_map(&tc.tm_q, q, c.B, L, c.H, c.D, striped_natural)) != RA_OK) return finish(rc);
+        if ((rc = encode_qkv_map(&tc.tm_k, k, c.B, L, c.H, c.D, striped_natural)) != RA_OK) return finish(rc);
+        if ((rc = encode_qkv_map(&tc.tm_v, v, c.B, L, c.H, c.D, striped_natural)) != RA_OK) return finish(rc);
         // upload the work list(s) from the cached pinned copy
         const FlatList* fl = nullptr;
         if ((rc = flat_items(c.B, c.H, L, c.D, args.causal, w.per_step, &fl)) != RA_OK) return finish(rc);
@@ -483,8 +491,9 @@ int host_device_facts(int* sms, bool* sm100, int** status) {
     *status = d.status;
     return RA_OK;
 }
-int host_encode_qkv_map(CUtensorMap* map, const void* base, int64_t B, const Layout& L, int64_t H, int64_t D) {
-    return encode_qkv_map(map, base, B, L, H, D);
+int host_encode_qkv_map(CUtensorMap* map, const void* base, int64_t B, const Layout& L, int64_t H, int64_t D,
+                        bool striped_natural) {
+    return encode_qkv_map(map, base, B, L, H, D, striped_natural);
 }
 int host_cuda_fail(cudaError_t e, const char* what) { return cuda_fail(e, what); }
 void host_set_error(const char* msg) { snprintf(g_last_error, sizeof g_last_error, "%s", msg); }

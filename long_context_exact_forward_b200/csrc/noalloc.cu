@@ -1,7 +1,7 @@
 // noalloc.cu -- ra_forward_noalloc: the fused tensor-core forward pass without any allocation.
 //
 // Who needs this.  ra_forward needs scratch memory (the work list of the persistent kernel and,
-// for the striped and zigzag layouts, shard-major copies of q, k and v) and, unless the caller
+// for the zigzag layout, shard-major copies of q, k and v) and, unless the caller
 // hands it a workspace, gets it with cudaMallocAsync.  Some callers cannot let a library
 // allocate device memory at all: code recording a CUDA graph (an allocation inside stream capture
 // either fails or becomes part of the graph), engines that own every byte of the GPU through
@@ -136,7 +136,7 @@ extern "C" int ra_forward_noalloc(const void* q, const void* k, const void* v, v
     const int64_t per_head = L.N * pairs;
     const int64_t n_items = B * H * per_head;
     const size_t tensor_bytes = (size_t)(B * S * H * D) * 2;
-    const bool permute = (layout != RA_LAYOUT_CONTIGUOUS);
+    const bool permute = (layout == RA_LAYOUT_ZIGZAG);  // striped is read in place
     const size_t counter_bytes = 256;  // the persistent kernel's work counter, zeroed every call
     const size_t items_bytes = align256((size_t)n_items * sizeof(int4));
     const size_t need = counter_bytes + items_bytes + (permute ? 3 * align256(tensor_bytes) : 0);
@@ -171,9 +171,10 @@ extern "C" int ra_forward_noalloc(const void* q, const void* k, const void* v, v
         vs = dst[2];
     }
     ra::TcLaunch t{};
-    if ((rc = ra::host_encode_qkv_map(&t.tm_q, qs, B, L, H, D)) != RA_OK) return rc;
-    if ((rc = ra::host_encode_qkv_map(&t.tm_k, ks, B, L, H, D)) != RA_OK) return rc;
-    if ((rc = ra::host_encode_qkv_map(&t.tm_v, vs, B, L, H, D)) != RA_OK) return rc;
+    const bool striped_natural = (layout == RA_LAYOUT_STRIPED);
+    if ((rc = ra::host_encode_qkv_map(&t.tm_q, qs, B, L, H, D, striped_natural)) != RA_OK) return rc;
+    if ((rc = ra::host_encode_qkv_map(&t.tm_k, ks, B, L, H, D, striped_natural)) != RA_OK) return rc;
+    if ((rc = ra::host_encode_qkv_map(&t.tm_v, vs, B, L, H, D, striped_natural)) != RA_OK) return rc;
     t.items = items;
     t.n_items = (int)n_items;
     t.counter = counter;

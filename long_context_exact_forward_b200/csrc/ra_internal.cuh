@@ -59,7 +59,8 @@ size_t tc_smem_bytes(int64_t D);
 // api.cu: host helpers shared by the entry points.
 int host_check_shape(int64_t B, int64_t H, int64_t S, int64_t D, int n_ring, int layout, int dtype);
 int host_device_facts(int* sms, bool* sm100, int** status);
-int host_encode_qkv_map(CUtensorMap* map, const void* base, int64_t B, const Layout& L, int64_t H, int64_t D);
+int host_encode_qkv_map(CUtensorMap* map, const void* base, int64_t B, const Layout& L, int64_t H, int64_t D,
+                        bool striped_natural);
 int host_cuda_fail(cudaError_t e, const char* what);
 void host_set_error(const char* msg);
 cudaError_t launch_attn_tc(const AttnArgs& a, const TcLaunch& t, cudaStream_t stream);

@@ -68,9 +68,11 @@ def test_workspace_size_grows_with_per_step_and_permute():
     fused_striped = ra.workspace_size(layout="striped", variant="fused", **args)
     per_step = ra.workspace_size(layout="contiguous", variant="per_step", **args)
     elems = 1 * 4096 * 4 * 128
-    assert fused_striped >= fused_contig + 3 * elems * 2          # permuted q, k, v
+    fused_zigzag = ra.workspace_size(layout="zigzag", variant="fused", **args)
+    assert fused_striped < fused_contig + elems                    # striped is read in place
+    assert fused_zigzag >= fused_contig + 3 * elems * 2           # permuted q, k, v
     assert per_step >= fused_contig + 2 * elems * 4               # running and step partials
-    simt = ra.workspace_size(layout="striped", variant="fused", kernel="simt", **args)
+    simt = ra.workspace_size(layout="zigzag", variant="fused", kernel="simt", **args)
     assert simt <= fused_contig                                   # SIMT reads natural order
 
 

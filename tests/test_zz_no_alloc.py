@@ -64,9 +64,9 @@ def test_noalloc_shard_grouped_order_matches():
 
 
 def test_noalloc_rejects_problems_beyond_its_scratch():
-    # striped needs 3 shard-major copies: 3 x 1 x 65536 x 4 x 128 x 2 B = 192 MiB > 64 MiB
+    # zigzag needs 3 shard-major copies: 3 x 1 x 65536 x 4 x 128 x 2 B = 192 MiB > 64 MiB
     q, k, v = inputs.make_qkv(1, 65536, 4, 128, torch.bfloat16, "cuda", seed=1)
-    rc, _, _ = call_noalloc(q, k, v, 8, True, "striped")
+    rc, _, _ = call_noalloc(q, k, v, 8, True, "zigzag")
     assert rc == -5  # RA_ERR_NO_WORKSPACE
     assert b"RA_NOALLOC_SCRATCH_BYTES" in ra.lib().ra_last_error_string()
     q2, k2, v2 = inputs.make_qkv(1, 256, 1, 96, torch.bfloat16, "cuda", seed=2)
