@@ -38,7 +38,7 @@ PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # DRAM bytes (read + write) per attention launch on s128k striped, from an ncu capture of the
 # 4-head case scaled by heads (profiles/attn_tc_fused_s128k_striped.md); valid only while
 # sha256(attn_tc.cu + api.cu) starts with the recorded prefix -- otherwise traffic is null.
-TRAFFIC_RECORD = {"source_sha256_prefix": "unmeasured", "bytes_per_launch": None}
+TRAFFIC_RECORD = {"source_sha256_prefix": "beb93a897462e639", "bytes_per_launch": 3.676e9 * 8}
 
 
 def recorded_traffic(args):
