@@ -23,7 +23,7 @@
 //   warps 0-3  softmax for query tile 0 (thread t owns row t = TMEM lane t)
 //   warps 4-7  softmax for query tile 1
 //   warp  8    TMA producer: Q tiles, then K and V tiles into a ring of 4 shared-memory slots
-//   warp  9    MMA issuer (one thread) and TMEM owner
+//   warp  9    MMA issuer (the whole warp runs the loop, one elected lane issues) and TMEM owner
 //   warps 10-11 idle
 // TMEM (512 columns): S0 [0,128), S1 [128,256), O0 [256,256+D), O1 [384,384+D).  P (bf16) is
 // written over the first 64 columns of its S tile and read from there by the P V MMA.
@@ -257,17 +257,18 @@ struct Roles {
         }
     }
 
-    // ------------------------------------------------------------ MMA issuer (one thread)
+    // ------------------------------------------------------------ MMA issuer (one warp, converged;
+    // the elected lane issues every MMA and commit)
     __device__ void issue_s(int q, uint32_t kslot) {
         constexpr uint32_t idesc = idesc_bf16_f32(kM, kN, 0, 0);
         const uint32_t qa = smem_addr(sm.q[q]), ka = smem_addr(sm.kv[kslot]);
 #pragma unroll
         for (int kk = 0; kk < kD / 16; ++kk) {
             const uint32_t off = (kk >> 2) * kColBlockBytes + (kk & 3) * 32;
-            mma_ss(tmem + s_col(q), smem_desc_sw128(qa + off, 16, 1024),
+            warp_mma_ss(tmem + s_col(q), smem_desc_sw128(qa + off, 16, 1024),
                    smem_desc_sw128(ka + off, 16, 1024), idesc, kk > 0);
         }
-        mma_commit(&sm.s_full[q]);
+        warp_mma_commit(&sm.s_full[q]);
     }
 
     __device__ void issue_pv(int q, uint32_t vslot, bool accumulate) {
@@ -276,7 +277,7 @@ struct Roles {
 #pragma unroll
         for (int kk = 0; kk < kN / 16; ++kk) {
             // 16 keys = 16 rows of 128 B of every column block; P: 16 bf16 = 8 TMEM columns
-            mma_ts(tmem + o_col<kD>(q), tmem + s_col(q) + kk * 8,
+            warp_mma_ts(tmem + o_col<kD>(q), tmem + s_col(q) + kk * 8,
                    smem_desc_sw128(va + kk * 16 * 128, kColBlockBytes, 1024), idesc,
                    (kk > 0 || accumulate) ? 1u : 0u);
         }
@@ -285,9 +286,10 @@ struct Roles {
     __device__ void mma() {
         uint32_t tile_it = 0, q_it = 0, p_cnt[2] = {0, 0}, act_items[2] = {0, 0};
         bool ok = true;
+        const bool leader = (threadIdx.x & 31) == 0;
         auto wait = [&](uint64_t* bar, uint32_t parity) {
             if (!ok) return false;
-            ok = mbar_wait(bar, parity, timeout, abort);
+            ok = __all_sync(0xffffffffu, mbar_wait(bar, parity, timeout, abort));
             if (ok) tc_fence_after();
             return ok;
         };
@@ -296,7 +298,8 @@ struct Roles {
             const uint32_t b = k & 1;
             if (!wait(&sm.item_full[b], (k >> 1) & 1)) break;
             const int idx = sm.item_idx[b];
-            mbar_arrive(&sm.item_empty[b]);
+            __syncwarp();
+            if (leader) mbar_arrive(&sm.item_empty[b]);
             if (idx < 0) break;
             const ItemGeom G = item_geom(L, items[idx]);
             TileIter cur;
@@ -313,10 +316,10 @@ struct Roles {
                     issue_s(q, kslot);
                     any_act[q] = true;
                 }
-            mma_commit(&sm.slot_empty[kslot]);
+            warp_mma_commit(&sm.slot_empty[kslot]);
             TileIter nxt = cur;
             nxt.next(L, A.causal, G);
-            if (!nxt.valid) mma_commit(&sm.q_empty);
+            if (!nxt.valid) warp_mma_commit(&sm.q_empty);
             for (;;) {
                 const uint32_t vslot = (2 * tile_it + 1) % kSlots;  // landed with K of this tile
                 for (int q = 0; q < 2; ++q) {
@@ -339,29 +342,29 @@ struct Roles {
                     }
                 }
                 if (!ok) break;
-                mma_commit(&sm.slot_empty[vslot]);
+                warp_mma_commit(&sm.slot_empty[vslot]);
                 if (!nxt.valid) break;
                 if (nxt.act(1)) {
                     issue_s(1, kslot);
                     any_act[1] = true;
                 }
-                mma_commit(&sm.slot_empty[kslot]);
+                warp_mma_commit(&sm.slot_empty[kslot]);
                 cur = nxt;
                 ++tile_it;
                 nxt.next(L, A.causal, G);
-                if (!nxt.valid) mma_commit(&sm.q_empty);
+                if (!nxt.valid) warp_mma_commit(&sm.q_empty);
             }
             if (!ok) break;
             ++tile_it;  // past the item's last key tile
             for (int q = 0; q < 2; ++q)
                 if (any_act[q]) {
-                    mma_commit(&sm.o_final[q]);
+                    warp_mma_commit(&sm.o_final[q]);
                     ++act_items[q];
                 }
         }
         if (!ok) {
-            give_up(abort, status);
-            mma_commit(&sm.drain);  // every MMA issued so far has finished once this arrives
+            if (leader) give_up(abort, status);
+            warp_mma_commit(&sm.drain);  // every MMA issued so far has finished once this arrives
             mbar_wait(&sm.drain, 0, timeout, nullptr);
         }
     }
@@ -583,7 +586,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int k = 0; k < kSlots; ++k) mbar_init(&sm.slot_empty[k], 1);
         for (int b = 0; b < 2; ++b) {
             mbar_init(&sm.item_full[b], 1);
-            mbar_init(&sm.item_empty[b], 9);  // the MMA thread + one lane of each softmax warp
+            mbar_init(&sm.item_empty[b], 9);  // one lane of the MMA warp and of each softmax warp
         }
         for (int q = 0; q < 2; ++q) {
             mbar_init(&sm.s_full[q], 1);
@@ -615,7 +618,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (lane == 0) roles.producer(&tm_q, &tm_k, &tm_v, debug);
             __syncwarp();
         } else if (warp == kMmaWarp) {
-            if (lane == 0) roles.mma();
+            roles.mma();
             __syncwarp();
         }
     } else {
