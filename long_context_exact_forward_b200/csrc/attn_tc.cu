@@ -22,14 +22,17 @@
 // counter, heaviest first):
 //   warps 0-3  softmax for query tile 0 (thread t owns row t = TMEM lane t)
 //   warps 4-7  softmax for query tile 1
-//   warp  8    TMA producer: Q tiles, then K and V tiles into a ring of 4 shared-memory slots
+//   warp  8    TMA producer (lane 0 issues): Q tiles, then K and V tiles into a ring of 4
+//              shared-memory slots; also hands out the work items
 //   warp  9    MMA issuer (the whole warp runs the loop, one elected lane issues) and TMEM owner
 //   warps 10-11 idle
 // TMEM (512 columns): S0 [0,128), S1 [128,256), O0 [256,256+D), O1 [384,384+D).  P (bf16) is
 // written over the first 64 columns of its S tile and read from there by the P V MMA.
 // The MMA order per key tile t is  P0V(t), S0(t+1), P1V(t), S1(t+1), so each query tile's softmax
-// overlaps the other tile's MMAs.  Because S0(t+1) is issued after P0V(t), the completion of
-// S0(t+1) also proves P0V(t) is done, which lets the softmax warps rescale O in place.
+// overlaps the other tile's MMAs.  Each P V is issued in two halves: keys 0..63 as soon as the
+// softmax warps have stored that half of P (they signal it mid-way), keys 64..127 when all of P
+// is stored.  Because S0(t+1) is issued after P0V(t), the completion of S0(t+1) also proves P0V(t)
+// is done, which lets the softmax warps rescale O in place before they store P of tile t+1.
 // Rescaling of O is lazy: it happens only when a row's max grows by more than 2^8.
 //
 // Every wait is bounded (timeout_ns); on give-up the CTA records RA_ERR_DEVICE_TIMEOUT in the
@@ -101,7 +104,7 @@ struct TcSmem {
     uint64_t q_full, q_empty, drain;
     uint64_t kv_full[2];              // K and V of key tile n have landed (barrier n % 2)
     uint64_t slot_empty[kSlots];      // key tile n uses slots 2n and 2n+1 (mod kSlots)
-    uint64_t s_full[2], p_full[2], o_final[2], o_free[2];
+    uint64_t s_full[2], p_half[2], p_full[2], o_final[2], o_free[2];  // p_half: P of keys 0..63 stored
     uint64_t item_full[2], item_empty[2];  // ring of work-item indices handed out by the load warp
     int item_idx[2];
     uint32_t tmem_base;
@@ -200,55 +203,64 @@ struct Roles {
     Layout32 L;
     int* counter;  // next work item of this launch (zeroed by the host before the launch)
 
-    // ------------------------------------------------------------ TMA producer (one thread)
+    // ------------------------------------------------------------ TMA producer (one warp, converged;
+    // lane 0 takes work items and issues the copies)
     __device__ void producer(const CUtensorMap* tm_q, const CUtensorMap* tm_k,
                              const CUtensorMap* tm_v, int debug) {
+        const bool leader = (threadIdx.x & 31) == 0;
         uint32_t tile_it = 0, q_it = 0, armed = 0;
         bool ok = true;
+        auto wait = [&](uint64_t* bar, uint32_t parity) {
+            ok = __all_sync(0xffffffffu, mbar_wait(bar, parity, timeout, abort));
+            return ok;
+        };
         // Dynamic schedule: take the next item from the launch-wide counter and publish its index
         // to the other roles through a two-entry ring (index -1 ends the loop).
         for (uint32_t k = 0; ok; ++k) {
             const uint32_t b = k & 1;
-            if (!mbar_wait(&sm.item_empty[b], ((k >> 1) & 1) ^ 1, timeout, abort)) { ok = false; break; }
-            int idx = atomicAdd(counter, 1);
-            if (idx >= n_items) idx = -1;
-            sm.item_idx[b] = idx;
-            mbar_arrive(&sm.item_full[b]);
+            if (!wait(&sm.item_empty[b], ((k >> 1) & 1) ^ 1)) break;
+            int idx = 0;
+            if (leader) {
+                idx = atomicAdd(counter, 1);
+                if (idx >= n_items) idx = -1;
+                sm.item_idx[b] = idx;
+                mbar_arrive(&sm.item_full[b]);
+            }
+            idx = __shfl_sync(0xffffffffu, idx, 0);
             if (idx < 0) break;
             const ItemGeom G = item_geom(L, items[idx]);
             TileIter t;
             t.init(A, L, G);
             if (!t.valid) continue;
             if (debug == RA_DEBUG_STALL_LOADS) continue;  // consumers must time out
-            if (!mbar_wait(&sm.q_empty, (q_it & 1) ^ 1, timeout, abort)) { ok = false; break; }
-            mbar_arrive_expect_tx(&sm.q_full, 2 * TcSmem<kD>::kTileBytes);
-            for (int q = 0; q < 2; ++q)
-                for (int cb = 0; cb < kD / 64; ++cb)
-                    tma_load_5d(sm.q[q] + cb * kColBlockBytes, tm_q, &sm.q_full, cb * 64, G.h,
-                                G.a0[q], G.i, G.b);
+            if (!wait(&sm.q_empty, (q_it & 1) ^ 1)) break;
+            if (leader) {
+                mbar_arrive_expect_tx(&sm.q_full, 2 * TcSmem<kD>::kTileBytes);
+                for (int q = 0; q < 2; ++q)
+                    for (int cb = 0; cb < kD / 64; ++cb)
+                        tma_load_5d(sm.q[q] + cb * kColBlockBytes, tm_q, &sm.q_full, cb * 64, G.h,
+                                    G.a0[q], G.i, G.b);
+            }
             ++q_it;
             for (; t.valid && ok; t.next(L, A.causal, G)) {
                 uint64_t* full = &sm.kv_full[tile_it & 1];
                 for (int w = 0; w < 2; ++w) {  // K then V of this tile, each as soon as its slot frees
                     const uint32_t use = 2 * tile_it + w;
                     const uint32_t slot = use % kSlots;
-                    if (!mbar_wait(&sm.slot_empty[slot], ((use / kSlots) & 1) ^ 1, timeout, abort)) {
-                        ok = false;
-                        break;
+                    if (!wait(&sm.slot_empty[slot], ((use / kSlots) & 1) ^ 1)) break;
+                    if (w == 0) armed = tile_it + 1;
+                    if (leader) {
+                        if (w == 0) mbar_arrive_expect_tx(full, 2 * TcSmem<kD>::kTileBytes);
+                        for (int cb = 0; cb < kD / 64; ++cb)
+                            tma_load_5d(sm.kv[slot] + cb * kColBlockBytes, w ? tm_v : tm_k, full, cb * 64,
+                                        G.h, t.kt * kN, t.j, G.b);
                     }
-                    if (w == 0) {
-                        mbar_arrive_expect_tx(full, 2 * TcSmem<kD>::kTileBytes);
-                        armed = tile_it + 1;
-                    }
-                    for (int cb = 0; cb < kD / 64; ++cb)
-                        tma_load_5d(sm.kv[slot] + cb * kColBlockBytes, w ? tm_v : tm_k, full, cb * 64,
-                                    G.h, t.kt * kN, t.j, G.b);
                 }
                 if (ok) ++tile_it;
             }
         }
         if (!ok) {
-            give_up(abort, status);
+            if (leader) give_up(abort, status);
             // let the copies already issued land before the CTA can exit (if the last tile's V
             // copy was never issued, its wait runs out after the K copy has landed)
             if (tile_it > 0) mbar_wait(&sm.kv_full[(tile_it - 1) & 1], ((tile_it - 1) >> 1) & 1, timeout, nullptr);
@@ -271,11 +283,13 @@ struct Roles {
         warp_mma_commit(&sm.s_full[q]);
     }
 
+    // O_q (+)= P_q V for the keys [16 * kk0, 16 * kk1) of the tile
+    template <int kk0, int kk1>
     __device__ void issue_pv(int q, uint32_t vslot, bool accumulate) {
         constexpr uint32_t idesc = idesc_bf16_f32(kM, kD, 0, 1);  // V is MN-major (D fastest)
         const uint32_t va = smem_addr(sm.kv[vslot]);
 #pragma unroll
-        for (int kk = 0; kk < kN / 16; ++kk) {
+        for (int kk = kk0; kk < kk1; ++kk) {
             // 16 keys = 16 rows of 128 B of every column block; P: 16 bf16 = 8 TMEM columns
             warp_mma_ts(tmem + o_col<kD>(q), tmem + s_col(q) + kk * 8,
                    smem_desc_sw128(va + kk * 16 * 128, kColBlockBytes, 1024), idesc,
@@ -324,12 +338,16 @@ struct Roles {
                 const uint32_t vslot = (2 * tile_it + 1) % kSlots;  // landed with K of this tile
                 for (int q = 0; q < 2; ++q) {
                     if (cur.act(q)) {
-                        if (!wait(&sm.p_full[q], p_cnt[q] & 1)) break;
-                        ++p_cnt[q];
+                        // P V in two halves: keys 0..63 as soon as their P is stored, while the
+                        // softmax warps still work on keys 64..127
+                        if (!wait(&sm.p_half[q], p_cnt[q] & 1)) break;
                         if (first_pv[q] && act_items[q] > 0 &&
                             !wait(&sm.o_free[q], (act_items[q] - 1) & 1))
                             break;
-                        issue_pv(q, vslot, !first_pv[q]);
+                        issue_pv<0, kN / 32>(q, vslot, !first_pv[q]);
+                        if (!wait(&sm.p_full[q], p_cnt[q] & 1)) break;
+                        ++p_cnt[q];
+                        issue_pv<kN / 32, kN / 16>(q, vslot, true);
                         first_pv[q] = false;
                     }
                     if (q == 0 && nxt.valid) {
@@ -438,6 +456,25 @@ struct Roles {
                         l *= alpha;
                         m_run = m_new;
                     }
+                    // rescale O before any P V of this tile accumulates into it (P_q V of the
+                    // previous tile is complete: S_q of this tile was issued after it)
+                    if (__any_sync(0xffffffffu, rescale)) {
+                        const uint64_t alpha2 = f32x2(alpha, alpha);
+#pragma unroll 1
+                        for (int c = 0; c < kD / 32; ++c) {
+                            uint32_t o[32];
+                            tmem_ld32(tO + c * 32, o);
+                            tmem_wait_ld_regs(o);
+#pragma unroll
+                            for (int x = 0; x < 16; ++x) {
+                                float v0, v1;
+                                split_f32x2(mul_f32x2(f32x2(__uint_as_float(o[2 * x]), __uint_as_float(o[2 * x + 1])), alpha2), v0, v1);
+                                o[2 * x] = __float_as_uint(v0);
+                                o[2 * x + 1] = __float_as_uint(v1);
+                            }
+                            tmem_st32(tO + c * 32, o);
+                        }
+                    }
                     const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
                     // P = 2^(S * scale * log2 e - m), two columns per packed op; every
                     // kExp2PolyEvery-th pair on the FMA pipe, the rest on MUFU
@@ -464,6 +501,12 @@ struct Roles {
                             pk[x] = pack_bf16x2(p0, p1);
                         }
                         tmem_st16(tS + c4 * 16, pk);
+                        if (c4 == 1) {  // P of keys 0..63 (and any rescaled O) visible to the MMA
+                            tmem_wait_st();
+                            tc_fence_before();
+                            __syncwarp();
+                            if ((threadIdx.x & 31) == 0) mbar_arrive(&sm.p_half[q]);
+                        }
                     }
                     {
                         float a0, a1, b0, b1;
@@ -473,23 +516,6 @@ struct Roles {
                         l += a0 + a1;
                     }
 #undef SF
-                    if (__any_sync(0xffffffffu, rescale)) {
-                        const uint64_t alpha2 = f32x2(alpha, alpha);
-#pragma unroll 1
-                        for (int c = 0; c < kD / 32; ++c) {
-                            uint32_t o[32];
-                            tmem_ld32(tO + c * 32, o);
-                            tmem_wait_ld_regs(o);
-#pragma unroll
-                            for (int x = 0; x < 16; ++x) {
-                                float v0, v1;
-                                split_f32x2(mul_f32x2(f32x2(__uint_as_float(o[2 * x]), __uint_as_float(o[2 * x + 1])), alpha2), v0, v1);
-                                o[2 * x] = __float_as_uint(v0);
-                                o[2 * x + 1] = __float_as_uint(v1);
-                            }
-                            tmem_st32(tO + c * 32, o);
-                        }
-                    }
                     tmem_wait_st();
                     tc_fence_before();
                     __syncwarp();
@@ -590,7 +616,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         for (int q = 0; q < 2; ++q) {
             mbar_init(&sm.s_full[q], 1);
-            mbar_init(&sm.p_full[q], 4);  // one arrival per softmax warp
+            mbar_init(&sm.p_half[q], 4);  // one arrival per softmax warp
+            mbar_init(&sm.p_full[q], 4);
             mbar_init(&sm.o_final[q], 1);
             mbar_init(&sm.o_free[q], 4);
         }
@@ -615,7 +642,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp >= 8) {
         setmaxnreg_dec112();
         if (warp == kLoadWarp) {
-            if (lane == 0) roles.producer(&tm_q, &tm_k, &tm_v, debug);
+            roles.producer(&tm_q, &tm_k, &tm_v, debug);
             __syncwarp();
         } else if (warp == kMmaWarp) {
             roles.mma();
