@@ -38,7 +38,10 @@ PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # DRAM bytes (read + write) per attention launch on s128k striped, from an ncu capture of the
 # 4-head case scaled by heads (profiles/attn_tc_fused_s128k_striped.md); valid only while
 # sha256(attn_tc.cu + api.cu) starts with the recorded prefix -- otherwise traffic is null.
-TRAFFIC_RECORD = {"source_sha256_prefix": "beb93a897462e639", "bytes_per_launch": 3.676e9 * 8}
+TRAFFIC_RECORD = {"source_sha256_prefix": "7caf598abf792ad0", "bytes_per_launch": 3.645195e9 * 8}
+# the files whose concatenation the record's hash covers: the kernel, the helpers it inlines and
+# the host code that decides the layout it reads
+TRAFFIC_SOURCES = ("attn_tc.cu", "sm100.cuh", "layout.cuh", "api.cu")
 
 
 def recorded_traffic(args):
@@ -46,7 +49,7 @@ def recorded_traffic(args):
     layout the kernel reads), or None."""
     import hashlib
     h = hashlib.sha256()
-    for rel in ("attn_tc.cu", "api.cu"):
+    for rel in TRAFFIC_SOURCES:
         try:
             h.update(open(os.path.join(ROOT, "long_context_exact_forward_b200", "csrc", rel), "rb").read())
         except OSError:
