@@ -9,9 +9,15 @@
 // the online-softmax identities (troisinh.com "Ring Attention", "Tai sao no hoat dong") whenever
 // m grows; the accumulator is divided by l at the end.
 //
-// Tiling: a CTA of 128 threads owns 32 query rows of one shard for one (b, h); 4 threads share a
-// row (each scores 8 of the 32 keys of a tile and owns every 4th output column).  Keys and values
-// are gathered straight from natural order with the layout map, so no permute is needed.
+// Tiling (register-blocked, like a single-precision GEMM): a CTA of 256 threads owns 64 query rows
+// of one shard for one (b, h) and walks 64-key tiles.  Thread (ty, tx) = (tid / 16, tid % 16)
+// computes the 4 x 4 block of scores of rows 4ty..4ty+3 and keys 4tx..4tx+3, one float4 of Q^T and
+// one of K^T per step over the head dim (16 FMAs per two shared-memory loads), and the
+// 4 x (kDMax / 16) block of the output of the same rows and the columns 4tx + 64c + (0..3) from P^T
+// and V, one float4 of P^T and kDMax / 64 float4s of V per key (8 consecutive threads read 128
+// consecutive bytes of V, so the float4 loads are free of bank conflicts).  Two CTAs share an SM.  Row maxima and sums are reduced over
+// the 16 threads of a row group with shuffles.  Keys and values are gathered straight from natural
+// order with the layout map, so no permute is needed.
 #include <cuda_bf16.h>
 
 #include "ra_internal.cuh"
@@ -19,9 +25,9 @@
 namespace ra {
 namespace {
 
-constexpr int kBQ = 32;       // query rows per CTA
-constexpr int kBK = 32;       // keys per tile
-constexpr int kThreads = 128; // 4 threads per query row
+constexpr int kBQ = 64;        // query rows per CTA
+constexpr int kBK = 64;        // keys per tile
+constexpr int kThreads = 256;  // 16 x 16 thread grid
 
 template <typename T>
 __device__ __forceinline__ float to_float(T x);
@@ -37,140 +43,200 @@ __device__ __forceinline__ float from_float<float>(float x) { return x; }
 template <>
 __device__ __forceinline__ __nv_bfloat16 from_float<__nv_bfloat16>(float x) { return __float2bfloat16_rn(x); }
 
-// Load `rows` token rows of shard `shard` starting at local row a0 into smem [kB][ld] as fp32;
-// rows past the shard end read as zero.
-template <typename T>
-__device__ void load_rows(float* dst, int ld, const T* __restrict__ src, const Layout& L,
-                          int64_t b, int64_t h, int64_t H, int64_t D, int64_t shard, int64_t a0,
-                          int rows) {
-    for (int idx = threadIdx.x; idx < rows * D; idx += kThreads) {
-        const int r = idx / (int)D, d = idx % (int)D;
-        const int64_t a = a0 + r;
-        float x = 0.f;
-        if (a < L.S_loc) {
-            const int64_t g = global_position(L, shard, a);
-            x = to_float<T>(src[((b * L.S + g) * H + h) * D + d]);
+// Gather `kB` token rows of shard `shard` from local row a0 (natural order through the layout map)
+// as fp32 into shared memory, transposed: dst[d * kB + r].  Rows past the shard end and columns
+// d >= D read as zero.  Thread t takes row t % kB and 4 consecutive columns at a time, so
+// consecutive threads write consecutive words and each thread reads whole sectors of its row.
+template <typename T, int kDMax, int kB>
+__device__ void load_transposed(float* dst, const T* __restrict__ src, const Layout& L, int64_t b,
+                                int64_t h, int64_t H, int64_t D, int64_t shard, int64_t a0) {
+    const int r = threadIdx.x % kB;
+    const int64_t a = a0 + r;
+    const T* row = nullptr;
+    if (a < L.S_loc) row = src + ((b * L.S + global_position(L, shard, a)) * H + h) * D;
+    for (int d4 = 4 * (threadIdx.x / kB); d4 < kDMax; d4 += 4 * (kThreads / kB)) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const int d = d4 + e;
+            dst[d * kB + r] = (row && d < D) ? to_float<T>(row[d]) : 0.f;
         }
-        dst[r * ld + d] = x;
     }
 }
 
+// Same rows, row-major: dst[r * kDMax + d].  Consecutive threads take consecutive columns.
+template <typename T, int kDMax, int kB>
+__device__ void load_rowmajor(float* dst, const T* __restrict__ src, const Layout& L, int64_t b,
+                              int64_t h, int64_t H, int64_t D, int64_t shard, int64_t a0) {
+    for (int idx = threadIdx.x; idx < kB * kDMax; idx += kThreads) {
+        const int r = idx / kDMax, d = idx % kDMax;
+        const int64_t a = a0 + r;
+        float x = 0.f;
+        if (a < L.S_loc && d < D)
+            x = to_float<T>(src[((b * L.S + global_position(L, shard, a)) * H + h) * D + d]);
+        dst[idx] = x;
+    }
+}
+
+// P^T is stored key-major with its 4-row groups permuted by an XOR with (key / 4) mod 16, so that
+// both the 16 threads of a row group writing one key each and the float4 reads of the P V loop
+// hit distinct banks.
+__device__ __forceinline__ int pt_index(int key, int row4) {
+    return key * kBQ + (((row4 >> 2) ^ ((key >> 2) & 15)) << 2);
+}
+
 template <typename T, int kDMax>
-__global__ void __launch_bounds__(kThreads) attn_simt_kernel(const T* __restrict__ q,
-                                                             const T* __restrict__ k,
-                                                             const T* __restrict__ v, AttnArgs args) {
-    constexpr int kCols = kDMax / 4;  // output columns owned per thread
-    extern __shared__ float smem[];
+__global__ void __launch_bounds__(kThreads, kDMax <= 128 ? 2 : 1)
+    attn_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
+                     AttnArgs args) {
+    constexpr int kOC = kDMax / 16;  // output columns per thread
+    static_assert(kOC % 4 == 0, "kDMax is a multiple of 64");
+    extern __shared__ __align__(16) float smem[];
+    float* Qt = smem;                 // [kDMax][kBQ]
+    float* Kt = Qt + kDMax * kBQ;     // [kDMax][kBK]
+    float* Vs = Kt + kDMax * kBK;     // [kBK][kDMax]
+    float* Pt = Vs + kBK * kDMax;     // [kBK][kBQ], swizzled (pt_index)
+
     const Layout L = args.L;
     const int64_t D = args.D, H = args.H;
-    const int ldq = (int)D + 1, ldk = (int)D + 1, ldv = (int)D, ldp = kBK + 1;
-    float* Qs = smem;
-    float* Ks = Qs + kBQ * ldq;
-    float* Vs = Ks + kBK * ldk;
-    float* Ps = Vs + kBK * ldv;
-
-    const int64_t i = blockIdx.y;
+    // heaviest shards first: under the causal mask with the contiguous layout shard i meets i + 1
+    // live blocks, so the CTAs of the last shards are launched first (a longest-first order)
+    const int64_t i = L.N - 1 - blockIdx.y;
     const int64_t bh = blockIdx.z;
     const int64_t b = bh / H, h = bh % H;
     const int64_t a0 = (int64_t)blockIdx.x * kBQ;
-    const int r = threadIdx.x >> 2, sub = threadIdx.x & 3;
-    const int64_t a = a0 + r;
-
-    load_rows<T>(Qs, ldq, q, L, b, h, H, D, i, a0, kBQ);
-
-    float m = -INFINITY, l = 0.f;
-    float o[kCols];
-#pragma unroll
-    for (int c = 0; c < kCols; ++c) o[c] = 0.f;
-
+    const int ty = threadIdx.x >> 4, tx = threadIdx.x & 15;
     const int64_t a_last = (a0 + kBQ - 1 < L.S_loc - 1) ? a0 + kBQ - 1 : L.S_loc - 1;
+
+    load_transposed<T, kDMax, kBQ>(Qt, q, L, b, h, H, D, i, a0);
+
+    float m[4], l[4], o[4][kOC];
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+        m[r] = -INFINITY;
+        l[r] = 0.f;
+#pragma unroll
+        for (int c = 0; c < kOC; ++c) o[r][c] = 0.f;
+    }
+
     for (int s = args.s_begin; s < args.s_end; ++s) {
         const int64_t j = ring_block(i, s, L.N);
-        const int64_t n_vis = visible_keys(L, args.causal, i, a, j);           // this row
+        int64_t n_vis[4];  // visible keys of block j for each of this thread's rows
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+            const int64_t a = a0 + 4 * ty + r;
+            n_vis[r] = a < L.S_loc ? visible_keys(L, args.causal, i, a, j) : 0;
+        }
         const int64_t n_vis_cta = visible_keys(L, args.causal, i, a_last, j);  // the CTA's widest
         for (int64_t b0 = 0; b0 < n_vis_cta; b0 += kBK) {
-            __syncthreads();  // previous tile fully consumed (and Q loaded on the first pass)
-            load_rows<T>(Ks, ldk, k, L, b, h, H, D, j, b0, kBK);
-            load_rows<T>(Vs, ldv, v, L, b, h, H, D, j, b0, kBK);
+            __syncthreads();  // previous tile consumed (and Q loaded on the first pass)
+            load_transposed<T, kDMax, kBK>(Kt, k, L, b, h, H, D, j, b0);
+            load_rowmajor<T, kDMax, kBK>(Vs, v, L, b, h, H, D, j, b0);
             __syncthreads();
 
-            // scores for keys b0 + sub*8 + x
-            float sc[8];
+            // S block: rows 4ty + r, keys 4tx + c
+            float sc[4][4];
 #pragma unroll
-            for (int x = 0; x < 8; ++x) sc[x] = 0.f;
+            for (int r = 0; r < 4; ++r)
+#pragma unroll
+                for (int c = 0; c < 4; ++c) sc[r][c] = 0.f;
+#pragma unroll 4
             for (int d = 0; d < D; ++d) {
-                const float qd = Qs[r * ldq + d];
+                const float4 qa = *reinterpret_cast<const float4*>(Qt + d * kBQ + 4 * ty);
+                const float4 kb = *reinterpret_cast<const float4*>(Kt + d * kBK + 4 * tx);
+                const float qv[4] = {qa.x, qa.y, qa.z, qa.w}, kv[4] = {kb.x, kb.y, kb.z, kb.w};
 #pragma unroll
-                for (int x = 0; x < 8; ++x) sc[x] = fmaf(qd, Ks[(sub * 8 + x) * ldk + d], sc[x]);
+                for (int r = 0; r < 4; ++r)
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) sc[r][c] = fmaf(qv[r], kv[c], sc[r][c]);
             }
-            float mx = -INFINITY;
+
+            float alpha[4];
 #pragma unroll
-            for (int x = 0; x < 8; ++x) {
-                const bool ok = (b0 + sub * 8 + x) < n_vis;
-                sc[x] = ok ? sc[x] * args.scale : -INFINITY;
-                mx = fmaxf(mx, sc[x]);
+            for (int r = 0; r < 4; ++r) {
+                float mx = -INFINITY;
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    const bool vis = (b0 + 4 * tx + c) < n_vis[r];
+                    sc[r][c] = vis ? sc[r][c] * args.scale : -INFINITY;
+                    mx = fmaxf(mx, sc[r][c]);
+                }
+#pragma unroll
+                for (int off = 1; off < 16; off <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+                const float m_new = fmaxf(m[r], mx);
+                // rows with nothing visible yet keep weight 0 and avoid (-inf) - (-inf)
+                const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
+                alpha[r] = expf(m[r] - m_use);
+                float psum = 0.f;
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    sc[r][c] = expf(sc[r][c] - m_use);
+                    psum += sc[r][c];
+                }
+#pragma unroll
+                for (int off = 1; off < 16; off <<= 1) psum += __shfl_xor_sync(0xffffffffu, psum, off);
+                l[r] = l[r] * alpha[r] + psum;
+                m[r] = m_new;
             }
-            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
-            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-            const float m_new = fmaxf(m, mx);
-            // rows with nothing visible yet keep weight 0 and avoid (-inf) - (-inf)
-            const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
-            const float alpha = expf(m - m_use);
-            float psum = 0.f;
 #pragma unroll
-            for (int x = 0; x < 8; ++x) {
-                const float p = expf(sc[x] - m_use);
-                psum += p;
-                Ps[r * ldp + sub * 8 + x] = p;
-            }
-            psum += __shfl_xor_sync(0xffffffffu, psum, 1);
-            psum += __shfl_xor_sync(0xffffffffu, psum, 2);
-            l = l * alpha + psum;
-            m = m_new;
-            __syncwarp();
+            for (int c = 0; c < 4; ++c)
+                *reinterpret_cast<float4*>(Pt + pt_index(4 * tx + c, 4 * ty)) =
+                    make_float4(sc[0][c], sc[1][c], sc[2][c], sc[3][c]);
 #pragma unroll
-            for (int c = 0; c < kCols; ++c) {
-                const int d = sub + 4 * c;
-                if (d < D) {
-                    float acc = o[c] * alpha;
-                    for (int kk = 0; kk < kBK; ++kk) acc = fmaf(Ps[r * ldp + kk], Vs[kk * ldv + d], acc);
-                    o[c] = acc;
+            for (int r = 0; r < 4; ++r)
+#pragma unroll
+                for (int c = 0; c < kOC; ++c) o[r][c] *= alpha[r];
+            __syncthreads();
+
+            // O block: rows 4ty + r, columns 4tx + 64 (c / 4) + c % 4
+#pragma unroll 2
+            for (int key = 0; key < kBK; ++key) {
+                const float4 pa = *reinterpret_cast<const float4*>(Pt + pt_index(key, 4 * ty));
+                const float pv[4] = {pa.x, pa.y, pa.z, pa.w};
+#pragma unroll
+                for (int c4 = 0; c4 < kOC / 4; ++c4) {
+                    const float4 vb = *reinterpret_cast<const float4*>(Vs + key * kDMax + 4 * tx + 64 * c4);
+                    const float vv[4] = {vb.x, vb.y, vb.z, vb.w};
+#pragma unroll
+                    for (int r = 0; r < 4; ++r)
+#pragma unroll
+                        for (int c = 0; c < 4; ++c) o[r][4 * c4 + c] = fmaf(pv[r], vv[c], o[r][4 * c4 + c]);
                 }
             }
-            __syncwarp();
         }
     }
 
-    if (a >= L.S_loc) return;
-    const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
-    const float lse = (l > 0.f) ? m + logf(l) : -INFINITY;
-    if (args.out_mode == kOutFinal) {
-        const int64_t g = global_position(L, i, a);
-        T* dst = static_cast<T*>(args.out) + ((b * L.S + g) * H + h) * D;
 #pragma unroll
-        for (int c = 0; c < kCols; ++c) {
-            const int d = sub + 4 * c;
-            if (d < D) dst[d] = from_float<T>(o[c] * inv_l);
-        }
-        if (sub == 0) args.lse[(b * H + h) * L.S + g] = lse;
-    } else {
-        const int64_t row = ((b * L.N + i) * L.S_loc + a) * H + h;
-        float* dst = static_cast<float*>(args.out) + row * D;
+    for (int r = 0; r < 4; ++r) {
+        const int64_t a = a0 + 4 * ty + r;
+        if (a >= L.S_loc) continue;
+        const float inv_l = (l[r] > 0.f) ? 1.f / l[r] : 0.f;
+        const float lse = (l[r] > 0.f) ? m[r] + logf(l[r]) : -INFINITY;
+        if (args.out_mode == kOutFinal) {
+            const int64_t g = global_position(L, i, a);
+            T* dst = static_cast<T*>(args.out) + ((b * L.S + g) * H + h) * D;
 #pragma unroll
-        for (int c = 0; c < kCols; ++c) {
-            const int d = sub + 4 * c;
-            if (d < D) dst[d] = o[c] * inv_l;
+            for (int c = 0; c < kOC; ++c) {
+                const int d = 4 * tx + 64 * (c / 4) + c % 4;
+                if (d < D) dst[d] = from_float<T>(o[r][c] * inv_l);
+            }
+            if (tx == 0) args.lse[(b * H + h) * L.S + g] = lse;
+        } else {
+            const int64_t row = ((b * L.N + i) * L.S_loc + a) * H + h;
+            float* dst = static_cast<float*>(args.out) + row * D;
+#pragma unroll
+            for (int c = 0; c < kOC; ++c) {
+                const int d = 4 * tx + 64 * (c / 4) + c % 4;
+                if (d < D) dst[d] = o[r][c] * inv_l;
+            }
+            if (tx == 0) args.lse[row] = lse;
         }
-        if (sub == 0) args.lse[row] = lse;
     }
 }
 
 template <typename T, int kDMax>
 cudaError_t launch_typed(const void* q, const void* k, const void* v, const AttnArgs& a,
                          cudaStream_t stream) {
-    const int D = (int)a.D;
-    const size_t smem = sizeof(float) * ((size_t)kBQ * (D + 1) + (size_t)kBK * (D + 1) +
-                                         (size_t)kBK * D + (size_t)kBQ * (kBK + 1));
+    const size_t smem = sizeof(float) * ((size_t)kDMax * kBQ + 2 * (size_t)kDMax * kBK + (size_t)kBK * kBQ);
     auto kern = attn_simt_kernel<T, kDMax>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
@@ -183,7 +249,6 @@ cudaError_t launch_typed(const void* q, const void* k, const void* v, const Attn
 template <typename T>
 cudaError_t launch_dispatch(const void* q, const void* k, const void* v, const AttnArgs& a,
                             cudaStream_t stream) {
-    if (a.D <= 32) return launch_typed<T, 32>(q, k, v, a, stream);
     if (a.D <= 64) return launch_typed<T, 64>(q, k, v, a, stream);
     if (a.D <= 128) return launch_typed<T, 128>(q, k, v, a, stream);
     return launch_typed<T, 256>(q, k, v, a, stream);
