@@ -54,7 +54,8 @@ def recorded_traffic(args):
             h.update(open(os.path.join(ROOT, "long_context_exact_forward_b200", "csrc", rel), "rb").read())
         except OSError:
             return None
-    default_run = args.workload == "s128k" and args.layout == "striped" and args.heads in (0, 32)
+    default_run = (args.workload == "s128k" and args.layout == "striped" and args.heads in (0, 32)
+                   and args.kernel == "tc" and args.variant == "fused")
     if default_run and h.hexdigest().startswith(TRAFFIC_RECORD["source_sha256_prefix"]):
         return TRAFFIC_RECORD["bytes_per_launch"]
     return None
@@ -205,10 +206,12 @@ def run_reference(args, w):
 def config_dict(w, args):
     return {
         "workload": f"{w.name}: batch {w.B}, {w.H} heads, head dim {w.D}, {w.S} tokens in {w.n_ring} "
-                    f"shards of {w.S_loc}, bf16, causal, {args.layout} layout",
+                    f"shards of {w.S_loc}, {args.dtype}, causal, {args.layout} layout",
         "B": w.B, "H": w.H, "S": w.S, "D": w.D, "n_ring": w.n_ring, "causal": True,
-        "layout": args.layout, "variant": args.variant,
-        "l2": "inputs (3 x B*S*H*D bf16) larger than the 126 MB L2; no flush",
+        "layout": args.layout, "variant": args.variant, "kernel": args.kernel,
+        "l2": f"inputs (3 x B*S*H*D {args.dtype}) larger than the 126 MB L2; no flush"
+              if 3 * w.B * w.S * w.H * w.D * (4 if args.dtype == "fp32" else 2) > 126e6
+              else "inputs smaller than the 126 MB L2 (kernel-level runs; not the headline)",
     }
 
 
@@ -264,16 +267,18 @@ def run_ours(args, w):
     dev = torch.device("cuda", torch.cuda.current_device())
     stream = torch.cuda.current_stream()
     B, H, S, D, N = w.B, w.H, w.S, w.D, w.n_ring
-    q, k, v = inputs.make_qkv(B, S, H, D, torch.bfloat16, dev, w.seed + rank)
+    fp32 = args.dtype == "fp32"
+    q, k, v = inputs.make_qkv(B, S, H, D, torch.float32 if fp32 else torch.bfloat16, dev, w.seed + rank)
     out = torch.empty_like(q)
     lse = torch.empty((B, H, S), dtype=torch.float32, device=dev)
-    ws = torch.empty(ra.workspace_size(B, H, S, D, N, True, args.layout, 1, variant=args.variant),
+    ws = torch.empty(ra.workspace_size(B, H, S, D, N, True, args.layout, 0 if fp32 else 1,
+                                       variant=args.variant, kernel=args.kernel),
                      dtype=torch.uint8, device=dev)
     flops = attention_flops(B, H, S, D, True)
 
     def step(ev=None):
-        ra.forward(q, k, v, N, True, args.layout, variant=args.variant, out=out, lse=lse,
-                   workspace=ws, stream=stream, events=ev)
+        ra.forward(q, k, v, N, True, args.layout, variant=args.variant, kernel=args.kernel, out=out,
+                   lse=lse, workspace=ws, stream=stream, events=ev)
 
     for _ in range(args.warmup):
         step()
@@ -331,7 +336,7 @@ def run_ours(args, w):
                 stream.wait_event(ev_in[b])
                 if st >= 2:
                     stream.wait_event(ev_free_out[b])
-                ra.forward(dq[b][0], dq[b][1], dq[b][2], N, True, args.layout, variant=args.variant,
+                ra.forward(dq[b][0], dq[b][1], dq[b][2], N, True, args.layout, variant=args.variant, kernel=args.kernel,
                            out=do[b], lse=dl[b], workspace=ws, stream=stream)
                 ev_free_in[b].record(stream)
                 ev_done[b].record(stream)
@@ -354,7 +359,7 @@ def run_ours(args, w):
         def serial_step():
             for dst, src in zip(dq[0], (qh, kh, vh)):
                 dst.copy_(src, non_blocking=True)
-            ra.forward(dq[0][0], dq[0][1], dq[0][2], N, True, args.layout, variant=args.variant,
+            ra.forward(dq[0][0], dq[0][1], dq[0][2], N, True, args.layout, variant=args.variant, kernel=args.kernel,
                        out=do[0], lse=dl[0], workspace=ws, stream=stream)
             oh[0].copy_(do[0], non_blocking=True)
             lh[0].copy_(dl[0], non_blocking=True)
@@ -387,15 +392,26 @@ def run_ours(args, w):
     peaks, peak_src = load_peaks()
     k_ms = statistics.mean(kernel_ms)
     achieved = flops / (k_ms / 1e3) / 1e12
-    peak = peaks["bf16_tflops_sustained"]
-    roofline = {
-        "bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
-        "traffic": args.traffic_bytes if args.traffic_bytes is not None else recorded_traffic(args),
-        "peak_kind": f"bf16 dense cuBLAS, sustained ({peak_src})",
-        "frac_of_burst_peak": achieved / peaks["bf16_tflops"],
-        "kernel": "attn_tc_kernel<128> (fused ring, tcgen05)", "kernel_ms": k_ms,
-        "algorithmic_flops_per_launch": flops,
-    }
+    if args.kernel == "simt":
+        # FP32 pipe: 148 SMs x 128 FMA lanes x 2 flops at the sampled maximum SM clock
+        peak = 148 * 128 * 2 * (clk.get("sm_max_mhz") or 1965.0) * 1e6 / 1e12
+        roofline = {
+            "bound": "alu", "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+            "traffic": args.traffic_bytes,
+            "peak_kind": "FP32 FMA pipe (148 SMs x 128 lanes x 2 flops x max SM clock; derived)",
+            "kernel": f"attn_simt_kernel<{'float' if fp32 else 'bf16'}> (fp32 arithmetic)", "kernel_ms": k_ms,
+            "algorithmic_flops_per_launch": flops,
+        }
+    else:
+        peak = peaks["bf16_tflops_sustained"]
+        roofline = {
+            "bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+            "traffic": args.traffic_bytes if args.traffic_bytes is not None else recorded_traffic(args),
+            "peak_kind": f"bf16 dense cuBLAS, sustained ({peak_src})",
+            "frac_of_burst_peak": achieved / peaks["bf16_tflops"],
+            "kernel": "attn_tc_kernel<128> (fused ring, tcgen05)", "kernel_ms": k_ms,
+            "algorithmic_flops_per_launch": flops,
+        }
 
     # ---- CPU baseline: the oracle on a bounded sample (rank 0, N = 1 only)
     cpu = None
@@ -414,7 +430,7 @@ def run_ours(args, w):
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32" if fp32 else "bf16", "data": "synthetic",
         "config": config_dict(w, args),
         "pct_of_bf16_peak": {"burst_measured": value / world / peaks["bf16_tflops"],
                              "sustained_measured": value / world / peaks["bf16_tflops_sustained"],
@@ -438,6 +454,9 @@ def main():
     ap.add_argument("--layout", default="striped", choices=["contiguous", "striped", "zigzag"])
     ap.add_argument("--variant", default="fused", choices=["fused", "per_step"])
     ap.add_argument("--heads", type=int, default=0, help="override the head count (profiling runs)")
+    ap.add_argument("--kernel", default="tc", choices=["tc", "simt"],
+                    help="tc: the tcgen05 kernel (the headline); simt: the fp32 CUDA-core kernel")
+    ap.add_argument("--dtype", default="bf16", choices=["bf16", "fp32"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-hbm-kernels", action="store_true")
@@ -446,6 +465,8 @@ def main():
     ap.add_argument("--traffic-bytes", type=float, default=None,
                     help="DRAM bytes per attention launch from an ncu capture of this kernel")
     args = ap.parse_args()
+    if args.kernel == "tc" and args.dtype == "fp32":
+        ap.error("the tensor-core kernel takes bf16 inputs; fp32 runs on --kernel simt")
     w = inputs.WORKLOADS[args.workload]
     if args.heads:
         from dataclasses import replace
