@@ -18,6 +18,9 @@ merge(m, l, O, m2, l2, O2)
     Online-softmax merge identities (troisinh.com "Ring Attention", "Tai sao no hoat dong").
 layout_positions(S, n_ring, layout)
     Global position of each (shard, local index) under a layout, shape [N, S/N].
+attention_backward(q, k, v, dout, causal, threads=1)
+    Gradients (dq, dk, dv) of the plain definition for the upstream gradient dout, in fp64, each
+    [B, S, H, D] (troisinh.com "Ring Attention", "Blockwise Backward"; chain rule written out).
 """
 import ctypes
 import os
@@ -58,6 +61,9 @@ def load(path=None):
     lib.ora_merge.argtypes = [i64, i64, dp, dp, dp, dp, dp, dp]
     lib.ora_layout_positions.restype = ctypes.c_int
     lib.ora_layout_positions.argtypes = [i64, i64, ctypes.c_int, vp]
+    lib.ora_attention_backward.restype = ctypes.c_int
+    lib.ora_attention_backward.argtypes = [vp, vp, vp, vp, ctypes.c_int, i64, i64, i64, i64,
+                                           ctypes.c_int, vp, vp, vp, ctypes.c_int]
     return lib
 
 
@@ -156,3 +162,19 @@ def layout_positions(S, n_ring, layout, lib=None):
     if lib.ora_layout_positions(S, n_ring, LAYOUTS[layout], pos.ctypes.data) != 0:
         raise ValueError("layout does not split S evenly")
     return pos
+
+
+def attention_backward(q, k, v, dout, causal, threads=1, lib=None):
+    """fp64 gradients (dq, dk, dv), each [B, S, H, D], of softmax(Q K^T / sqrt(D)) V for dout."""
+    lib = lib or _get()
+    q, k, v, dout = _as_input(q), _as_input(k), _as_input(v), _as_input(dout)
+    if not (q.dtype == k.dtype == v.dtype == dout.dtype):
+        raise TypeError("q, k, v, dout must share a dtype")
+    B, S, H, D = q.shape
+    dq, dk, dv = (np.empty((B, S, H, D), dtype=np.float64) for _ in range(3))
+    rc = lib.ora_attention_backward(q.ctypes.data, k.ctypes.data, v.ctypes.data, dout.ctypes.data,
+                                    _code(q), B, H, S, D, int(bool(causal)), dq.ctypes.data,
+                                    dk.ctypes.data, dv.ctypes.data, int(threads))
+    if rc != 0:
+        raise ValueError("ora_attention_backward rejected its arguments")
+    return dq, dk, dv

@@ -22,6 +22,13 @@
 //   * ora_merge          -- the online-softmax merge identities of troisinh.com "Ring Attention",
 //                            section "Tai sao no hoat dong": m' = max(m_p, m_n),
 //                            l' = e^{m_p - m'} l_p + e^{m_n - m'} l_n, output rescaled alike.
+//   * ora_attention_backward -- the gradients dQ, dK, dV of the same plain definition for an
+//                            upstream gradient dO (troisinh.com "Ring Attention", "Blockwise
+//                            Backward": the backward pass recomputes the attention statistics
+//                            instead of storing the S x S weights).  Written out by the chain rule
+//                            with no blocking: P = softmax(S), dV = P^T dO, dP = dO V^T,
+//                            dS = P * (dP - rowsum(P * dP)), dQ = dS K / sqrt(D),
+//                            dK = dS^T Q / sqrt(D).
 //
 // Readings where the pages are silent (listed again in the design notes):
 //   * scale = 1/sqrt(D) (the toy divides the scores by dim**0.5);
@@ -244,6 +251,80 @@ int ora_ring_blockwise(const void* q, const void* k, const void* v, int dtype, i
                     lse[(b * H + h) * S + g] = m[a] + std::log(l[a]);
                 }
             }
+    return 0;
+}
+
+// Gradients of the plain definition.  dout, dq, dk, dv: [B, S, H, D] (dout in `dtype`, the
+// gradients fp64).  Each (b, h) is one task (its dk and dv rows belong to it alone); `threads`
+// host threads take whole tasks, so the result does not depend on the thread count.
+// Per query row r, in the order the chain rule gives them:
+//   s_c  = scale * q_r . k_c over the allowed keys c, lse_r = max + ln(sum exp(s - max))
+//   P_rc = exp(s_c - lse_r)                       (the softmax row)
+//   dP_rc = dO_r . v_c                            (gradient of out_r = sum_c P_rc v_c w.r.t. P_rc)
+//   dS_rc = P_rc * (dP_rc - sum_c' P_rc' dP_rc')  (softmax Jacobian)
+//   dq_r += scale * dS_rc k_c,  dk_c += scale * dS_rc q_r,  dv_c += P_rc dO_r
+// Returns 0, or -1 on a bad argument.
+int ora_attention_backward(const void* q, const void* k, const void* v, const void* dout, int dtype,
+                           int64_t B, int64_t H, int64_t S, int64_t D, int causal, double* dq,
+                           double* dk, double* dv, int threads) {
+    if (!q || !k || !v || !dout || !dq || !dk || !dv || B < 0 || H < 0 || S < 0 || D <= 0) return -1;
+    if (dtype < 0 || dtype > 2) return -1;
+    const double scale = 1.0 / std::sqrt((double)D);
+    const int64_t n_tasks = B * H;
+    std::atomic<int64_t> next{0};
+    auto worker = [&]() {
+        std::vector<double> qr(D), dor(D), s(std::max<int64_t>(S, 1)), P(std::max<int64_t>(S, 1)),
+            dP(std::max<int64_t>(S, 1));
+        for (;;) {
+            const int64_t t = next.fetch_add(1);
+            if (t >= n_tasks) break;
+            const int64_t b = t / H, h = t % H;
+            for (int64_t r = 0; r < S; ++r)
+                for (int64_t d = 0; d < D; ++d) {
+                    dq[at(b, r, h, d, S, H, D)] = 0.0;
+                    dk[at(b, r, h, d, S, H, D)] = 0.0;
+                    dv[at(b, r, h, d, S, H, D)] = 0.0;
+                }
+            for (int64_t r = 0; r < S; ++r) {
+                for (int64_t d = 0; d < D; ++d) {
+                    qr[d] = to_f64(q, dtype, at(b, r, h, d, S, H, D));
+                    dor[d] = to_f64(dout, dtype, at(b, r, h, d, S, H, D));
+                }
+                const int64_t n_keys = causal ? r + 1 : S;
+                double m = -std::numeric_limits<double>::infinity();
+                for (int64_t c = 0; c < n_keys; ++c) {
+                    double dot = 0.0;
+                    for (int64_t d = 0; d < D; ++d) dot += qr[d] * to_f64(k, dtype, at(b, c, h, d, S, H, D));
+                    s[c] = scale * dot;
+                    m = std::max(m, s[c]);
+                }
+                double l = 0.0;
+                for (int64_t c = 0; c < n_keys; ++c) l += std::exp(s[c] - m);
+                const double lse = m + std::log(l);
+                double row_dot = 0.0;  // sum_c P_rc dP_rc
+                for (int64_t c = 0; c < n_keys; ++c) {
+                    P[c] = std::exp(s[c] - lse);
+                    double dot = 0.0;
+                    for (int64_t d = 0; d < D; ++d) dot += dor[d] * to_f64(v, dtype, at(b, c, h, d, S, H, D));
+                    dP[c] = dot;
+                    row_dot += P[c] * dP[c];
+                }
+                for (int64_t c = 0; c < n_keys; ++c) {
+                    const double dS = P[c] * (dP[c] - row_dot);
+                    for (int64_t d = 0; d < D; ++d) {
+                        dq[at(b, r, h, d, S, H, D)] += scale * dS * to_f64(k, dtype, at(b, c, h, d, S, H, D));
+                        dk[at(b, c, h, d, S, H, D)] += scale * dS * qr[d];
+                        dv[at(b, c, h, d, S, H, D)] += P[c] * dor[d];
+                    }
+                }
+            }
+        }
+    };
+    const int n_threads = std::max(1, std::min<int>(threads, (int)std::max<int64_t>(n_tasks, 1)));
+    std::vector<std::thread> pool;
+    for (int w = 1; w < n_threads; ++w) pool.emplace_back(worker);
+    worker();
+    for (auto& th : pool) th.join();
     return 0;
 }
 
