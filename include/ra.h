@@ -182,6 +182,27 @@ RA_API int ra_forward_noalloc(const void* q, const void* k, const void* v, void*
                               int64_t B, int64_t H, int64_t S, int64_t D, int n_ring, int causal,
                               int layout, void* stream);
 
+/* ra_backward: gradients dq, dk, dv of out = softmax(q k^T / sqrt(D)) v (causal mask on original
+ * token positions, diagonal included, when `causal`) for the upstream gradient dout.  The
+ * backward pass recomputes the attention statistics block by block from the saved lse instead of
+ * storing the S x S weights (troisinh.com "Ring Attention", "Blockwise Backward"): dq of query
+ * shard i accumulates over the key blocks j = (i - s) mod N in ring order, and dk, dv of key block
+ * j over the query shards (j + s) mod N it visits, s = 0..N-1.
+ *   q, k, v, out, dout, dq, dk, dv: [B, S, H, D] row-major in natural token order, `dtype` (fp32 or
+ *     bf16); out and lse are the results of ra_forward on the same q, k, v, n_ring, causal
+ *     (layout only changes the order of the work, not the result).
+ *   lse: [B, H, S] fp32, natural log.
+ *   Arithmetic is fp32 on CUDA cores: Delta = rowsum(dout * out), then per tile
+ *   P = exp(q k^T / sqrt(D) - lse), dP = dout v^T, dS = P (dP - Delta), dq = dS k / sqrt(D),
+ *   dk = dS^T q / sqrt(D), dv = P^T dout; dq, dk, dv are written once each (no atomics).
+ *   D <= 128 (RA_ERR_UNSUPPORTED otherwise); pointers aligned to their element size.
+ *   The caller owns every buffer; a B*H*S fp32 scratch for Delta is allocated and freed
+ *   stream-ordered on `stream` (cudaMallocAsync / cudaFreeAsync).  Asynchronous on `stream`.
+ * Returns RA_OK or a negative status (validation errors before anything is enqueued). */
+RA_API int ra_backward(const void* q, const void* k, const void* v, const void* out, const float* lse,
+                       const void* dout, void* dq, void* dk, void* dv, int64_t B, int64_t H, int64_t S,
+                       int64_t D, int n_ring, int causal, int layout, int dtype, void* stream);
+
 /* ra_status_string: static description of a status code. */
 RA_API const char* ra_status_string(int status);
 
