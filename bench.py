@@ -32,6 +32,9 @@ sys.path.insert(0, ROOT)
 from long_context_exact_forward_b200 import inputs  # noqa: E402
 
 METRIC = "ring-attn fwd TFLOP/s (bf16, causal) and % of B200 dense BF16 tensor peak"
+# --backward runs: gradient flops counted as 2.5x the forward flops (five S x S x D products:
+# the recomputed scores, dP, dV, dQ, dK), halved for causal like the forward
+METRIC_BWD = "ring-attn bwd TFLOP/s (causal; 2.5x forward flops)"
 UNIT = "TFLOP/s"
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
@@ -280,6 +283,21 @@ def run_ours(args, w):
         ra.forward(q, k, v, N, True, args.layout, variant=args.variant, kernel=args.kernel, out=out,
                    lse=lse, workspace=ws, stream=stream, events=ev)
 
+    if args.backward:
+        # one forward pass outside the timed region supplies out and lse; a step is one ra_backward
+        gen = torch.Generator(device=dev).manual_seed(w.seed + 1000 + rank)
+        dout = torch.randn(q.shape, generator=gen, device=dev, dtype=torch.float32).to(q.dtype)
+        step()
+        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+        flops = 2.5 * attention_flops(B, H, S, D, True)
+
+        def step(ev=None):
+            if ev is not None:
+                ev[0].record(stream)
+            ra.backward(q, k, v, out, lse, dout, N, True, args.layout, dq=dq, dk=dk, dv=dv, stream=stream)
+            if ev is not None:
+                ev[1].record(stream)
+
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
@@ -392,14 +410,16 @@ def run_ours(args, w):
     peaks, peak_src = load_peaks()
     k_ms = statistics.mean(kernel_ms)
     achieved = flops / (k_ms / 1e3) / 1e12
-    if args.kernel == "simt":
+    if args.kernel == "simt" or args.backward:
         # FP32 pipe: 148 SMs x 128 FMA lanes x 2 flops at the sampled maximum SM clock
         peak = 148 * 128 * 2 * (clk.get("sm_max_mhz") or 1965.0) * 1e6 / 1e12
         roofline = {
             "bound": "alu", "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
             "traffic": args.traffic_bytes,
             "peak_kind": "FP32 FMA pipe (148 SMs x 128 lanes x 2 flops x max SM clock; derived)",
-            "kernel": f"attn_simt_kernel<{'float' if fp32 else 'bf16'}> (fp32 arithmetic)", "kernel_ms": k_ms,
+            "kernel": ("bwd_delta + bwd_dq + bwd_dkv kernels (fp32 arithmetic), timed as one ra_backward call"
+                       if args.backward else f"attn_simt_kernel<{'float' if fp32 else 'bf16'}> (fp32 arithmetic)"),
+            "kernel_ms": k_ms,
             "algorithmic_flops_per_launch": flops,
         }
     else:
@@ -427,8 +447,10 @@ def run_ours(args, w):
     # the last one a single final merge)
     launches_per_step = (1 if args.layout == "zigzag" else 0) + (
         1 if args.variant in ("fused", "auto") else N + 2 * (N - 2) + 1)
+    if args.backward:
+        launches_per_step = 3  # Delta, dq, dk/dv
     line = {
-        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "metric": METRIC_BWD if args.backward else METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f32" if fp32 else "bf16", "data": "synthetic",
         "config": config_dict(w, args),
@@ -457,6 +479,8 @@ def main():
     ap.add_argument("--kernel", default="tc", choices=["tc", "simt"],
                     help="tc: the tcgen05 kernel (the headline); simt: the fp32 CUDA-core kernel")
     ap.add_argument("--dtype", default="bf16", choices=["bf16", "fp32"])
+    ap.add_argument("--backward", action="store_true",
+                    help="time ra_backward (needs --no-e2e and --no-cpu-baseline; not the headline)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-hbm-kernels", action="store_true")
@@ -465,6 +489,8 @@ def main():
     ap.add_argument("--traffic-bytes", type=float, default=None,
                     help="DRAM bytes per attention launch from an ncu capture of this kernel")
     args = ap.parse_args()
+    if args.backward and not (args.no_e2e and args.no_cpu_baseline):
+        ap.error("--backward runs time the device call only: add --no-e2e --no-cpu-baseline")
     if args.kernel == "tc" and args.dtype == "fp32":
         ap.error("the tensor-core kernel takes bf16 inputs; fp32 runs on --kernel simt")
     w = inputs.WORKLOADS[args.workload]
