@@ -81,6 +81,8 @@ def lib():
         L.ra_forward_noalloc.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i64, ci, ci, ci, vp]
         L.ra_backward.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i64, i64, i64, i64, ci, ci, ci,
                                   ci, vp]
+        L.ra_backward_ex.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i64, i64, i64, i64, ci, ci, ci,
+                                     ci, ci, vp]
         L.ra_layout_positions.argtypes = [i64, ci, ci, vp]
         L.ra_plan_tiles.argtypes = [i64, ci, ci, ci, ci, vp]
         L.ra_plan_items.argtypes = [i64, i64, i64, i64, ci, ci, ci, vp, i64, ctypes.POINTER(ctypes.c_int64)]
@@ -91,7 +93,7 @@ def lib():
         L.ra_get_device_status.argtypes = []
         for name in ("ra_forward", "ra_forward_ex", "ra_forward_noalloc", "ra_workspace_size", "ra_permute",
                      "ra_unpermute", "ra_merge_partials", "ra_layout_positions", "ra_plan_tiles",
-                     "ra_plan_items", "ra_get_device_status", "ra_backward"):
+                     "ra_plan_items", "ra_get_device_status", "ra_backward", "ra_backward_ex"):
             getattr(L, name).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -207,11 +209,12 @@ def forward_noalloc(q, k, v, n_ring, causal=True, layout="contiguous", *, out=No
     return out, lse
 
 
-def backward(q, k, v, out, lse, dout, n_ring, causal=True, layout="contiguous", *, dq=None, dk=None,
-             dv=None, stream=None):
-    """ra_backward: gradients (dq, dk, dv) of forward(q, k, v, n_ring, causal, layout) for the upstream
-    gradient dout, recomputed block by block in ring order from the saved out and lse (fp32
-    arithmetic on CUDA cores; D <= 128).  All tensors [B, S, H, D] in q's dtype except lse."""
+def backward(q, k, v, out, lse, dout, n_ring, causal=True, layout="contiguous", *, kernel="auto", dq=None,
+             dk=None, dv=None, stream=None):
+    """ra_backward_ex: gradients (dq, dk, dv) of forward(q, k, v, n_ring, causal, layout) for the
+    upstream gradient dout, recomputed block by block in ring order from the saved out and lse.
+    kernel: "auto" (tensor cores for bf16 with D in {64, 128} and the contiguous or striped layout,
+    else CUDA cores), "tc" or "simt".  All tensors [B, S, H, D] in q's dtype except lse."""
     torch = _torch()
     _check_cuda(q, k, v, out, lse, dout)
     if not (q.shape == k.shape == v.shape == out.shape == dout.shape) or q.dim() != 4:
@@ -226,11 +229,11 @@ def backward(q, k, v, out, lse, dout, n_ring, causal=True, layout="contiguous", 
     dv = torch.empty_like(v) if dv is None else dv
     _check_cuda(dq, dk, dv)
     with torch.cuda.device(q.device):
-        rc = lib().ra_backward(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
-                               dout.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, H, S, D,
-                               int(n_ring), int(bool(causal)), LAYOUTS[layout], _dtype_code(q),
-                               _stream_handle(stream))
-    _check(rc, "ra_backward")
+        rc = lib().ra_backward_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
+                                  dout.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, H, S, D,
+                                  int(n_ring), int(bool(causal)), LAYOUTS[layout], _dtype_code(q),
+                                  KERNELS[kernel], _stream_handle(stream))
+    _check(rc, "ra_backward_ex")
     return dq, dk, dv
 
 

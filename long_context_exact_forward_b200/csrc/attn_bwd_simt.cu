@@ -15,6 +15,10 @@
 // as in the forward pass.  dK and dV of key block j travel with the block in the distributed form:
 // at step s the block visits query shard i = (j + s) mod N, and that is the order here.
 //
+// Entry points: ra_backward / ra_backward_ex (kernel choice).  bf16 inputs with D in {64, 128} and
+// the contiguous or striped layout go to the tensor-core kernels of attn_bwd_tc.cu; everything
+// else (fp32, other head dims, zigzag) to the CUDA-core kernels below.
+//
 // Kernels (one CTA of 256 threads per 64-row query tile or 64-key tile, fp32 arithmetic, inputs
 // gathered from natural order through the layout map):
 //   bwd_delta_kernel  Delta = rowsum(dO * O), one warp per row                        (HBM bound)
@@ -375,14 +379,17 @@ cudaError_t launch_grads(const void* q, const void* k, const void* v, const void
 }
 
 template <typename T>
-cudaError_t launch_backward(const void* q, const void* k, const void* v, const void* out, const void* dout,
-                            void* dq, void* dk, void* dv, float* delta, const BwdArgs& A, cudaStream_t stream) {
+cudaError_t launch_delta(const void* out, const void* dout, float* delta, const BwdArgs& A, cudaStream_t stream) {
     const int64_t rows = A.B * A.L.S * A.H;
     const int blocks = (int)((rows + 7) / 8 < 4096 ? (rows + 7) / 8 : 4096);
     bwd_delta_kernel<T><<<blocks, 256, 0, stream>>>(static_cast<const T*>(out), static_cast<const T*>(dout),
                                                      delta, A.B, A.L.S, A.H, A.D);
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
+    return cudaGetLastError();
+}
+
+template <typename T>
+cudaError_t launch_grads_simt(const void* q, const void* k, const void* v, const void* dout, void* dq, void* dk,
+                              void* dv, const BwdArgs& A, cudaStream_t stream) {
     if (A.D <= 64) return launch_grads<T, 64>(q, k, v, dout, dq, dk, dv, A, stream);
     return launch_grads<T, 128>(q, k, v, dout, dq, dk, dv, A, stream);
 }
@@ -390,21 +397,34 @@ cudaError_t launch_backward(const void* q, const void* k, const void* v, const v
 }  // namespace
 }  // namespace ra
 
-extern "C" int ra_backward(const void* q, const void* k, const void* v, const void* out, const float* lse,
-                           const void* dout, void* dq, void* dk, void* dv, int64_t B, int64_t H, int64_t S,
-                           int64_t D, int n_ring, int causal, int layout, int dtype, void* stream_handle) {
+extern "C" int ra_backward_ex(const void* q, const void* k, const void* v, const void* out, const float* lse,
+                              const void* dout, void* dq, void* dk, void* dv, int64_t B, int64_t H, int64_t S,
+                              int64_t D, int n_ring, int causal, int layout, int dtype, int kernel,
+                              void* stream_handle) {
     int rc = ra::host_check_shape(B, H, S, D, n_ring, layout, dtype);
     if (rc != RA_OK) return rc;
     if (!q || !k || !v || !out || !lse || !dout || !dq || !dk || !dv) return RA_ERR_INVALID_ARG;
+    if (kernel < RA_KERNEL_AUTO || kernel > RA_KERNEL_SIMT) return RA_ERR_INVALID_ARG;
     const uintptr_t esize = dtype == RA_DTYPE_FP32 ? 4 : 2;
     const void* ptrs[8] = {q, k, v, out, dout, dq, dk, dv};
-    for (const void* p : ptrs)
+    bool a16 = true;
+    for (const void* p : ptrs) {
         if (reinterpret_cast<uintptr_t>(p) % esize) return RA_ERR_ALIGN;
+        a16 = a16 && (reinterpret_cast<uintptr_t>(p) & 15u) == 0;
+    }
     if (reinterpret_cast<uintptr_t>(lse) & 3u) return RA_ERR_ALIGN;
     if (D > 128) {
         ra::host_set_error("ra_backward: head dims above 128 are not supported");
         return RA_ERR_UNSUPPORTED;
     }
+    int sms = 0;
+    bool sm100 = false;
+    int* status = nullptr;
+    if ((rc = ra::host_device_facts(&sms, &sm100, &status)) != RA_OK) return rc;
+    // tensor cores: bf16, D in {64, 128}, a layout the kernels read in place, 16-byte alignment
+    const bool tc_ok = sm100 && dtype == RA_DTYPE_BF16 && (D == 64 || D == 128) && layout != RA_LAYOUT_ZIGZAG && a16;
+    if (kernel == RA_KERNEL_TC && !tc_ok) return RA_ERR_UNSUPPORTED;
+    const bool use_tc = kernel != RA_KERNEL_SIMT && tc_ok;
     if (B * H * S == 0) return RA_OK;
     cudaStream_t stream = static_cast<cudaStream_t>(stream_handle);
     float* delta = nullptr;
@@ -419,11 +439,27 @@ extern "C" int ra_backward(const void* q, const void* k, const void* v, const vo
     A.scale = (float)(1.0 / std::sqrt((double)D));
     A.lse = lse;
     A.delta = delta;
-    e = dtype == RA_DTYPE_FP32
-            ? ra::launch_backward<float>(q, k, v, out, dout, dq, dk, dv, delta, A, stream)
-            : ra::launch_backward<__nv_bfloat16>(q, k, v, out, dout, dq, dk, dv, delta, A, stream);
+    e = dtype == RA_DTYPE_FP32 ? ra::launch_delta<float>(out, dout, delta, A, stream)
+                               : ra::launch_delta<__nv_bfloat16>(out, dout, delta, A, stream);
+    if (e == cudaSuccess) {
+        if (use_tc) {
+            rc = ra::launch_backward_tc(q, k, v, dout, dq, dk, dv, lse, delta, B, H, A.L, D, causal, status, stream);
+        } else {
+            e = dtype == RA_DTYPE_FP32
+                    ? ra::launch_grads_simt<float>(q, k, v, dout, dq, dk, dv, A, stream)
+                    : ra::launch_grads_simt<__nv_bfloat16>(q, k, v, dout, dq, dk, dv, A, stream);
+        }
+    }
     const cudaError_t ef = cudaFreeAsync(delta, stream);
     if (e != cudaSuccess) return ra::host_cuda_fail(e, "backward launch");
+    if (rc != RA_OK) return rc;
     if (ef != cudaSuccess) return ra::host_cuda_fail(ef, "cudaFreeAsync(delta)");
     return RA_OK;
+}
+
+extern "C" int ra_backward(const void* q, const void* k, const void* v, const void* out, const float* lse,
+                           const void* dout, void* dq, void* dk, void* dv, int64_t B, int64_t H, int64_t S,
+                           int64_t D, int n_ring, int causal, int layout, int dtype, void* stream_handle) {
+    return ra_backward_ex(q, k, v, out, lse, dout, dq, dk, dv, B, H, S, D, n_ring, causal, layout, dtype,
+                          RA_KERNEL_AUTO, stream_handle);
 }

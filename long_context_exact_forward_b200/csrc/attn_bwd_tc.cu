@@ -1,0 +1,579 @@
+// attn_bwd_tc.cu -- the backward pass on the sm_100a tensor cores (tcgen05 + TMEM + TMA), bf16 inputs.
+//
+// Same mathematics and ring order as attn_bwd_simt.cu (troisinh.com "Ring Attention", "Blockwise
+// Backward": the weights are recomputed per block from the saved lse, never stored):
+//     P = exp(S / sqrt(D) - lse),  dP = dO V^T,  dS = P (dP - Delta),  Delta = rowsum(dO * O)
+//     dQ = dS K / sqrt(D),  dK = dS^T Q / sqrt(D),  dV = P^T dO
+// with the four products of a 128 x 128 tile on the tensor cores (bf16 operands, fp32 accumulators
+// in TMEM) and the elementwise step on 128 threads, one TMEM lane (tile row) each.
+//
+// bwd_dq_tc_kernel   one CTA per 128-row query tile of shard i; key tiles of the blocks
+//                    j = (i - s) mod N in ring order.  TMEM: S [0,128), dP [128,256), dQ [256,384).
+//                    Per key tile: S = Q K^T and dP = dO V^T (SS), the elementwise warps write dS
+//                    (bf16) over the first 64 columns of S, then dQ += dS K (TS, K as the MN-major
+//                    operand, like V in the forward P V).
+// bwd_dkv_tc_kernel  one CTA per 128-key tile of shard j; query tiles of the shards
+//                    i = (j + s) mod N the block visits.  TMEM: S^T [0,128), dP^T [128,256),
+//                    dV [256,384), dK [384,512).  Per query tile: S^T = K Q^T and dP^T = V dO^T (SS),
+//                    the elementwise warps write P^T over S^T and dS^T over dP^T (bf16), then
+//                    dV += P^T dO and dK += dS^T Q (TS, dO and Q as MN-major operands).
+//
+// Roles (192 threads): warp 0 TMA producer (lane 0 issues), warp 1 MMA issuer (converged warp,
+// elect.sync picks the issuing lane) and TMEM owner, warps 2-5 elementwise (warp w reads TMEM lanes
+// 32 (w mod 4) .. +31).  The streamed tiles go through two shared-memory stages.  Every wait is
+// bounded; on give-up the CTA records RA_ERR_DEVICE_TIMEOUT, lets its copies and MMAs drain, frees
+// TMEM and exits.
+#include <cuda_bf16.h>
+
+#include "ra.h"
+#include "ra_internal.cuh"
+#include "sm100.cuh"
+
+namespace ra {
+namespace {
+using namespace sm100;
+
+constexpr int kTile = 128;
+constexpr int kThreads = 192;
+constexpr int kProducerWarp = 0, kMmaWarp = 1;
+constexpr uint32_t kTmemCols = 512;
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr int kColBlockBytes = 128 * 128;  // 128 rows x 64 bf16 (128-byte rows, 128-byte swizzle)
+
+template <int kD>
+struct BwdSmem {
+    static constexpr int kTileBytes = kTile * kD * 2;
+    uint8_t fixed[2][kTileBytes];      // dq: Q, dO of the CTA's query tile; dkv: K, V of its key tile
+    uint8_t stream[2][2][kTileBytes];  // [stage][0/1]: dq: K, V of a key tile; dkv: Q, dO of a query tile
+    float col_lse2[2][kTile];          // dkv: lse * log2(e) and Delta of the stage's 128 query rows
+    float col_delta[2][kTile];
+    uint64_t fixed_full, stage_full[2], stage_empty[2], s_full, ds_full, acc_full, drain;
+    uint32_t tmem_base;
+    int abort;
+};
+
+struct BwdTcArgs {
+    Layout32 L;
+    int B, H, D;
+    int causal;
+    float scale;
+    const float* lse;    // [B, H, S] natural
+    const float* delta;  // [B, H, S] natural
+    __nv_bfloat16* dq;   // [B, S, H, D] natural
+    __nv_bfloat16* dk;
+    __nv_bfloat16* dv;
+    uint64_t timeout_ns;
+    int* status;
+};
+
+__device__ __forceinline__ void give_up(volatile int* abort, int* status) {
+    *abort = 1;
+    atomicExch(status, RA_ERR_DEVICE_TIMEOUT);
+}
+
+__device__ __forceinline__ void tma_tile(uint8_t* dst, const CUtensorMap* map, uint64_t* bar, int kD, int h,
+                                         int a0, int shard, int b) {
+    for (int cb = 0; cb < kD / 64; ++cb) tma_load_5d(dst + cb * kColBlockBytes, map, bar, cb * 64, h, a0, shard, b);
+}
+
+// D[tmem] (+)= A B^T over the head dim, A and B K-major tiles in shared memory (SS, N = 128)
+template <int kD>
+__device__ __forceinline__ void mma_tile_ss(uint32_t d_tmem, const uint8_t* a, const uint8_t* b) {
+    constexpr uint32_t idesc = idesc_bf16_f32(kTile, kTile, 0, 0);
+    const uint32_t aa = smem_addr(a), ba = smem_addr(b);
+#pragma unroll
+    for (int kk = 0; kk < kD / 16; ++kk) {
+        const uint32_t off = (kk >> 2) * kColBlockBytes + (kk & 3) * 32;
+        warp_mma_ss(d_tmem, smem_desc_sw128(aa + off, 16, 1024), smem_desc_sw128(ba + off, 16, 1024), idesc,
+                    kk > 0);
+    }
+}
+
+// D[tmem] (+)= A[tmem, bf16, 128 x 128] B, B an MN-major 128 x kD tile in shared memory (TS, N = kD)
+template <int kD>
+__device__ __forceinline__ void mma_tile_ts(uint32_t d_tmem, uint32_t a_tmem, const uint8_t* b, bool accumulate) {
+    constexpr uint32_t idesc = idesc_bf16_f32(kTile, kD, 0, 1);
+    const uint32_t ba = smem_addr(b);
+#pragma unroll
+    for (int kk = 0; kk < kTile / 16; ++kk)
+        warp_mma_ts(d_tmem, a_tmem + kk * 8, smem_desc_sw128(ba + kk * 16 * 128, kColBlockBytes, 1024), idesc,
+                    (kk > 0 || accumulate) ? 1u : 0u);
+}
+
+// Number of live 128-key tiles of block j for the query tile at a0 of shard i.
+__device__ __forceinline__ int key_tiles(const Layout32& L, int causal, int i, int a0, int j) {
+    if (a0 >= L.S_loc) return 0;
+    const int last = a0 + kTile - 1 < L.S_loc - 1 ? a0 + kTile - 1 : L.S_loc - 1;
+    return (visible_keys(L, causal, i, last, j) + kTile - 1) / kTile;
+}
+
+// Does the query tile at a0 of shard i see any key of the key tile at c0 of block j?
+__device__ __forceinline__ bool query_tile_live(const Layout32& L, int causal, int i, int a0, int j, int c0) {
+    const int last = a0 + kTile - 1 < L.S_loc - 1 ? a0 + kTile - 1 : L.S_loc - 1;
+    return visible_keys(L, causal, i, last, j) > c0;
+}
+
+// Store 32 fp32 values (times `mul`) of one row as bf16 at dst[0..31] (only the first `n` valid).
+__device__ __forceinline__ void store_row_chunk(__nv_bfloat16* dst, const uint32_t (&v)[32], float mul, int n) {
+    if (n >= 32) {
+        uint4* d4 = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+        for (int x = 0; x < 4; ++x) {
+            uint4 u;
+            u.x = pack_bf16x2(__uint_as_float(v[8 * x + 0]) * mul, __uint_as_float(v[8 * x + 1]) * mul);
+            u.y = pack_bf16x2(__uint_as_float(v[8 * x + 2]) * mul, __uint_as_float(v[8 * x + 3]) * mul);
+            u.z = pack_bf16x2(__uint_as_float(v[8 * x + 4]) * mul, __uint_as_float(v[8 * x + 5]) * mul);
+            u.w = pack_bf16x2(__uint_as_float(v[8 * x + 6]) * mul, __uint_as_float(v[8 * x + 7]) * mul);
+            d4[x] = u;
+        }
+    } else {
+        for (int x = 0; x < n; ++x) dst[x] = __float2bfloat16_rn(__uint_as_float(v[x]) * mul);
+    }
+}
+
+// ================================================================ dQ
+template <int kD>
+__global__ void __launch_bounds__(kThreads, 1)
+    bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+                     const BwdTcArgs A) {
+    extern __shared__ uint8_t smem_raw[];
+    BwdSmem<kD>& sm = *reinterpret_cast<BwdSmem<kD>*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                                     ~static_cast<uintptr_t>(1023));
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const Layout32 L = A.L;
+    const int i = L.N - 1 - (int)blockIdx.y;  // heaviest shards first under the contiguous layout
+    const int b = (int)blockIdx.z / A.H, h = (int)blockIdx.z % A.H;
+    const int a0 = (int)blockIdx.x * kTile;
+    const uint64_t timeout = A.timeout_ns;
+    volatile int* abort = &sm.abort;
+
+    if (threadIdx.x == 0) {
+        mbar_init(&sm.fixed_full, 1);
+        for (int st = 0; st < 2; ++st) {
+            mbar_init(&sm.stage_full[st], 1);
+            mbar_init(&sm.stage_empty[st], 1);
+        }
+        mbar_init(&sm.s_full, 1);
+        mbar_init(&sm.ds_full, 4);
+        mbar_init(&sm.acc_full, 1);
+        mbar_init(&sm.drain, 1);
+        sm.abort = 0;
+        fence_barrier_init();
+    }
+    if (warp == kMmaWarp) {
+        tmem_alloc(&sm.tmem_base, kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = sm.tmem_base;
+    constexpr uint32_t kS = 0, kdP = 128, kdQ = 256;
+
+    if (warp == kProducerWarp) {
+        bool ok = true;
+        uint32_t it = 0;
+        if (lane == 0) {
+            mbar_arrive_expect_tx(&sm.fixed_full, 2 * BwdSmem<kD>::kTileBytes);
+            tma_tile(sm.fixed[0], &tm_q, &sm.fixed_full, kD, h, a0, i, b);
+            tma_tile(sm.fixed[1], &tm_do, &sm.fixed_full, kD, h, a0, i, b);
+        }
+        for (int s = 0; s < L.N && ok; ++s) {
+            const int j = ring_block32(i, s, L.N);
+            const int nt = key_tiles(L, A.causal, i, a0, j);
+            for (int kt = 0; kt < nt && ok; ++kt, ++it) {
+                const uint32_t st = it & 1;
+                ok = __all_sync(0xffffffffu, mbar_wait(&sm.stage_empty[st], ((it >> 1) & 1) ^ 1, timeout, abort));
+                if (!ok) break;
+                if (lane == 0) {
+                    mbar_arrive_expect_tx(&sm.stage_full[st], 2 * BwdSmem<kD>::kTileBytes);
+                    tma_tile(sm.stream[st][0], &tm_k, &sm.stage_full[st], kD, h, kt * kTile, j, b);
+                    tma_tile(sm.stream[st][1], &tm_v, &sm.stage_full[st], kD, h, kt * kTile, j, b);
+                }
+            }
+        }
+        if (!ok) {
+            if (lane == 0) give_up(abort, A.status);
+            // the copies in flight: the two stages' last tiles and the fixed tiles
+            for (uint32_t u = it > 2 ? it - 2 : 0; u < it; ++u)
+                mbar_wait(&sm.stage_full[u & 1], (u >> 1) & 1, timeout, nullptr);
+            mbar_wait(&sm.fixed_full, 0, timeout, nullptr);
+        }
+    } else if (warp == kMmaWarp) {
+        bool ok = true;
+        auto wait = [&](uint64_t* bar, uint32_t parity) {
+            if (!ok) return false;
+            ok = __all_sync(0xffffffffu, mbar_wait(bar, parity, timeout, abort));
+            if (ok) tc_fence_after();
+            return ok;
+        };
+        uint32_t it = 0;
+        bool any = false;
+        if (wait(&sm.fixed_full, 0)) {
+            for (int s = 0; s < L.N && ok; ++s) {
+                const int j = ring_block32(i, s, L.N);
+                const int nt = key_tiles(L, A.causal, i, a0, j);
+                for (int kt = 0; kt < nt && ok; ++kt, ++it) {
+                    const uint32_t st = it & 1;
+                    if (!wait(&sm.stage_full[st], (it >> 1) & 1)) break;
+                    // S = Q K^T and dP = dO V^T (the previous tile's dQ MMA, issued before, has read dS)
+                    mma_tile_ss<kD>(tmem + kS, sm.fixed[0], sm.stream[st][0]);
+                    mma_tile_ss<kD>(tmem + kdP, sm.fixed[1], sm.stream[st][1]);
+                    warp_mma_commit(&sm.s_full);
+                    if (!wait(&sm.ds_full, it & 1)) break;
+                    // dQ += dS K: dS (bf16) in the first 64 columns of S, K as the MN-major operand
+                    mma_tile_ts<kD>(tmem + kdQ, tmem + kS, sm.stream[st][0], any);
+                    any = true;
+                    warp_mma_commit(&sm.stage_empty[st]);
+                }
+            }
+        }
+        if (ok) warp_mma_commit(&sm.acc_full);
+        if (!ok) {
+            if (lane == 0) give_up(abort, A.status);
+            warp_mma_commit(&sm.drain);
+            mbar_wait(&sm.drain, 0, timeout, nullptr);
+        }
+    } else {
+        // elementwise: row r of the query tile
+        const int r = 32 * (warp & 3) + lane;
+        const int a = a0 + r;
+        const bool row_ok = a < L.S_loc;
+        const uint32_t lane_base = tmem + ((uint32_t)(32 * (warp & 3)) << 16);
+        const int g = row_ok ? global_position(L, i, a) : 0;
+        const size_t row_stat = ((size_t)b * A.H + h) * L.S + g;
+        const float lse2 = row_ok ? A.lse[row_stat] * kLog2e : 0.f;
+        const float del = row_ok ? A.delta[row_stat] : 0.f;
+        const float sl2 = A.scale * kLog2e;
+        bool ok = true;
+        auto wait_all = [&](uint64_t* bar, uint32_t parity) {
+            ok = __all_sync(0xffffffffu, mbar_wait(bar, parity, timeout, abort));
+            if (ok) tc_fence_after();
+            return ok;
+        };
+        uint32_t it = 0;
+        bool any = false;
+        for (int s = 0; s < L.N && ok; ++s) {
+            const int j = ring_block32(i, s, L.N);
+            const int nt = key_tiles(L, A.causal, i, a0, j);
+            const int cnt = row_ok ? visible_keys(L, A.causal, i, a, j) : 0;
+            for (int kt = 0; kt < nt && ok; ++kt, ++it) {
+                if (!wait_all(&sm.s_full, it & 1)) break;
+                any = true;
+                const int valid = cnt - kt * kTile;
+#pragma unroll 1
+                for (int c = 0; c < kTile / 32; ++c) {
+                    uint32_t sv[32], pv[32], pk[16];
+                    tmem_ld32(lane_base + kS + 32 * c, sv);
+                    tmem_ld32(lane_base + kdP + 32 * c, pv);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int x = 0; x < 16; ++x) {
+                        float ds[2];
+#pragma unroll
+                        for (int e = 0; e < 2; ++e) {
+                            const int col = 32 * c + 2 * x + e;
+                            const float p = col < valid ? ex2(fmaf(__uint_as_float(sv[2 * x + e]), sl2, -lse2)) : 0.f;
+                            ds[e] = p * (__uint_as_float(pv[2 * x + e]) - del);
+                        }
+                        pk[x] = pack_bf16x2(ds[0], ds[1]);
+                    }
+                    // dS of columns 32c..32c+31 -> TMEM columns 16c..16c+15 (already read)
+                    tmem_st16(lane_base + kS + 16 * c, pk);
+                }
+                tmem_wait_st();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&sm.ds_full);
+            }
+        }
+        if (ok && any) {
+            if (wait_all(&sm.acc_full, 0)) {
+                __nv_bfloat16* dst = A.dq + (((size_t)b * L.S + g) * A.H + h) * A.D;
+#pragma unroll 1
+                for (int c = 0; c < kD / 32; ++c) {
+                    uint32_t v[32];
+                    tmem_ld32(lane_base + kdQ + 32 * c, v);
+                    tmem_wait_ld();
+                    if (row_ok) store_row_chunk(dst + 32 * c, v, A.scale, 32);
+                }
+            }
+        } else if (ok && row_ok) {  // no visible key at all: the gradient is zero
+            __nv_bfloat16* dst = A.dq + (((size_t)b * L.S + g) * A.H + h) * A.D;
+            for (int d = 0; d < kD; ++d) dst[d] = __float2bfloat16_rn(0.f);
+        }
+        if (!ok && lane == 0) give_up(abort, A.status);
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == kMmaWarp) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+// ================================================================ dK, dV
+template <int kD>
+__global__ void __launch_bounds__(kThreads, 1)
+    bwd_dkv_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                      const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+                      const BwdTcArgs A) {
+    extern __shared__ uint8_t smem_raw[];
+    BwdSmem<kD>& sm = *reinterpret_cast<BwdSmem<kD>*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                                     ~static_cast<uintptr_t>(1023));
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const Layout32 L = A.L;
+    const int j = (int)blockIdx.y;
+    const int b = (int)blockIdx.z / A.H, h = (int)blockIdx.z % A.H;
+    const int c0 = (int)blockIdx.x * kTile;  // first local key of this tile
+    const uint64_t timeout = A.timeout_ns;
+    volatile int* abort = &sm.abort;
+
+    if (threadIdx.x == 0) {
+        mbar_init(&sm.fixed_full, 1);
+        for (int st = 0; st < 2; ++st) {
+            mbar_init(&sm.stage_full[st], 2);  // the copies (expect_tx) + the query statistics
+            mbar_init(&sm.stage_empty[st], 1);
+        }
+        mbar_init(&sm.s_full, 1);
+        mbar_init(&sm.ds_full, 4);
+        mbar_init(&sm.acc_full, 1);
+        mbar_init(&sm.drain, 1);
+        sm.abort = 0;
+        fence_barrier_init();
+    }
+    if (warp == kMmaWarp) {
+        tmem_alloc(&sm.tmem_base, kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = sm.tmem_base;
+    constexpr uint32_t kST = 0, kdPT = 128, kdV = 256, kdK = 384;
+
+    if (warp == kProducerWarp) {
+        bool ok = true;
+        uint32_t it = 0;
+        if (lane == 0) {
+            mbar_arrive_expect_tx(&sm.fixed_full, 2 * BwdSmem<kD>::kTileBytes);
+            tma_tile(sm.fixed[0], &tm_k, &sm.fixed_full, kD, h, c0, j, b);
+            tma_tile(sm.fixed[1], &tm_v, &sm.fixed_full, kD, h, c0, j, b);
+        }
+        for (int s = 0; s < L.N && ok; ++s) {
+            const int i = (j + s) % L.N;
+            for (int q0 = 0; q0 < L.S_loc && ok; q0 += kTile) {
+                if (!query_tile_live(L, A.causal, i, q0, j, c0)) continue;
+                const uint32_t st = it & 1;
+                ok = __all_sync(0xffffffffu, mbar_wait(&sm.stage_empty[st], ((it >> 1) & 1) ^ 1, timeout, abort));
+                if (!ok) break;
+                if (lane == 0) {
+                    mbar_arrive_expect_tx(&sm.stage_full[st], 2 * BwdSmem<kD>::kTileBytes);
+                    tma_tile(sm.stream[st][0], &tm_q, &sm.stage_full[st], kD, h, q0, i, b);
+                    tma_tile(sm.stream[st][1], &tm_do, &sm.stage_full[st], kD, h, q0, i, b);
+                }
+                // lse (log2 units) and Delta of the tile's query rows, for the elementwise warps
+#pragma unroll
+                for (int e = 0; e < kTile / 32; ++e) {
+                    const int r = lane * (kTile / 32) + e, a = q0 + r;
+                    float l2 = 0.f, dl = 0.f;
+                    if (a < L.S_loc) {
+                        const size_t ix = ((size_t)b * A.H + h) * L.S + global_position(L, i, a);
+                        l2 = A.lse[ix] * kLog2e;
+                        dl = A.delta[ix];
+                    }
+                    sm.col_lse2[st][r] = l2;
+                    sm.col_delta[st][r] = dl;
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&sm.stage_full[st]);
+                ++it;
+            }
+        }
+        if (!ok) {
+            if (lane == 0) give_up(abort, A.status);
+            for (uint32_t u = it > 2 ? it - 2 : 0; u < it; ++u)
+                mbar_wait(&sm.stage_full[u & 1], (u >> 1) & 1, timeout, nullptr);
+            mbar_wait(&sm.fixed_full, 0, timeout, nullptr);
+        }
+    } else if (warp == kMmaWarp) {
+        bool ok = true;
+        auto wait = [&](uint64_t* bar, uint32_t parity) {
+            if (!ok) return false;
+            ok = __all_sync(0xffffffffu, mbar_wait(bar, parity, timeout, abort));
+            if (ok) tc_fence_after();
+            return ok;
+        };
+        uint32_t it = 0;
+        bool any = false;
+        if (wait(&sm.fixed_full, 0)) {
+            for (int s = 0; s < L.N && ok; ++s) {
+                const int i = (j + s) % L.N;
+                for (int q0 = 0; q0 < L.S_loc && ok; q0 += kTile) {
+                    if (!query_tile_live(L, A.causal, i, q0, j, c0)) continue;
+                    const uint32_t st = it & 1;
+                    if (!wait(&sm.stage_full[st], (it >> 1) & 1)) break;
+                    // S^T = K Q^T and dP^T = V dO^T
+                    mma_tile_ss<kD>(tmem + kST, sm.fixed[0], sm.stream[st][0]);
+                    mma_tile_ss<kD>(tmem + kdPT, sm.fixed[1], sm.stream[st][1]);
+                    warp_mma_commit(&sm.s_full);
+                    if (!wait(&sm.ds_full, it & 1)) break;
+                    // dV += P^T dO and dK += dS^T Q (P^T over S^T, dS^T over dP^T; dO, Q MN-major)
+                    mma_tile_ts<kD>(tmem + kdV, tmem + kST, sm.stream[st][1], any);
+                    mma_tile_ts<kD>(tmem + kdK, tmem + kdPT, sm.stream[st][0], any);
+                    any = true;
+                    warp_mma_commit(&sm.stage_empty[st]);
+                    ++it;
+                }
+            }
+        }
+        if (ok) warp_mma_commit(&sm.acc_full);
+        if (!ok) {
+            if (lane == 0) give_up(abort, A.status);
+            warp_mma_commit(&sm.drain);
+            mbar_wait(&sm.drain, 0, timeout, nullptr);
+        }
+    } else {
+        // elementwise: row r = key c0 + r of this tile, columns = the 128 query rows of a tile
+        const int r = 32 * (warp & 3) + lane;
+        const int key = c0 + r;
+        const bool row_ok = key < L.S_loc;
+        const uint32_t lane_base = tmem + ((uint32_t)(32 * (warp & 3)) << 16);
+        const float sl2 = A.scale * kLog2e;
+        const int gk = row_ok ? global_position(L, j, key) : 0;
+        bool ok = true;
+        auto wait_all = [&](uint64_t* bar, uint32_t parity) {
+            ok = __all_sync(0xffffffffu, mbar_wait(bar, parity, timeout, abort));
+            if (ok) tc_fence_after();
+            return ok;
+        };
+        uint32_t it = 0;
+        bool any = false;
+        for (int s = 0; s < L.N && ok; ++s) {
+            const int i = (j + s) % L.N;
+            // queries a >= a_min of shard i see this key (positions are increasing within a shard)
+            const int a_min = !row_ok ? L.S_loc : (A.causal ? key_count(L, i, gk - 1) : 0);
+            for (int q0 = 0; q0 < L.S_loc && ok; q0 += kTile) {
+                if (!query_tile_live(L, A.causal, i, q0, j, c0)) continue;
+                const uint32_t st = it & 1;
+                if (!wait_all(&sm.s_full, it & 1)) break;
+                if (!wait_all(&sm.stage_full[st], (it >> 1) & 1)) break;  // the query statistics
+                any = true;
+#pragma unroll 1
+                for (int c = 0; c < kTile / 32; ++c) {
+                    uint32_t sv[32], pv[32], pk[16], dk16[16];
+                    tmem_ld32(lane_base + kST + 32 * c, sv);
+                    tmem_ld32(lane_base + kdPT + 32 * c, pv);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int x = 0; x < 16; ++x) {
+                        float p[2], ds[2];
+#pragma unroll
+                        for (int e = 0; e < 2; ++e) {
+                            const int col = 32 * c + 2 * x + e, a = q0 + col;
+                            const bool vis = a >= a_min && a < L.S_loc;
+                            const float pe = vis ? ex2(fmaf(__uint_as_float(sv[2 * x + e]), sl2, -sm.col_lse2[st][col])) : 0.f;
+                            p[e] = pe;
+                            ds[e] = pe * (__uint_as_float(pv[2 * x + e]) - sm.col_delta[st][col]);
+                        }
+                        pk[x] = pack_bf16x2(p[0], p[1]);
+                        dk16[x] = pack_bf16x2(ds[0], ds[1]);
+                    }
+                    tmem_st16(lane_base + kST + 16 * c, pk);
+                    tmem_st16(lane_base + kdPT + 16 * c, dk16);
+                }
+                tmem_wait_st();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&sm.ds_full);
+                ++it;
+            }
+        }
+        __nv_bfloat16* dkr = A.dk + (((size_t)b * L.S + gk) * A.H + h) * A.D;
+        __nv_bfloat16* dvr = A.dv + (((size_t)b * L.S + gk) * A.H + h) * A.D;
+        if (ok && any) {
+            if (wait_all(&sm.acc_full, 0)) {
+#pragma unroll 1
+                for (int c = 0; c < kD / 32; ++c) {
+                    uint32_t v[32];
+                    tmem_ld32(lane_base + kdV + 32 * c, v);
+                    tmem_wait_ld();
+                    if (row_ok) store_row_chunk(dvr + 32 * c, v, 1.f, 32);
+                    tmem_ld32(lane_base + kdK + 32 * c, v);
+                    tmem_wait_ld();
+                    if (row_ok) store_row_chunk(dkr + 32 * c, v, A.scale, 32);
+                }
+            }
+        } else if (ok && row_ok) {  // no query sees these keys: the gradients are zero
+            for (int d = 0; d < kD; ++d) {
+                dkr[d] = __float2bfloat16_rn(0.f);
+                dvr[d] = __float2bfloat16_rn(0.f);
+            }
+        }
+        if (!ok && lane == 0) give_up(abort, A.status);
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == kMmaWarp) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+}  // namespace
+
+static_assert(sizeof(BwdSmem<128>) + 1024 <= 232448, "shared memory of one CTA (227 KB)");
+
+// Launch both gradient kernels (after Delta is computed) for bf16 q, k, v, dout in natural order,
+// contiguous or striped layout (read in place through the strided TMA view), D in {64, 128}.
+int launch_backward_tc(const void* q, const void* k, const void* v, const void* dout, void* dq, void* dk,
+                       void* dv, const float* lse, const float* delta, int64_t B, int64_t H, const Layout& L,
+                       int64_t D, int causal, int* status, cudaStream_t stream) {
+    CUtensorMap maps[4];
+    const void* srcs[4] = {q, k, v, dout};
+    const bool striped = L.kind == RA_LAYOUT_STRIPED;
+    for (int t = 0; t < 4; ++t) {
+        const int rc = host_encode_qkv_map(&maps[t], srcs[t], B, L, H, D, striped);
+        if (rc != RA_OK) return rc;
+    }
+    BwdTcArgs A{};
+    A.L = narrow(L);
+    A.B = (int)B;
+    A.H = (int)H;
+    A.D = (int)D;
+    A.causal = causal ? 1 : 0;
+    A.scale = (float)(1.0 / sqrt((double)D));
+    A.lse = lse;
+    A.delta = delta;
+    A.dq = static_cast<__nv_bfloat16*>(dq);
+    A.dk = static_cast<__nv_bfloat16*>(dk);
+    A.dv = static_cast<__nv_bfloat16*>(dv);
+    A.timeout_ns = 2000000000ull;
+    A.status = status;
+    const dim3 grid((unsigned)((L.S_loc + kTile - 1) / kTile), (unsigned)L.N, (unsigned)(B * H));
+    cudaError_t e;
+    if (D == 64) {
+        const size_t smem = sizeof(BwdSmem<64>) + 1024;
+        if ((e = cudaFuncSetAttribute(bwd_dq_tc_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess ||
+            (e = cudaFuncSetAttribute(bwd_dkv_tc_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess)
+            return host_cuda_fail(e, "backward kernel attributes");
+        bwd_dq_tc_kernel<64><<<grid, kThreads, smem, stream>>>(maps[0], maps[1], maps[2], maps[3], A);
+        if ((e = cudaGetLastError()) != cudaSuccess) return host_cuda_fail(e, "dq launch");
+        bwd_dkv_tc_kernel<64><<<grid, kThreads, smem, stream>>>(maps[0], maps[1], maps[2], maps[3], A);
+    } else {
+        const size_t smem = sizeof(BwdSmem<128>) + 1024;
+        if ((e = cudaFuncSetAttribute(bwd_dq_tc_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess ||
+            (e = cudaFuncSetAttribute(bwd_dkv_tc_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess)
+            return host_cuda_fail(e, "backward kernel attributes");
+        bwd_dq_tc_kernel<128><<<grid, kThreads, smem, stream>>>(maps[0], maps[1], maps[2], maps[3], A);
+        if ((e = cudaGetLastError()) != cudaSuccess) return host_cuda_fail(e, "dq launch");
+        bwd_dkv_tc_kernel<128><<<grid, kThreads, smem, stream>>>(maps[0], maps[1], maps[2], maps[3], A);
+    }
+    if ((e = cudaGetLastError()) != cudaSuccess) return host_cuda_fail(e, "dkv launch");
+    return RA_OK;
+}
+
+}  // namespace ra

@@ -24,12 +24,12 @@ pytestmark = pytest.mark.gpu
 THREADS = os.cpu_count() or 1
 
 
-def grads_vs_oracle(B, H, S, D, N, causal, layout, dtype, seed=0, kernel="auto"):
+def grads_vs_oracle(B, H, S, D, N, causal, layout, dtype, seed=0, kernel="auto", bwd_kernel="auto"):
     q, k, v = inputs.make_qkv(B, S, H, D, dtype=dtype, device="cuda", seed=seed)
     g = torch.Generator(device="cuda").manual_seed(seed + 1000)
     dout = torch.randn((B, S, H, D), generator=g, device="cuda", dtype=torch.float32).to(dtype)
     out, lse = ra.forward(q, k, v, N, causal, layout, kernel=kernel)
-    dq, dk, dv = ra.backward(q, k, v, out, lse, dout, N, causal, layout)
+    dq, dk, dv = ra.backward(q, k, v, out, lse, dout, N, causal, layout, kernel=bwd_kernel)
     torch.cuda.synchronize()
     assert ra.get_device_status() == 0
     ref = oracle.attention_backward(q.cpu(), k.cpu(), v.cpu(), dout.cpu(), causal, threads=THREADS)
@@ -60,9 +60,31 @@ def test_fp32_backward(layout, causal):
 
 
 @pytest.mark.parametrize("layout", ["contiguous", "striped", "zigzag"])
-def test_bf16_backward_d128(layout):
+def test_bf16_backward_d128_simt(layout):
     # forward on the tensor-core path, backward on CUDA cores
-    grads_vs_oracle(1, 2, 1024, 128, 4, True, layout, torch.bfloat16, seed=5)
+    grads_vs_oracle(1, 2, 1024, 128, 4, True, layout, torch.bfloat16, seed=5, bwd_kernel="simt")
+
+
+@pytest.mark.parametrize("layout", ["contiguous", "striped"])
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("D", [64, 128])
+def test_bf16_backward_tensor_cores(layout, causal, D):
+    grads_vs_oracle(1, 2, 1024, D, 4, causal, layout, torch.bfloat16, seed=6 + D, bwd_kernel="tc")
+
+
+def test_bf16_backward_tensor_cores_ragged():
+    # S_loc = 200: a ragged last 128-row tile in every shard
+    grads_vs_oracle(2, 2, 600, 128, 3, True, "striped", torch.bfloat16, seed=21, bwd_kernel="tc")
+    grads_vs_oracle(1, 2, 600, 64, 3, True, "contiguous", torch.bfloat16, seed=22, bwd_kernel="tc")
+
+
+def test_backward_auto_picks_a_path_for_every_layout():
+    # zigzag falls to CUDA cores under "auto"; asking for tensor cores there is refused
+    grads_vs_oracle(1, 1, 512, 128, 4, True, "zigzag", torch.bfloat16, seed=23)
+    q = torch.zeros(1, 512, 1, 128, device="cuda", dtype=torch.bfloat16)
+    lse = torch.zeros(1, 1, 512, device="cuda")
+    with pytest.raises(ra.RAError):
+        ra.backward(q, q, q, q, lse, q, 4, True, "zigzag", kernel="tc")
 
 
 def test_ragged_tiles_and_odd_head_dim():
