@@ -294,7 +294,8 @@ def run_ours(args, w):
         def step(ev=None):
             if ev is not None:
                 ev[0].record(stream)
-            ra.backward(q, k, v, out, lse, dout, N, True, args.layout, dq=dq, dk=dk, dv=dv, stream=stream)
+            ra.backward(q, k, v, out, lse, dout, N, True, args.layout, kernel=args.bwd_kernel, dq=dq, dk=dk,
+                        dv=dv, stream=stream)
             if ev is not None:
                 ev[1].record(stream)
 
@@ -410,7 +411,8 @@ def run_ours(args, w):
     peaks, peak_src = load_peaks()
     k_ms = statistics.mean(kernel_ms)
     achieved = flops / (k_ms / 1e3) / 1e12
-    if args.kernel == "simt" or args.backward:
+    bwd_tc = args.backward and args.bwd_kernel != "simt" and not fp32 and D in (64, 128) and args.layout != "zigzag"
+    if args.kernel == "simt" or (args.backward and not bwd_tc):
         # FP32 pipe: 148 SMs x 128 FMA lanes x 2 flops at the sampled maximum SM clock
         peak = 148 * 128 * 2 * (clk.get("sm_max_mhz") or 1965.0) * 1e6 / 1e12
         roofline = {
@@ -426,10 +428,13 @@ def run_ours(args, w):
         peak = peaks["bf16_tflops_sustained"]
         roofline = {
             "bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
-            "traffic": args.traffic_bytes if args.traffic_bytes is not None else recorded_traffic(args),
+            "traffic": (args.traffic_bytes if args.traffic_bytes is not None
+                        else None if args.backward else recorded_traffic(args)),
             "peak_kind": f"bf16 dense cuBLAS, sustained ({peak_src})",
             "frac_of_burst_peak": achieved / peaks["bf16_tflops"],
-            "kernel": "attn_tc_kernel<128> (fused ring, tcgen05)", "kernel_ms": k_ms,
+            "kernel": ("bwd_dq_tc_kernel + bwd_dkv_tc_kernel (tcgen05), timed as one ra_backward call"
+                       if args.backward else "attn_tc_kernel<128> (fused ring, tcgen05)"),
+            "kernel_ms": k_ms,
             "algorithmic_flops_per_launch": flops,
         }
 
@@ -479,6 +484,8 @@ def main():
     ap.add_argument("--kernel", default="tc", choices=["tc", "simt"],
                     help="tc: the tcgen05 kernel (the headline); simt: the fp32 CUDA-core kernel")
     ap.add_argument("--dtype", default="bf16", choices=["bf16", "fp32"])
+    ap.add_argument("--bwd-kernel", default="auto", choices=["auto", "tc", "simt"],
+                    help="backward path for --backward runs (auto: tensor cores where they apply)")
     ap.add_argument("--backward", action="store_true",
                     help="time ra_backward (needs --no-e2e and --no-cpu-baseline; not the headline)")
     ap.add_argument("--no-e2e", action="store_true")
