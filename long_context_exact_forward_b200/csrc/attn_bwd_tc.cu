@@ -8,10 +8,13 @@
 // in TMEM) and the elementwise step on 128 threads, one TMEM lane (tile row) each.
 //
 // bwd_dq_tc_kernel   one CTA per 128-row query tile of shard i; key tiles of the blocks
-//                    j = (i - s) mod N in ring order.  TMEM: S [0,128), dP [128,256), dQ [256,384).
-//                    Per key tile: S = Q K^T and dP = dO V^T (SS), the elementwise warps write dS
-//                    (bf16) over the first 64 columns of S, then dQ += dS K (TS, K as the MN-major
-//                    operand, like V in the forward P V).
+//                    j = (i - s) mod N in ring order.  TMEM: S of even / odd tiles [0,128) /
+//                    [128,256), dP [256,384), dQ [384,512).  Per key tile t: S = Q K^T and dP = dO V^T
+//                    (SS), the elementwise warps write dS (bf16) over the first 64 columns of S_t,
+//                    then dQ += dS K (TS, K as the MN-major operand, like V in the forward P V).
+//                    S of tile t + 1 is computed while the elementwise warps work on tile t, and
+//                    dP of tile t + 1 goes before dQ of tile t, so the elementwise warps wait only
+//                    for one product between tiles.
 // bwd_dkv_tc_kernel  one CTA per 128-key tile of shard j; query tiles of the shards
 //                    i = (j + s) mod N the block visits.  TMEM: S^T [0,128), dP^T [128,256),
 //                    dV [256,384), dK [384,512).  Per query tile: S^T = K Q^T and dP^T = V dO^T (SS),
@@ -169,7 +172,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = sm.tmem_base;
-    constexpr uint32_t kS = 0, kdP = 128, kdQ = 256;
+    // S of tile t in [128 (t mod 2), +128): the next tile's S is computed while the elementwise
+    // warps work on this one
+    constexpr uint32_t kdP = 256, kdQ = 384;
 
     if (warp == kProducerWarp) {
         bool ok = true;
@@ -208,25 +213,30 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (ok) tc_fence_after();
             return ok;
         };
-        uint32_t it = 0;
-        bool any = false;
-        if (wait(&sm.fixed_full, 0)) {
-            for (int s = 0; s < L.N && ok; ++s) {
-                const int j = ring_block32(i, s, L.N);
-                const int nt = key_tiles(L, A.causal, i, a0, j);
-                for (int kt = 0; kt < nt && ok; ++kt, ++it) {
-                    const uint32_t st = it & 1;
-                    if (!wait(&sm.stage_full[st], (it >> 1) & 1)) break;
-                    // S = Q K^T and dP = dO V^T (the previous tile's dQ MMA, issued before, has read dS)
-                    mma_tile_ss<kD>(tmem + kS, sm.fixed[0], sm.stream[st][0]);
-                    mma_tile_ss<kD>(tmem + kdP, sm.fixed[1], sm.stream[st][1]);
-                    warp_mma_commit(&sm.s_full);
-                    if (!wait(&sm.ds_full, it & 1)) break;
-                    // dQ += dS K: dS (bf16) in the first 64 columns of S, K as the MN-major operand
-                    mma_tile_ts<kD>(tmem + kdQ, tmem + kS, sm.stream[st][0], any);
-                    any = true;
-                    warp_mma_commit(&sm.stage_empty[st]);
+        uint32_t n_tiles = 0;  // key tiles of all ring steps, in the order the producer loads them
+        for (int s = 0; s < L.N; ++s) n_tiles += key_tiles(L, A.causal, i, a0, ring_block32(i, s, L.N));
+        if (wait(&sm.fixed_full, 0) && n_tiles > 0 && wait(&sm.stage_full[0], 0)) {
+            mma_tile_ss<kD>(tmem + 0, sm.fixed[0], sm.stream[0][0]);
+            mma_tile_ss<kD>(tmem + kdP, sm.fixed[1], sm.stream[0][1]);
+            warp_mma_commit(&sm.s_full);
+            for (uint32_t t = 0; t < n_tiles && ok; ++t) {
+                const uint32_t st = t & 1, sn = (t + 1) & 1;
+                const bool more = t + 1 < n_tiles;
+                // S of the next tile into the other S buffer (its dS was read by the dQ MMA of tile
+                // t - 1, issued before), while the elementwise warps work on tile t
+                if (more) {
+                    if (!wait(&sm.stage_full[sn], ((t + 1) >> 1) & 1)) break;
+                    mma_tile_ss<kD>(tmem + 128 * sn, sm.fixed[0], sm.stream[sn][0]);
                 }
+                if (!wait(&sm.ds_full, t & 1)) break;
+                // dP of the next tile (the elementwise warps have read dP of this one), then
+                // dQ += dS K of this tile: dS (bf16) in the first 64 columns of S_t, K MN-major
+                if (more) {
+                    mma_tile_ss<kD>(tmem + kdP, sm.fixed[1], sm.stream[sn][1]);
+                    warp_mma_commit(&sm.s_full);
+                }
+                mma_tile_ts<kD>(tmem + kdQ, tmem + 128 * st, sm.stream[st][0], t > 0);
+                warp_mma_commit(&sm.stage_empty[st]);
             }
         }
         if (ok) warp_mma_commit(&sm.acc_full);
@@ -262,6 +272,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (!wait_all(&sm.s_full, it & 1)) break;
                 any = true;
                 const int valid = cnt - kt * kTile;
+                const uint32_t kS = 128 * (it & 1);
 #pragma unroll 1
                 for (int c = 0; c < kTile / 32; ++c) {
                     uint32_t sv[32], pv[32], pk[16];
