@@ -50,7 +50,7 @@ struct BwdSmem {
     uint8_t stream[2][2][kTileBytes];  // [stage][0/1]: dq: K, V of a key tile; dkv: Q, dO of a query tile
     float col_lse2[2][kTile];          // dkv: lse * log2(e) and Delta of the stage's 128 query rows
     float col_delta[2][kTile];
-    uint64_t fixed_full, stage_full[2], stage_empty[2], s_full, ds_full, acc_full, drain;
+    uint64_t fixed_full, stage_full[2], stage_empty[2], s_full, dp_full, ds_full, acc_full, drain;
     uint32_t tmem_base;
     int abort;
 };
@@ -68,6 +68,26 @@ struct BwdTcArgs {
     uint64_t timeout_ns;
     int* status;
 };
+
+// Each thread reads 16 consecutive 32-bit columns of its own TMEM lane.
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+        "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+          "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr));
+}
+
+// Wait for the asynchronous TMEM loads and tie the destination registers to the wait, so that no
+// use of them is scheduled before it.
+template <int N>
+__device__ __forceinline__ void wait_ld_tied(uint32_t (&r)[N]) {
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+    for (int x = 0; x < N; ++x) asm volatile("" : "+r"(r[x]));
+}
 
 __device__ __forceinline__ void give_up(volatile int* abort, int* status) {
     *abort = 1;
@@ -158,6 +178,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&sm.stage_empty[st], 1);
         }
         mbar_init(&sm.s_full, 1);
+        mbar_init(&sm.dp_full, 1);
         mbar_init(&sm.ds_full, 4);
         mbar_init(&sm.acc_full, 1);
         mbar_init(&sm.drain, 1);
@@ -278,7 +299,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     uint32_t sv[32], pv[32], pk[16];
                     tmem_ld32(lane_base + kS + 32 * c, sv);
                     tmem_ld32(lane_base + kdP + 32 * c, pv);
-                    tmem_wait_ld();
+                    wait_ld_tied(sv);
+                    wait_ld_tied(pv);
 #pragma unroll
                     for (int x = 0; x < 16; ++x) {
                         float ds[2];
@@ -306,7 +328,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int c = 0; c < kD / 32; ++c) {
                     uint32_t v[32];
                     tmem_ld32(lane_base + kdQ + 32 * c, v);
-                    tmem_wait_ld();
+                    wait_ld_tied(v);
                     if (row_ok) store_row_chunk(dst + 32 * c, v, A.scale, 32);
                 }
             }
@@ -349,6 +371,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&sm.stage_empty[st], 1);
         }
         mbar_init(&sm.s_full, 1);
+        mbar_init(&sm.dp_full, 1);
         mbar_init(&sm.ds_full, 4);
         mbar_init(&sm.acc_full, 1);
         mbar_init(&sm.drain, 1);
@@ -417,26 +440,33 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (ok) tc_fence_after();
             return ok;
         };
-        uint32_t it = 0;
-        bool any = false;
-        if (wait(&sm.fixed_full, 0)) {
-            for (int s = 0; s < L.N && ok; ++s) {
-                const int i = (j + s) % L.N;
-                for (int q0 = 0; q0 < L.S_loc && ok; q0 += kTile) {
-                    if (!query_tile_live(L, A.causal, i, q0, j, c0)) continue;
-                    const uint32_t st = it & 1;
-                    if (!wait(&sm.stage_full[st], (it >> 1) & 1)) break;
-                    // S^T = K Q^T and dP^T = V dO^T
-                    mma_tile_ss<kD>(tmem + kST, sm.fixed[0], sm.stream[st][0]);
-                    mma_tile_ss<kD>(tmem + kdPT, sm.fixed[1], sm.stream[st][1]);
+        uint32_t n_tiles = 0;  // live query tiles over the ring steps, in the producer's order
+        for (int s = 0; s < L.N; ++s)
+            for (int q0 = 0; q0 < L.S_loc; q0 += kTile)
+                n_tiles += query_tile_live(L, A.causal, (j + s) % L.N, q0, j, c0) ? 1u : 0u;
+        if (wait(&sm.fixed_full, 0) && n_tiles > 0 && wait(&sm.stage_full[0], 0)) {
+            mma_tile_ss<kD>(tmem + kST, sm.fixed[0], sm.stream[0][0]);
+            warp_mma_commit(&sm.s_full);
+            mma_tile_ss<kD>(tmem + kdPT, sm.fixed[1], sm.stream[0][1]);
+            warp_mma_commit(&sm.dp_full);
+            for (uint32_t t = 0; t < n_tiles && ok; ++t) {
+                const uint32_t st = t & 1, sn = (t + 1) & 1;
+                const bool more = t + 1 < n_tiles;
+                if (!wait(&sm.ds_full, t & 1)) break;
+                // dV += P^T dO (P^T over S^T), then S^T of the next tile into the columns just read,
+                // so the elementwise warps start its exponentials while dK and dP^T run
+                mma_tile_ts<kD>(tmem + kdV, tmem + kST, sm.stream[st][1], t > 0);
+                if (more) {
+                    if (!wait(&sm.stage_full[sn], ((t + 1) >> 1) & 1)) break;
+                    mma_tile_ss<kD>(tmem + kST, sm.fixed[0], sm.stream[sn][0]);
                     warp_mma_commit(&sm.s_full);
-                    if (!wait(&sm.ds_full, it & 1)) break;
-                    // dV += P^T dO and dK += dS^T Q (P^T over S^T, dS^T over dP^T; dO, Q MN-major)
-                    mma_tile_ts<kD>(tmem + kdV, tmem + kST, sm.stream[st][1], any);
-                    mma_tile_ts<kD>(tmem + kdK, tmem + kdPT, sm.stream[st][0], any);
-                    any = true;
-                    warp_mma_commit(&sm.stage_empty[st]);
-                    ++it;
+                }
+                // dK += dS^T Q (dS^T over dP^T), then dP^T of the next tile
+                mma_tile_ts<kD>(tmem + kdK, tmem + kdPT, sm.stream[st][0], t > 0);
+                warp_mma_commit(&sm.stage_empty[st]);
+                if (more) {
+                    mma_tile_ss<kD>(tmem + kdPT, sm.fixed[1], sm.stream[sn][1]);
+                    warp_mma_commit(&sm.dp_full);
                 }
             }
         }
@@ -472,27 +502,45 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (!wait_all(&sm.s_full, it & 1)) break;
                 if (!wait_all(&sm.stage_full[st], (it >> 1) & 1)) break;  // the query statistics
                 any = true;
+                // phase 1 (S^T ready): P^T = exp(S^T / sqrt(D) - lse), bf16, over the first 64
+                // columns of S^T (chunk c writes columns 16c.., already read)
 #pragma unroll 1
                 for (int c = 0; c < kTile / 32; ++c) {
-                    uint32_t sv[32], pv[32], pk[16], dk16[16];
+                    uint32_t sv[32], pk[16];
                     tmem_ld32(lane_base + kST + 32 * c, sv);
-                    tmem_ld32(lane_base + kdPT + 32 * c, pv);
-                    tmem_wait_ld();
+                    wait_ld_tied(sv);
 #pragma unroll
                     for (int x = 0; x < 16; ++x) {
-                        float p[2], ds[2];
+                        float p[2];
 #pragma unroll
                         for (int e = 0; e < 2; ++e) {
                             const int col = 32 * c + 2 * x + e, a = q0 + col;
                             const bool vis = a >= a_min && a < L.S_loc;
-                            const float pe = vis ? ex2(fmaf(__uint_as_float(sv[2 * x + e]), sl2, -sm.col_lse2[st][col])) : 0.f;
-                            p[e] = pe;
-                            ds[e] = pe * (__uint_as_float(pv[2 * x + e]) - sm.col_delta[st][col]);
+                            p[e] = vis ? ex2(fmaf(__uint_as_float(sv[2 * x + e]), sl2, -sm.col_lse2[st][col])) : 0.f;
                         }
                         pk[x] = pack_bf16x2(p[0], p[1]);
-                        dk16[x] = pack_bf16x2(ds[0], ds[1]);
                     }
                     tmem_st16(lane_base + kST + 16 * c, pk);
+                }
+                // phase 2 (dP^T ready): dS^T = P^T (dP^T - Delta) from the stored bf16 P^T, over the
+                // first 64 columns of dP^T
+                tmem_wait_st();
+                if (!wait_all(&sm.dp_full, it & 1)) break;
+#pragma unroll 1
+                for (int c = 0; c < kTile / 32; ++c) {
+                    uint32_t pv[32], pb[16], dk16[16];
+                    tmem_ld32(lane_base + kdPT + 32 * c, pv);
+                    tmem_ld16(lane_base + kST + 16 * c, pb);
+                    wait_ld_tied(pv);
+                    wait_ld_tied(pb);
+#pragma unroll
+                    for (int x = 0; x < 16; ++x) {
+                        const float p0 = __uint_as_float(pb[x] << 16), p1 = __uint_as_float(pb[x] & 0xffff0000u);
+                        const int col = 32 * c + 2 * x;
+                        const float d0 = p0 * (__uint_as_float(pv[2 * x]) - sm.col_delta[st][col]);
+                        const float d1 = p1 * (__uint_as_float(pv[2 * x + 1]) - sm.col_delta[st][col + 1]);
+                        dk16[x] = pack_bf16x2(d0, d1);
+                    }
                     tmem_st16(lane_base + kdPT + 16 * c, dk16);
                 }
                 tmem_wait_st();
@@ -510,10 +558,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int c = 0; c < kD / 32; ++c) {
                     uint32_t v[32];
                     tmem_ld32(lane_base + kdV + 32 * c, v);
-                    tmem_wait_ld();
+                    wait_ld_tied(v);
                     if (row_ok) store_row_chunk(dvr + 32 * c, v, 1.f, 32);
                     tmem_ld32(lane_base + kdK + 32 * c, v);
-                    tmem_wait_ld();
+                    wait_ld_tied(v);
                     if (row_ok) store_row_chunk(dkr + 32 * c, v, A.scale, 32);
                 }
             }
