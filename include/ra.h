@@ -192,13 +192,14 @@ RA_API int ra_forward_noalloc(const void* q, const void* k, const void* v, void*
  *     bf16); out and lse are the results of ra_forward on the same q, k, v, n_ring, causal
  *     (layout only changes the order of the work, not the result).
  *   lse: [B, H, S] fp32, natural log.
- *   Arithmetic (CUDA-core path; the tensor-core path of ra_backward_ex takes bf16, D in {64, 128},
- *   contiguous or striped): Delta = rowsum(dout * out), then per tile
+ *   Arithmetic (CUDA-core path; the tensor-core path, taken for bf16 with D in {64, 128}, is
+ *   described under ra_backward_ex): Delta = rowsum(dout * out), then per tile
  *   P = exp(q k^T / sqrt(D) - lse), dP = dout v^T, dS = P (dP - Delta), dq = dS k / sqrt(D),
  *   dk = dS^T q / sqrt(D), dv = P^T dout; dq, dk, dv are written once each (no atomics).
  *   D <= 128 (RA_ERR_UNSUPPORTED otherwise); pointers aligned to their element size.
- *   The caller owns every buffer; a B*H*S fp32 scratch for Delta is allocated and freed
- *   stream-ordered on `stream` (cudaMallocAsync / cudaFreeAsync).  Asynchronous on `stream`.
+ *   The caller owns every buffer; scratch (B*H*S fp32 for Delta, plus shard-major copies for
+ *   zigzag on the tensor-core path) is allocated and freed stream-ordered on `stream`
+ *   (cudaMallocAsync / cudaFreeAsync).  Asynchronous on `stream`.
  * Returns RA_OK or a negative status (validation errors before anything is enqueued). */
 RA_API int ra_backward(const void* q, const void* k, const void* v, const void* out, const float* lse,
                        const void* dout, void* dq, void* dk, void* dv, int64_t B, int64_t H, int64_t S,
@@ -207,8 +208,9 @@ RA_API int ra_backward(const void* q, const void* k, const void* v, const void* 
 /* ra_backward_ex: ra_backward with the kernel choice (no counterpart on the pages; for callers and
  * tests that pick the path):
  *   RA_KERNEL_AUTO  tensor cores when they apply, else CUDA cores (what ra_backward does);
- *   RA_KERNEL_TC    tcgen05 kernels: bf16, D in {64, 128}, contiguous or striped layout, all eight
- *                   tensors 16-byte aligned, sm_100 (RA_ERR_UNSUPPORTED otherwise).  S and dP (or
+ *   RA_KERNEL_TC    tcgen05 kernels: bf16, D in {64, 128}, all eight tensors 16-byte aligned, sm_100
+ *                   (RA_ERR_UNSUPPORTED otherwise); zigzag inputs are first copied to shard-major
+ *                   order in stream-ordered scratch (4 x B*S*H*D bf16).  S and dP (or
  *                   their transposes) and the three gradient products run on the tensor cores
  *                   with fp32 accumulation; P and dS are rounded to bf16 as the product operands;
  *                   the elementwise step is fp32.  Bounded waits report RA_ERR_DEVICE_TIMEOUT

@@ -15,9 +15,9 @@
 // as in the forward pass.  dK and dV of key block j travel with the block in the distributed form:
 // at step s the block visits query shard i = (j + s) mod N, and that is the order here.
 //
-// Entry points: ra_backward / ra_backward_ex (kernel choice).  bf16 inputs with D in {64, 128} and
-// the contiguous or striped layout go to the tensor-core kernels of attn_bwd_tc.cu; everything
-// else (fp32, other head dims, zigzag) to the CUDA-core kernels below.
+// Entry points: ra_backward / ra_backward_ex (kernel choice).  bf16 inputs with D in {64, 128} go to
+// the tensor-core kernels of attn_bwd_tc.cu; everything else (fp32, other head dims) to the
+// CUDA-core kernels below.
 //
 // Kernels (one CTA of 256 threads per 64-row query tile or 64-key tile, fp32 arithmetic, inputs
 // gathered from natural order through the layout map):
@@ -421,15 +421,21 @@ extern "C" int ra_backward_ex(const void* q, const void* k, const void* v, const
     bool sm100 = false;
     int* status = nullptr;
     if ((rc = ra::host_device_facts(&sms, &sm100, &status)) != RA_OK) return rc;
-    // tensor cores: bf16, D in {64, 128}, a layout the kernels read in place, 16-byte alignment
-    const bool tc_ok = sm100 && dtype == RA_DTYPE_BF16 && (D == 64 || D == 128) && layout != RA_LAYOUT_ZIGZAG && a16;
+    // tensor cores: bf16, D in {64, 128}, 16-byte alignment (zigzag through shard-major copies)
+    const bool tc_ok = sm100 && dtype == RA_DTYPE_BF16 && (D == 64 || D == 128) && a16;
     if (kernel == RA_KERNEL_TC && !tc_ok) return RA_ERR_UNSUPPORTED;
     const bool use_tc = kernel != RA_KERNEL_SIMT && tc_ok;
     if (B * H * S == 0) return RA_OK;
     cudaStream_t stream = static_cast<cudaStream_t>(stream_handle);
-    float* delta = nullptr;
-    cudaError_t e = cudaMallocAsync(reinterpret_cast<void**>(&delta), sizeof(float) * (size_t)(B * H * S), stream);
-    if (e != cudaSuccess) return ra::host_cuda_fail(e, "cudaMallocAsync(delta)");
+    // scratch: Delta, and for the tensor-core path with zigzag the shard-major q, k, v, dout
+    const size_t delta_bytes = (sizeof(float) * (size_t)(B * H * S) + 255) / 256 * 256;
+    const size_t copy_bytes = ((size_t)(B * S * H * D) * 2 + 255) / 256 * 256;
+    const bool copies = use_tc && layout == RA_LAYOUT_ZIGZAG;
+    uint8_t* scratch = nullptr;
+    cudaError_t e = cudaMallocAsync(reinterpret_cast<void**>(&scratch), delta_bytes + (copies ? 4 * copy_bytes : 0),
+                                    stream);
+    if (e != cudaSuccess) return ra::host_cuda_fail(e, "cudaMallocAsync(backward scratch)");
+    float* delta = reinterpret_cast<float*>(scratch);
     ra::BwdArgs A{};
     A.L = ra::Layout{S, (int64_t)n_ring, S / n_ring, layout};
     A.B = B;
@@ -443,17 +449,18 @@ extern "C" int ra_backward_ex(const void* q, const void* k, const void* v, const
                                : ra::launch_delta<__nv_bfloat16>(out, dout, delta, A, stream);
     if (e == cudaSuccess) {
         if (use_tc) {
-            rc = ra::launch_backward_tc(q, k, v, dout, dq, dk, dv, lse, delta, B, H, A.L, D, causal, status, stream);
+            rc = ra::launch_backward_tc(q, k, v, dout, dq, dk, dv, lse, delta, B, H, A.L, D, causal, status,
+                                        copies ? scratch + delta_bytes : nullptr, stream);
         } else {
             e = dtype == RA_DTYPE_FP32
                     ? ra::launch_grads_simt<float>(q, k, v, dout, dq, dk, dv, A, stream)
                     : ra::launch_grads_simt<__nv_bfloat16>(q, k, v, dout, dq, dk, dv, A, stream);
         }
     }
-    const cudaError_t ef = cudaFreeAsync(delta, stream);
+    const cudaError_t ef = cudaFreeAsync(scratch, stream);
     if (e != cudaSuccess) return ra::host_cuda_fail(e, "backward launch");
     if (rc != RA_OK) return rc;
-    if (ef != cudaSuccess) return ra::host_cuda_fail(ef, "cudaFreeAsync(delta)");
+    if (ef != cudaSuccess) return ra::host_cuda_fail(ef, "cudaFreeAsync(backward scratch)");
     return RA_OK;
 }
 

@@ -7,6 +7,9 @@
 // with the four products of a 128 x 128 tile on the tensor cores (bf16 operands, fp32 accumulators
 // in TMEM) and the elementwise step on 128 threads, one TMEM lane (tile row) each.
 //
+// Inputs are read through 5-D TMA maps: in place for the contiguous and striped layouts, from
+// shard-major copies for zigzag.
+//
 // bwd_dq_tc_kernel   one CTA per 128-row query tile of shard i; key tiles of the blocks
 //                    j = (i - s) mod N in ring order.  TMEM: S of even / odd tiles [0,128) /
 //                    [128,256), dP [256,384), dQ [384,512).  Per key tile t: S = Q K^T and dP = dO V^T
@@ -587,13 +590,25 @@ __global__ void __launch_bounds__(kThreads, 1)
 static_assert(sizeof(BwdSmem<128>) + 1024 <= 232448, "shared memory of one CTA (227 KB)");
 
 // Launch both gradient kernels (after Delta is computed) for bf16 q, k, v, dout in natural order,
-// contiguous or striped layout (read in place through the strided TMA view), D in {64, 128}.
+// D in {64, 128}.  Contiguous and striped inputs are read in place (striped through the strided
+// TMA view); for zigzag, `shard_major` holds room for shard-major copies of q, k, v and dout
+// (4 x B*S*H*D bf16, 256-byte aligned each), made here with the permute kernel.  The gradients are
+// written in natural order either way.
 int launch_backward_tc(const void* q, const void* k, const void* v, const void* dout, void* dq, void* dk,
                        void* dv, const float* lse, const float* delta, int64_t B, int64_t H, const Layout& L,
-                       int64_t D, int causal, int* status, cudaStream_t stream) {
+                       int64_t D, int causal, int* status, void* shard_major, cudaStream_t stream) {
     CUtensorMap maps[4];
     const void* srcs[4] = {q, k, v, dout};
     const bool striped = L.kind == RA_LAYOUT_STRIPED;
+    if (L.kind == RA_LAYOUT_ZIGZAG) {
+        if (!shard_major) return RA_ERR_NO_WORKSPACE;
+        const size_t bytes = ((size_t)(B * L.S * H * D) * 2 + 255) / 256 * 256;
+        void* dst[4];
+        for (int t = 0; t < 4; ++t) dst[t] = static_cast<uint8_t*>(shard_major) + t * bytes;
+        const cudaError_t e = launch_permute(srcs, dst, 4, B, L, H, D, 2, false, stream);
+        if (e != cudaSuccess) return host_cuda_fail(e, "permute launch");
+        for (int t = 0; t < 4; ++t) srcs[t] = dst[t];
+    }
     for (int t = 0; t < 4; ++t) {
         const int rc = host_encode_qkv_map(&maps[t], srcs[t], B, L, H, D, striped);
         if (rc != RA_OK) return rc;

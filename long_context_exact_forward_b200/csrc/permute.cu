@@ -16,9 +16,11 @@ namespace {
 
 constexpr int kRowsPerBlock = 8;  // 8 warps, one row each
 
+constexpr int kMaxTensors = 4;  // tensors moved by one launch (grid.y)
+
 struct PermuteArgs {
-    const void* src[3];
-    void* dst[3];
+    const void* src[kMaxTensors];
+    void* dst[kMaxTensors];
 };
 
 // Vector path: row bytes are a multiple of 16.
@@ -60,6 +62,7 @@ __global__ void __launch_bounds__(256) permute_rows_elem(PermuteArgs args, int64
 cudaError_t launch_permute(const void* const* src, void* const* dst, int n_tensors, int64_t B,
                            const Layout& L, int64_t H, int64_t D, int esize, bool inverse,
                            cudaStream_t stream) {
+    if (n_tensors < 1 || n_tensors > kMaxTensors) return cudaErrorInvalidValue;
     PermuteArgs args{};
     for (int t = 0; t < n_tensors; ++t) {
         args.src[t] = src[t];

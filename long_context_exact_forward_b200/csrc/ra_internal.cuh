@@ -65,10 +65,11 @@ int host_cuda_fail(cudaError_t e, const char* what);
 void host_set_error(const char* msg);
 cudaError_t launch_attn_tc(const AttnArgs& a, const TcLaunch& t, cudaStream_t stream);
 
-// attn_bwd_tc.cu: the gradient kernels of ra_backward on the tensor cores (bf16, D in {64, 128},
-// contiguous or striped layout); Delta must already be in `delta`.  Returns an RA_* status.
+// attn_bwd_tc.cu: the gradient kernels of ra_backward on the tensor cores (bf16, D in {64, 128});
+// Delta must already be in `delta`; zigzag needs `shard_major` scratch of 4 tensors (see the
+// definition).  Returns an RA_* status.
 int launch_backward_tc(const void* q, const void* k, const void* v, const void* dout, void* dq, void* dk,
                        void* dv, const float* lse, const float* delta, int64_t B, int64_t H, const Layout& L,
-                       int64_t D, int causal, int* status, cudaStream_t stream);
+                       int64_t D, int causal, int* status, void* shard_major, cudaStream_t stream);
 
 }  // namespace ra

@@ -65,7 +65,7 @@ def test_bf16_backward_d128_simt(layout):
     grads_vs_oracle(1, 2, 1024, 128, 4, True, layout, torch.bfloat16, seed=5, bwd_kernel="simt")
 
 
-@pytest.mark.parametrize("layout", ["contiguous", "striped"])
+@pytest.mark.parametrize("layout", ["contiguous", "striped", "zigzag"])
 @pytest.mark.parametrize("causal", [False, True])
 @pytest.mark.parametrize("D", [64, 128])
 def test_bf16_backward_tensor_cores(layout, causal, D):
@@ -78,13 +78,17 @@ def test_bf16_backward_tensor_cores_ragged():
     grads_vs_oracle(1, 2, 600, 64, 3, True, "contiguous", torch.bfloat16, seed=22, bwd_kernel="tc")
 
 
-def test_backward_auto_picks_a_path_for_every_layout():
-    # zigzag falls to CUDA cores under "auto"; asking for tensor cores there is refused
+def test_backward_auto_and_refusals():
+    # "auto" takes the tensor cores for bf16 zigzag too (through shard-major copies); they refuse
+    # fp32 and head dims other than 64 and 128
     grads_vs_oracle(1, 1, 512, 128, 4, True, "zigzag", torch.bfloat16, seed=23)
-    q = torch.zeros(1, 512, 1, 128, device="cuda", dtype=torch.bfloat16)
+    q = torch.zeros(1, 512, 1, 128, device="cuda", dtype=torch.float32)
     lse = torch.zeros(1, 1, 512, device="cuda")
     with pytest.raises(ra.RAError):
-        ra.backward(q, q, q, q, lse, q, 4, True, "zigzag", kernel="tc")
+        ra.backward(q, q, q, q, lse, q, 4, True, "striped", kernel="tc")
+    q = torch.zeros(1, 512, 1, 96, device="cuda", dtype=torch.bfloat16)
+    with pytest.raises(ra.RAError):
+        ra.backward(q, q, q, q, lse, q, 4, True, "striped", kernel="tc")
 
 
 def test_ragged_tiles_and_odd_head_dim():
