@@ -205,8 +205,10 @@ RA_API int ra_backward(const void* q, const void* k, const void* v, const void* 
                        const void* dout, void* dq, void* dk, void* dv, int64_t B, int64_t H, int64_t S,
                        int64_t D, int n_ring, int causal, int layout, int dtype, void* stream);
 
-/* ra_backward_ex: ra_backward with the kernel choice (no counterpart on the pages; for callers and
- * tests that pick the path):
+/* ra_backward_ex: ra_backward with the kernel choice, the bound of every in-kernel wait of the
+ * tensor-core kernels (timeout_ns; 0 = 2 s) and a debug knob (RA_DEBUG_STALL_LOADS: their load warp
+ * issues no streamed tile, so the waits run out and report RA_ERR_DEVICE_TIMEOUT -- for tests).
+ * No counterpart on the pages.  Kernel choice:
  *   RA_KERNEL_AUTO  tensor cores when they apply, else CUDA cores (what ra_backward does);
  *   RA_KERNEL_TC    tcgen05 kernels: bf16, D in {64, 128}, all eight tensors 16-byte aligned, sm_100
  *                   (RA_ERR_UNSUPPORTED otherwise); zigzag inputs are first copied to shard-major
@@ -218,7 +220,8 @@ RA_API int ra_backward(const void* q, const void* k, const void* v, const void* 
  *   RA_KERNEL_SIMT  fp32 arithmetic on CUDA cores for every dtype, D <= 128. */
 RA_API int ra_backward_ex(const void* q, const void* k, const void* v, const void* out, const float* lse,
                           const void* dout, void* dq, void* dk, void* dv, int64_t B, int64_t H, int64_t S,
-                          int64_t D, int n_ring, int causal, int layout, int dtype, int kernel, void* stream);
+                          int64_t D, int n_ring, int causal, int layout, int dtype, int kernel,
+                          uint64_t timeout_ns, int debug, void* stream);
 
 /* ra_status_string: static description of a status code. */
 RA_API const char* ra_status_string(int status);

@@ -82,7 +82,7 @@ def lib():
         L.ra_backward.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i64, i64, i64, i64, ci, ci, ci,
                                   ci, vp]
         L.ra_backward_ex.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i64, i64, i64, i64, ci, ci, ci,
-                                     ci, ci, vp]
+                                     ci, ci, ctypes.c_uint64, ci, vp]
         L.ra_layout_positions.argtypes = [i64, ci, ci, vp]
         L.ra_plan_tiles.argtypes = [i64, ci, ci, ci, ci, vp]
         L.ra_plan_items.argtypes = [i64, i64, i64, i64, ci, ci, ci, vp, i64, ctypes.POINTER(ctypes.c_int64)]
@@ -210,7 +210,7 @@ def forward_noalloc(q, k, v, n_ring, causal=True, layout="contiguous", *, out=No
 
 
 def backward(q, k, v, out, lse, dout, n_ring, causal=True, layout="contiguous", *, kernel="auto", dq=None,
-             dk=None, dv=None, stream=None):
+             dk=None, dv=None, stream=None, timeout_ns=0, debug=0):
     """ra_backward_ex: gradients (dq, dk, dv) of forward(q, k, v, n_ring, causal, layout) for the
     upstream gradient dout, recomputed block by block in ring order from the saved out and lse.
     kernel: "auto" (tensor cores for bf16 with D in {64, 128} and the contiguous or striped layout,
@@ -232,7 +232,7 @@ def backward(q, k, v, out, lse, dout, n_ring, causal=True, layout="contiguous", 
         rc = lib().ra_backward_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
                                   dout.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, H, S, D,
                                   int(n_ring), int(bool(causal)), LAYOUTS[layout], _dtype_code(q),
-                                  KERNELS[kernel], _stream_handle(stream))
+                                  KERNELS[kernel], int(timeout_ns), int(debug), _stream_handle(stream))
     _check(rc, "ra_backward_ex")
     return dq, dk, dv
 

@@ -400,7 +400,7 @@ cudaError_t launch_grads_simt(const void* q, const void* k, const void* v, const
 extern "C" int ra_backward_ex(const void* q, const void* k, const void* v, const void* out, const float* lse,
                               const void* dout, void* dq, void* dk, void* dv, int64_t B, int64_t H, int64_t S,
                               int64_t D, int n_ring, int causal, int layout, int dtype, int kernel,
-                              void* stream_handle) {
+                              uint64_t timeout_ns, int debug, void* stream_handle) {
     int rc = ra::host_check_shape(B, H, S, D, n_ring, layout, dtype);
     if (rc != RA_OK) return rc;
     if (!q || !k || !v || !out || !lse || !dout || !dq || !dk || !dv) return RA_ERR_INVALID_ARG;
@@ -450,7 +450,7 @@ extern "C" int ra_backward_ex(const void* q, const void* k, const void* v, const
     if (e == cudaSuccess) {
         if (use_tc) {
             rc = ra::launch_backward_tc(q, k, v, dout, dq, dk, dv, lse, delta, B, H, A.L, D, causal, status,
-                                        copies ? scratch + delta_bytes : nullptr, stream);
+                                        copies ? scratch + delta_bytes : nullptr, timeout_ns, debug, stream);
         } else {
             e = dtype == RA_DTYPE_FP32
                     ? ra::launch_grads_simt<float>(q, k, v, dout, dq, dk, dv, A, stream)
@@ -468,5 +468,5 @@ extern "C" int ra_backward(const void* q, const void* k, const void* v, const vo
                            const void* dout, void* dq, void* dk, void* dv, int64_t B, int64_t H, int64_t S,
                            int64_t D, int n_ring, int causal, int layout, int dtype, void* stream_handle) {
     return ra_backward_ex(q, k, v, out, lse, dout, dq, dk, dv, B, H, S, D, n_ring, causal, layout, dtype,
-                          RA_KERNEL_AUTO, stream_handle);
+                          RA_KERNEL_AUTO, 0, RA_DEBUG_NONE, stream_handle);
 }

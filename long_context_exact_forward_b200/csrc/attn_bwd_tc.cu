@@ -69,6 +69,7 @@ struct BwdTcArgs {
     __nv_bfloat16* dk;
     __nv_bfloat16* dv;
     uint64_t timeout_ns;
+    int debug;           // RA_DEBUG_STALL_LOADS: the producer issues no streamed tile (tests)
     int* status;
 };
 
@@ -213,6 +214,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int nt = key_tiles(L, A.causal, i, a0, j);
             for (int kt = 0; kt < nt && ok; ++kt, ++it) {
                 const uint32_t st = it & 1;
+                if (A.debug == RA_DEBUG_STALL_LOADS) break;  // consumers must time out
                 ok = __all_sync(0xffffffffu, mbar_wait(&sm.stage_empty[st], ((it >> 1) & 1) ^ 1, timeout, abort));
                 if (!ok) break;
                 if (lane == 0) {
@@ -404,6 +406,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int q0 = 0; q0 < L.S_loc && ok; q0 += kTile) {
                 if (!query_tile_live(L, A.causal, i, q0, j, c0)) continue;
                 const uint32_t st = it & 1;
+                if (A.debug == RA_DEBUG_STALL_LOADS) break;  // consumers must time out
                 ok = __all_sync(0xffffffffu, mbar_wait(&sm.stage_empty[st], ((it >> 1) & 1) ^ 1, timeout, abort));
                 if (!ok) break;
                 if (lane == 0) {
@@ -596,7 +599,8 @@ static_assert(sizeof(BwdSmem<128>) + 1024 <= 232448, "shared memory of one CTA (
 // written in natural order either way.
 int launch_backward_tc(const void* q, const void* k, const void* v, const void* dout, void* dq, void* dk,
                        void* dv, const float* lse, const float* delta, int64_t B, int64_t H, const Layout& L,
-                       int64_t D, int causal, int* status, void* shard_major, cudaStream_t stream) {
+                       int64_t D, int causal, int* status, void* shard_major, uint64_t timeout_ns, int debug,
+                       cudaStream_t stream) {
     CUtensorMap maps[4];
     const void* srcs[4] = {q, k, v, dout};
     const bool striped = L.kind == RA_LAYOUT_STRIPED;
@@ -625,7 +629,8 @@ int launch_backward_tc(const void* q, const void* k, const void* v, const void* 
     A.dq = static_cast<__nv_bfloat16*>(dq);
     A.dk = static_cast<__nv_bfloat16*>(dk);
     A.dv = static_cast<__nv_bfloat16*>(dv);
-    A.timeout_ns = 2000000000ull;
+    A.timeout_ns = timeout_ns ? timeout_ns : 2000000000ull;
+    A.debug = debug;
     A.status = status;
     const dim3 grid((unsigned)((L.S_loc + kTile - 1) / kTile), (unsigned)L.N, (unsigned)(B * H));
     cudaError_t e;

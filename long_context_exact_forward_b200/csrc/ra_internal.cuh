@@ -67,9 +67,10 @@ cudaError_t launch_attn_tc(const AttnArgs& a, const TcLaunch& t, cudaStream_t st
 
 // attn_bwd_tc.cu: the gradient kernels of ra_backward on the tensor cores (bf16, D in {64, 128});
 // Delta must already be in `delta`; zigzag needs `shard_major` scratch of 4 tensors (see the
-// definition).  Returns an RA_* status.
+// definition).  timeout_ns = 0 means 2 s.  Returns an RA_* status.
 int launch_backward_tc(const void* q, const void* k, const void* v, const void* dout, void* dq, void* dk,
                        void* dv, const float* lse, const float* delta, int64_t B, int64_t H, const Layout& L,
-                       int64_t D, int causal, int* status, void* shard_major, cudaStream_t stream);
+                       int64_t D, int causal, int* status, void* shard_major, uint64_t timeout_ns, int debug,
+                       cudaStream_t stream);
 
 }  // namespace ra

@@ -56,3 +56,27 @@ def test_host_validation_errors_enqueue_nothing():
     assert e.value.code == -4
     torch.cuda.synchronize()
     assert ra.get_device_status() == 0
+
+
+def test_backward_stalled_loads_time_out_and_report():
+    # the tensor-core backward kernels bound their waits the same way
+    q, k, v = inputs.make_qkv(1, 4 * 256, 2, 128, torch.bfloat16, "cuda", seed=4)
+    out, lse = ra.forward(q, k, v, 4, True, "striped")
+    dout = torch.randn_like(q)
+    torch.cuda.synchronize()
+    assert ra.get_device_status() == 0
+    t0 = time.time()
+    ra.backward(q, k, v, out, lse, dout, 4, True, "striped", kernel="tc",
+                debug=ra.DEBUG_STALL_LOADS, timeout_ns=100_000_000)
+    torch.cuda.synchronize()
+    assert time.time() - t0 < 30
+    assert ra.get_device_status() == RA_ERR_DEVICE_TIMEOUT
+    assert ra.get_device_status() == 0
+    # the context still works: the same backward without the knob is correct
+    dq, dk, dv = ra.backward(q, k, v, out, lse, dout, 4, True, "striped", kernel="tc")
+    torch.cuda.synchronize()
+    assert ra.get_device_status() == 0
+    ref = oracle.attention_backward(q.cpu(), k.cpu(), v.cpu(), dout.cpu(), True, threads=8)
+    for x, r in zip((dq, dk, dv), ref):
+        scale = max(1.0, float(np.abs(r).max()))
+        assert np.abs(x.float().cpu().double().numpy() - r).max() <= 2e-2 * scale
