@@ -18,6 +18,9 @@ merge(m, l, O, m2, l2, O2)
     Online-softmax merge identities (troisinh.com "Ring Attention", "Tai sao no hoat dong").
 layout_positions(S, n_ring, layout)
     Global position of each (shard, local index) under a layout, shape [N, S/N].
+rope(x, pos_offset=0, base=10000.0)
+    Rotary embedding with global positions (troisinh.com "Ring Attention", "RoPE va Position
+    Embedding"), pairs (2p, 2p+1) rotated by m * base^(-2p/D), in fp64.  Returns [B, S, H, D].
 attention_backward(q, k, v, dout, causal, threads=1)
     Gradients (dq, dk, dv) of the plain definition for the upstream gradient dout, in fp64, each
     [B, S, H, D] (troisinh.com "Ring Attention", "Blockwise Backward"; chain rule written out).
@@ -61,6 +64,8 @@ def load(path=None):
     lib.ora_merge.argtypes = [i64, i64, dp, dp, dp, dp, dp, dp]
     lib.ora_layout_positions.restype = ctypes.c_int
     lib.ora_layout_positions.argtypes = [i64, i64, ctypes.c_int, vp]
+    lib.ora_rope.restype = ctypes.c_int
+    lib.ora_rope.argtypes = [vp, ctypes.c_int, i64, i64, i64, i64, i64, ctypes.c_double, vp]
     lib.ora_attention_backward.restype = ctypes.c_int
     lib.ora_attention_backward.argtypes = [vp, vp, vp, vp, ctypes.c_int, i64, i64, i64, i64,
                                            ctypes.c_int, vp, vp, vp, ctypes.c_int]
@@ -178,3 +183,14 @@ def attention_backward(q, k, v, dout, causal, threads=1, lib=None):
     if rc != 0:
         raise ValueError("ora_attention_backward rejected its arguments")
     return dq, dk, dv
+
+
+def rope(x, pos_offset=0, base=10000.0, lib=None):
+    """fp64 rotary embedding of x [B, S, H, D]; token g takes the position g + pos_offset."""
+    lib = lib or _get()
+    x = _as_input(x)
+    B, S, H, D = x.shape
+    y = np.empty((B, S, H, D), dtype=np.float64)
+    if lib.ora_rope(x.ctypes.data, _code(x), B, S, H, D, int(pos_offset), float(base), y.ctypes.data) != 0:
+        raise ValueError("ora_rope rejected its arguments")
+    return y

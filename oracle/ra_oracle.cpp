@@ -29,6 +29,12 @@
 //                            with no blocking: P = softmax(S), dV = P^T dO, dP = dO V^T,
 //                            dS = P * (dP - rowsum(P * dP)), dQ = dS K / sqrt(D),
 //                            dK = dS^T Q / sqrt(D).
+//   * ora_rope           -- rotary position embedding applied with each token's GLOBAL position m
+//                            (troisinh.com "Ring Attention", "RoPE va Position Embedding": when K/V
+//                            travel round the ring, each position m must still be rotated by the
+//                            angle m theta).  Reading: the pairs (x[2p], x[2p+1]) of the head dim are
+//                            rotated by m theta_p with theta_p = base^(-2p/D), the original
+//                            rotary embedding, base 10000 by default.
 //
 // Readings where the pages are silent (listed again in the design notes):
 //   * scale = 1/sqrt(D) (the toy divides the scores by dim**0.5);
@@ -325,6 +331,27 @@ int ora_attention_backward(const void* q, const void* k, const void* v, const vo
     for (int w = 1; w < n_threads; ++w) pool.emplace_back(worker);
     worker();
     for (auto& th : pool) th.join();
+    return 0;
+}
+
+// Rotary embedding of x [B, S, H, D] (dtype as above) into y (fp64), the token at natural index g
+// taking the position m = g + pos_offset; D must be even.  Returns 0, or -1 on a bad argument.
+int ora_rope(const void* x, int dtype, int64_t B, int64_t S, int64_t H, int64_t D, int64_t pos_offset,
+             double base, double* y) {
+    if (!x || !y || B < 0 || S < 0 || H < 0 || D <= 0 || (D & 1) || !(base > 0.0)) return -1;
+    if (dtype < 0 || dtype > 2) return -1;
+    for (int64_t b = 0; b < B; ++b)
+        for (int64_t g = 0; g < S; ++g)
+            for (int64_t h = 0; h < H; ++h)
+                for (int64_t p = 0; p < D / 2; ++p) {
+                    const double m = (double)(g + pos_offset);
+                    const double theta = std::pow(base, -2.0 * (double)p / (double)D);
+                    const double c = std::cos(m * theta), sn = std::sin(m * theta);
+                    const double x0 = to_f64(x, dtype, at(b, g, h, 2 * p, S, H, D));
+                    const double x1 = to_f64(x, dtype, at(b, g, h, 2 * p + 1, S, H, D));
+                    y[at(b, g, h, 2 * p, S, H, D)] = x0 * c - x1 * sn;
+                    y[at(b, g, h, 2 * p + 1, S, H, D)] = x0 * sn + x1 * c;
+                }
     return 0;
 }
 
