@@ -224,6 +224,7 @@ def hbm_kernels(ra, q, n_ring, layout, stream, reps=10):
     permute: q [B, S, H, D] bf16 -> shard-major copy; algorithmic bytes = read + write of q.
     merge:   one ring step's partial folded into the running result (fp32 [B*S*H, D] and
              lse [B*S*H]); algorithmic bytes = 12 per output element + 12 per row.
+    rope:    rotary embedding of q with global positions, out of place; bytes = read + write of q.
     """
     peaks, src = load_peaks()
     res = {"peak_gbs": peaks["hbm_gbs"], "peak_kind": f"copy ({src})"}
@@ -257,6 +258,11 @@ def hbm_kernels(ra, q, n_ring, layout, stream, reps=10):
     byts = 12.0 * rows * D + 12.0 * rows
     res["merge"] = {"rows": rows, "D": D, "ms": ms, "bytes": byts, "achieved_gbs": byts / ms / 1e6,
                     "frac": byts / ms / 1e6 / peaks["hbm_gbs"]}
+    del O_r, O_s, l_r, l_s
+    yr = torch.empty_like(q)
+    ms = timed(lambda: ra.rope(q, out=yr, stream=stream))
+    byts = 2.0 * q.numel() * q.element_size()
+    res["rope"] = {"ms": ms, "bytes": byts, "achieved_gbs": byts / ms / 1e6, "frac": byts / ms / 1e6 / peaks["hbm_gbs"]}
     return res
 
 

@@ -223,6 +223,18 @@ RA_API int ra_backward_ex(const void* q, const void* k, const void* v, const voi
                           int64_t D, int n_ring, int causal, int layout, int dtype, int kernel,
                           uint64_t timeout_ns, int debug, void* stream);
 
+/* ra_rope: rotary position embedding with global token positions (troisinh.com "Ring Attention",
+ * "RoPE va Position Embedding": a token must be rotated by the angle m theta of its own position m
+ * wherever its block travels on the ring).  x, y: [B, S, H, D] in natural token order, dtype fp32 or
+ * bf16; the token at natural index g takes the position m = g + pos_offset (so a later chunk of a
+ * sequence passes the length before it).  The pair (x[2p], x[2p+1]) is rotated by m * theta_p,
+ * theta_p = base^(-2p/D) (10000 is the usual base).  y may equal x (in place).  D even, <= 256;
+ * pos_offset >= 0; base > 0; pointers aligned to their element size.  The angle is reduced in fp64,
+ * the rotation is fp32, the result rounds to the dtype.  Asynchronous on `stream`; returns RA_OK
+ * or a validation error before anything is enqueued. */
+RA_API int ra_rope(const void* x, void* y, int64_t B, int64_t S, int64_t H, int64_t D, int64_t pos_offset,
+                   double base, int dtype, void* stream);
+
 /* ra_status_string: static description of a status code. */
 RA_API const char* ra_status_string(int status);
 

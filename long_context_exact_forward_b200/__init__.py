@@ -81,6 +81,7 @@ def lib():
         L.ra_forward_noalloc.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i64, ci, ci, ci, vp]
         L.ra_backward.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i64, i64, i64, i64, ci, ci, ci,
                                   ci, vp]
+        L.ra_rope.argtypes = [vp, vp, i64, i64, i64, i64, i64, ctypes.c_double, ci, vp]
         L.ra_backward_ex.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i64, i64, i64, i64, ci, ci, ci,
                                      ci, ci, ctypes.c_uint64, ci, vp]
         L.ra_layout_positions.argtypes = [i64, ci, ci, vp]
@@ -93,7 +94,7 @@ def lib():
         L.ra_get_device_status.argtypes = []
         for name in ("ra_forward", "ra_forward_ex", "ra_forward_noalloc", "ra_workspace_size", "ra_permute",
                      "ra_unpermute", "ra_merge_partials", "ra_layout_positions", "ra_plan_tiles",
-                     "ra_plan_items", "ra_get_device_status", "ra_backward", "ra_backward_ex"):
+                     "ra_plan_items", "ra_get_device_status", "ra_backward", "ra_backward_ex", "ra_rope"):
             getattr(L, name).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -235,6 +236,23 @@ def backward(q, k, v, out, lse, dout, n_ring, causal=True, layout="contiguous", 
                                   KERNELS[kernel], int(timeout_ns), int(debug), _stream_handle(stream))
     _check(rc, "ra_backward_ex")
     return dq, dk, dv
+
+
+def rope(x, pos_offset=0, base=10000.0, out=None, stream=None):
+    """ra_rope: rotary embedding of x [B, S, H, D] with global positions (token g at g + pos_offset);
+    out may be x itself (in place)."""
+    torch = _torch()
+    _check_cuda(x)
+    if x.dim() != 4:
+        raise ValueError("x must be [B, S, H, D]")
+    out = torch.empty_like(x) if out is None else out
+    _check_cuda(out)
+    B, S, H, D = x.shape
+    with torch.cuda.device(x.device):
+        rc = lib().ra_rope(x.data_ptr(), out.data_ptr(), B, S, H, D, int(pos_offset), float(base),
+                           _dtype_code(x), _stream_handle(stream))
+    _check(rc, "ra_rope")
+    return out
 
 
 def permute(x, n_ring, layout, out=None, stream=None, inverse=False):
