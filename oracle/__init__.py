@@ -18,6 +18,9 @@ merge(m, l, O, m2, l2, O2)
     Online-softmax merge identities (troisinh.com "Ring Attention", "Tai sao no hoat dong").
 layout_positions(S, n_ring, layout)
     Global position of each (shard, local index) under a layout, shape [N, S/N].
+attention_varlen(q, k, v, cu_seqlens, causal, threads=1)
+    The plain definition for sequences packed along the token axis of q, k, v [1, S_total, H, D]
+    (sequence k = tokens cu[k]..cu[k+1]-1).  Returns out [S_total, H, D] and lse [H, S_total].
 rope(x, pos_offset=0, base=10000.0)
     Rotary embedding with global positions (troisinh.com "Ring Attention", "RoPE va Position
     Embedding"), pairs (2p, 2p+1) rotated by m * base^(-2p/D), in fp64.  Returns [B, S, H, D].
@@ -64,6 +67,9 @@ def load(path=None):
     lib.ora_merge.argtypes = [i64, i64, dp, dp, dp, dp, dp, dp]
     lib.ora_layout_positions.restype = ctypes.c_int
     lib.ora_layout_positions.argtypes = [i64, i64, ctypes.c_int, vp]
+    lib.ora_attention_varlen.restype = ctypes.c_int
+    lib.ora_attention_varlen.argtypes = [vp, vp, vp, ctypes.c_int, i64, i64, i64, ctypes.c_int, vp, i64, vp, vp,
+                                         ctypes.c_int]
     lib.ora_rope.restype = ctypes.c_int
     lib.ora_rope.argtypes = [vp, ctypes.c_int, i64, i64, i64, i64, i64, ctypes.c_double, vp]
     lib.ora_attention_backward.restype = ctypes.c_int
@@ -194,3 +200,22 @@ def rope(x, pos_offset=0, base=10000.0, lib=None):
     if lib.ora_rope(x.ctypes.data, _code(x), B, S, H, D, int(pos_offset), float(base), y.ctypes.data) != 0:
         raise ValueError("ora_rope rejected its arguments")
     return y
+
+
+def attention_varlen(q, k, v, cu_seqlens, causal, threads=1, lib=None):
+    """fp64 attention of packed sequences: q, k, v [1, S_total, H, D]; returns (out [S_total, H, D],
+    lse [H, S_total])."""
+    lib = lib or _get()
+    q, k, v = _as_input(q), _as_input(k), _as_input(v)
+    if q.shape[0] != 1:
+        raise ValueError("packed sequences take batch 1")
+    _, S, H, D = q.shape
+    cu = np.ascontiguousarray(np.asarray(cu_seqlens, dtype=np.int64))
+    out = np.empty((S, H, D), dtype=np.float64)
+    lse = np.empty((H, S), dtype=np.float64)
+    rc = lib.ora_attention_varlen(q.ctypes.data, k.ctypes.data, v.ctypes.data, _code(q), S, H, D,
+                                  int(bool(causal)), cu.ctypes.data, cu.size - 1, out.ctypes.data,
+                                  lse.ctypes.data, int(threads))
+    if rc != 0:
+        raise ValueError("ora_attention_varlen rejected its arguments")
+    return out, lse

@@ -29,6 +29,12 @@
 //                            with no blocking: P = softmax(S), dV = P^T dO, dP = dO V^T,
 //                            dS = P * (dP - rowsum(P * dP)), dQ = dS K / sqrt(D),
 //                            dK = dS^T Q / sqrt(D).
+//   * ora_attention_varlen -- the plain definition for several sequences packed one after another
+//                            along the token axis: a query attends only to keys of its own sequence
+//                            (and, causal, at or before its own position).  troisinh.com "Ring
+//                            Attention", "Trade-off thuc te" (Complexity) names load balancing
+//                            with sequences of different lengths as a challenge; the result is
+//                            still exact attention per sequence, which is what this writes out.
 //   * ora_rope           -- rotary position embedding applied with each token's GLOBAL position m
 //                            (troisinh.com "Ring Attention", "RoPE va Position Embedding": when K/V
 //                            travel round the ring, each position m must still be rotated by the
@@ -352,6 +358,57 @@ int ora_rope(const void* x, int dtype, int64_t B, int64_t S, int64_t H, int64_t 
                     y[at(b, g, h, 2 * p, S, H, D)] = x0 * c - x1 * sn;
                     y[at(b, g, h, 2 * p + 1, S, H, D)] = x0 * sn + x1 * c;
                 }
+    return 0;
+}
+
+// Packed sequences: q, k, v [S_total, H, D] (one batch), sequence k holding tokens
+// [cu[k], cu[k+1]).  out [S_total, H, D] fp64 (natural order), lse [H, S_total] fp64.  A query
+// attends to the keys of its own sequence only (and, causal, to those at or before it).
+// Returns 0, or -1 on a bad argument.
+int ora_attention_varlen(const void* q, const void* k, const void* v, int dtype, int64_t S_total, int64_t H,
+                         int64_t D, int causal, const int64_t* cu, int64_t n_seqs, double* out, double* lse,
+                         int threads) {
+    if (!q || !k || !v || !cu || !out || !lse || S_total < 0 || H <= 0 || D <= 0 || n_seqs < 1) return -1;
+    if (dtype < 0 || dtype > 2 || cu[0] != 0 || cu[n_seqs] != S_total) return -1;
+    for (int64_t s = 0; s < n_seqs; ++s)
+        if (cu[s + 1] < cu[s]) return -1;
+    const double scale = 1.0 / std::sqrt((double)D);
+    const int64_t total = S_total * H;
+    std::atomic<int64_t> next{0};
+    auto worker = [&]() {
+        std::vector<double> qrow(D), sc(std::max<int64_t>(S_total, 1));
+        for (;;) {
+            const int64_t t = next.fetch_add(1);
+            if (t >= total) break;
+            const int64_t r = t / H, h = t % H;
+            int64_t seq = 0;
+            while (cu[seq + 1] <= r) ++seq;
+            const int64_t lo = cu[seq], hi = causal ? r + 1 : cu[seq + 1];
+            for (int64_t d = 0; d < D; ++d) qrow[d] = to_f64(q, dtype, at(0, r, h, d, S_total, H, D));
+            double m = -std::numeric_limits<double>::infinity();
+            for (int64_t c = lo; c < hi; ++c) {
+                double dot = 0.0;
+                for (int64_t d = 0; d < D; ++d) dot += qrow[d] * to_f64(k, dtype, at(0, c, h, d, S_total, H, D));
+                sc[c] = scale * dot;
+                m = std::max(m, sc[c]);
+            }
+            double l = 0.0;
+            double* o = out + (r * H + h) * D;
+            for (int64_t d = 0; d < D; ++d) o[d] = 0.0;
+            for (int64_t c = lo; c < hi; ++c) {
+                const double p = std::exp(sc[c] - m);
+                l += p;
+                for (int64_t d = 0; d < D; ++d) o[d] += p * to_f64(v, dtype, at(0, c, h, d, S_total, H, D));
+            }
+            for (int64_t d = 0; d < D; ++d) o[d] /= l;
+            lse[h * S_total + r] = m + std::log(l);
+        }
+    };
+    const int n_threads = std::max(1, std::min<int>(threads, (int)std::max<int64_t>(total, 1)));
+    std::vector<std::thread> pool;
+    for (int w = 1; w < n_threads; ++w) pool.emplace_back(worker);
+    worker();
+    for (auto& th : pool) th.join();
     return 0;
 }
 
