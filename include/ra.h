@@ -223,6 +223,22 @@ RA_API int ra_backward_ex(const void* q, const void* k, const void* v, const voi
                           int64_t D, int n_ring, int causal, int layout, int dtype, int kernel,
                           uint64_t timeout_ns, int debug, void* stream);
 
+/* ra_forward_varlen: exact attention over several sequences packed one after another on the token
+ * axis -- each query attends only to the keys of its own sequence (and, when `causal`, to those at or
+ * before its position inside that sequence).  troisinh.com "Ring Attention", "Trade-off thuc te",
+ * names load balancing with sequences of different lengths as the challenge; every sequence is split
+ * into n_ring shards with `layout` and all their work items join one longest-first list for the
+ * fused tensor-core kernel.
+ *   q, k, v, out: [S_total, H, D] bf16 (batch 1), natural order; lse: [H, S_total] fp32, natural log.
+ *   cu_seqlens: HOST array of n_seqs + 1 int64 offsets, cu[0] = 0, non-decreasing, cu[n_seqs] =
+ *     S_total; every length a multiple of n_ring (RA_ERR_SHAPE otherwise); empty sequences allowed.
+ *   layout: contiguous or striped (zigzag: RA_ERR_UNSUPPORTED); D in {64, 128}; sm_100; q, k, v, out
+ *   16-byte aligned.  Scratch (work list, sequence table, counter) is allocated stream-ordered.
+ *   Asynchronous on `stream`; bounded waits report through ra_get_device_status. */
+RA_API int ra_forward_varlen(const void* q, const void* k, const void* v, void* out, float* lse,
+                             const int64_t* cu_seqlens, int n_seqs, int64_t H, int64_t D, int n_ring,
+                             int causal, int layout, void* stream);
+
 /* ra_rope: rotary position embedding with global token positions (troisinh.com "Ring Attention",
  * "RoPE va Position Embedding": a token must be rotated by the angle m theta of its own position m
  * wherever its block travels on the ring).  x, y: [B, S, H, D] in natural token order, dtype fp32 or

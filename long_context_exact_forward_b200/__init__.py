@@ -81,6 +81,7 @@ def lib():
         L.ra_forward_noalloc.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i64, ci, ci, ci, vp]
         L.ra_backward.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i64, i64, i64, i64, ci, ci, ci,
                                   ci, vp]
+        L.ra_forward_varlen.argtypes = [vp, vp, vp, vp, vp, vp, ci, i64, i64, ci, ci, ci, vp]
         L.ra_rope.argtypes = [vp, vp, i64, i64, i64, i64, i64, ctypes.c_double, ci, vp]
         L.ra_backward_ex.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i64, i64, i64, i64, ci, ci, ci,
                                      ci, ci, ctypes.c_uint64, ci, vp]
@@ -94,7 +95,7 @@ def lib():
         L.ra_get_device_status.argtypes = []
         for name in ("ra_forward", "ra_forward_ex", "ra_forward_noalloc", "ra_workspace_size", "ra_permute",
                      "ra_unpermute", "ra_merge_partials", "ra_layout_positions", "ra_plan_tiles",
-                     "ra_plan_items", "ra_get_device_status", "ra_backward", "ra_backward_ex", "ra_rope"):
+                     "ra_plan_items", "ra_get_device_status", "ra_backward", "ra_backward_ex", "ra_rope", "ra_forward_varlen"):
             getattr(L, name).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -236,6 +237,29 @@ def backward(q, k, v, out, lse, dout, n_ring, causal=True, layout="contiguous", 
                                   KERNELS[kernel], int(timeout_ns), int(debug), _stream_handle(stream))
     _check(rc, "ra_backward_ex")
     return dq, dk, dv
+
+
+def forward_varlen(q, k, v, cu_seqlens, n_ring, causal=True, layout="contiguous", *, out=None, lse=None,
+                   stream=None):
+    """ra_forward_varlen: attention over sequences packed on the token axis of q, k, v [S_total, H, D]
+    (bf16); cu_seqlens: n_seqs + 1 offsets (a host sequence of ints).  Returns (out [S_total, H, D],
+    lse [H, S_total])."""
+    torch = _torch()
+    import numpy as np
+    _check_cuda(q, k, v)
+    if q.dim() != 3 or q.shape != k.shape or q.shape != v.shape:
+        raise ValueError("q, k, v must all be [S_total, H, D]")
+    S, H, D = q.shape
+    cu = np.ascontiguousarray(np.asarray(cu_seqlens, dtype=np.int64))
+    out = torch.empty_like(q) if out is None else out
+    lse = torch.empty((H, S), dtype=torch.float32, device=q.device) if lse is None else lse
+    _check_cuda(out, lse)
+    with torch.cuda.device(q.device):
+        rc = lib().ra_forward_varlen(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
+                                     cu.ctypes.data, int(cu.size - 1), H, D, int(n_ring), int(bool(causal)),
+                                     LAYOUTS[layout], _stream_handle(stream))
+    _check(rc, "ra_forward_varlen")
+    return out, lse
 
 
 def rope(x, pos_offset=0, base=10000.0, out=None, stream=None):

@@ -51,6 +51,16 @@ constexpr int kM = 128;           // query rows per tile
 constexpr int kN = 128;           // keys per tile
 constexpr int kSlots = 4;         // K/V tile slots
 constexpr int kThreads = 384;
+#ifndef RA_REGS_SOFTMAX
+#define RA_REGS_SOFTMAX 184
+#endif
+#ifndef RA_REGS_OTHER
+#define RA_REGS_OTHER 112
+#endif
+// register split: 256 softmax threads and 128 load / MMA threads, within the 384 x 168 registers
+// the CTA is launched with
+constexpr int kRegsSoftmax = RA_REGS_SOFTMAX, kRegsOther = RA_REGS_OTHER;
+static_assert(256 * kRegsSoftmax + 128 * kRegsOther <= 384 * 168, "register split exceeds the launch budget");
 constexpr int kLoadWarp = 8;
 constexpr int kMmaWarp = 9;
 constexpr uint32_t kTmemCols = 512;
@@ -116,22 +126,46 @@ template <int kD>
 __device__ __forceinline__ uint32_t o_col(int q) { return 256u + (uint32_t)q * 128u; }
 
 struct ItemGeom {
+    Layout32 L;   // the item's sequence: the whole problem, or one packed sequence
+    int base;     // first token of the sequence on the packed axis (0 in batch mode)
     int b, h, i;
     int a0[2];    // first local row of each query tile
     int last[2];  // last valid local row of each query tile (clamped to the shard)
 };
 
-__device__ __forceinline__ ItemGeom item_geom(const Layout32& L, int4 it) {
+// kVarlen is a template flag so that the batch-mode kernel keeps the problem's layout in the
+// roles' registers instead of a per-item copy.
+template <bool kVarlen>
+__device__ __forceinline__ ItemGeom item_geom(const AttnArgs& A, const Layout32& Lg, int4 it) {
     ItemGeom G;
-    G.b = it.x;
     G.h = it.y;
     G.i = it.z;
+    if (kVarlen) {  // packed sequences: x is the sequence
+        const int2 sd = A.seqs[it.x];
+        G.L = Layout32{sd.x, Lg.N, sd.x / Lg.N, Lg.kind};
+        G.base = sd.y;
+        G.b = 0;
+    } else {
+        G.L = Lg;
+        G.base = 0;
+        G.b = it.x;
+    }
     for (int q = 0; q < 2; ++q) {
         G.a0[q] = it.w * 2 * kM + q * kM;
         const int e = G.a0[q] + kM - 1;
-        G.last[q] = e < L.S_loc - 1 ? e : L.S_loc - 1;
+        G.last[q] = e < G.L.S_loc - 1 ? e : G.L.S_loc - 1;
     }
     return G;
+}
+
+// TMA row coordinates (dims 2 and 3 of the 5-D map) of local row a of shard `shard`: in batch mode
+// (row, shard); packed contiguous, the map's token axis is the packed axis; packed striped, the
+// map is (token / N, token mod N) and sequences start on multiples of N.
+template <bool kVarlen>
+__device__ __forceinline__ int2 tma_rows(const AttnArgs& A, const ItemGeom& G, int shard, int a) {
+    if (!kVarlen) return make_int2(a, shard);
+    if (A.varlen_striped) return make_int2(G.base / G.L.N + a, shard);
+    return make_int2(G.base + shard * G.L.S_loc + a, 0);
 }
 
 // Live key tiles of block j for query tile q (0 if the tile lies past the shard end).
@@ -190,7 +224,7 @@ __device__ __forceinline__ void tmem_wait_ld_regs(uint32_t (&r)[32]) {
                  : "memory");
 }
 
-template <int kD>
+template <int kD, bool kVarlen>
 struct Roles {
     TcSmem<kD>& sm;
     const AttnArgs& A;
@@ -228,21 +262,23 @@ struct Roles {
             }
             idx = __shfl_sync(0xffffffffu, idx, 0);
             if (idx < 0) break;
-            const ItemGeom G = item_geom(L, items[idx]);
+            const ItemGeom G = item_geom<kVarlen>(A, L, items[idx]);
             TileIter t;
-            t.init(A, L, G);
+            t.init(A, G.L, G);
             if (!t.valid) continue;
             if (debug == RA_DEBUG_STALL_LOADS) continue;  // consumers must time out
             if (!wait(&sm.q_empty, (q_it & 1) ^ 1)) break;
             if (leader) {
                 mbar_arrive_expect_tx(&sm.q_full, 2 * TcSmem<kD>::kTileBytes);
-                for (int q = 0; q < 2; ++q)
+                for (int q = 0; q < 2; ++q) {
+                    const int2 rc = tma_rows<kVarlen>(A, G, G.i, G.a0[q]);
                     for (int cb = 0; cb < kD / 64; ++cb)
-                        tma_load_5d(sm.q[q] + cb * kColBlockBytes, tm_q, &sm.q_full, cb * 64, G.h,
-                                    G.a0[q], G.i, G.b);
+                        tma_load_5d(sm.q[q] + cb * kColBlockBytes, tm_q, &sm.q_full, cb * 64, G.h, rc.x,
+                                    rc.y, G.b);
+                }
             }
             ++q_it;
-            for (; t.valid && ok; t.next(L, A.causal, G)) {
+            for (; t.valid && ok; t.next(G.L, A.causal, G)) {
                 uint64_t* full = &sm.kv_full[tile_it & 1];
                 for (int w = 0; w < 2; ++w) {  // K then V of this tile, each as soon as its slot frees
                     const uint32_t use = 2 * tile_it + w;
@@ -251,9 +287,10 @@ struct Roles {
                     if (w == 0) armed = tile_it + 1;
                     if (leader) {
                         if (w == 0) mbar_arrive_expect_tx(full, 2 * TcSmem<kD>::kTileBytes);
+                        const int2 rc = tma_rows<kVarlen>(A, G, t.j, t.kt * kN);
                         for (int cb = 0; cb < kD / 64; ++cb)
                             tma_load_5d(sm.kv[slot] + cb * kColBlockBytes, w ? tm_v : tm_k, full, cb * 64,
-                                        G.h, t.kt * kN, t.j, G.b);
+                                        G.h, rc.x, rc.y, G.b);
                     }
                 }
                 if (ok) ++tile_it;
@@ -315,9 +352,9 @@ struct Roles {
             __syncwarp();
             if (leader) mbar_arrive(&sm.item_empty[b]);
             if (idx < 0) break;
-            const ItemGeom G = item_geom(L, items[idx]);
+            const ItemGeom G = item_geom<kVarlen>(A, L, items[idx]);
             TileIter cur;
-            cur.init(A, L, G);
+            cur.init(A, G.L, G);
             if (!cur.valid) continue;
             if (!wait_tma(&sm.q_full, q_it & 1)) break;
             ++q_it;
@@ -332,7 +369,7 @@ struct Roles {
                 }
             warp_mma_commit(&sm.slot_empty[kslot]);
             TileIter nxt = cur;
-            nxt.next(L, A.causal, G);
+            nxt.next(G.L, A.causal, G);
             if (!nxt.valid) warp_mma_commit(&sm.q_empty);
             for (;;) {
                 const uint32_t vslot = (2 * tile_it + 1) % kSlots;  // landed with K of this tile
@@ -369,7 +406,7 @@ struct Roles {
                 warp_mma_commit(&sm.slot_empty[kslot]);
                 cur = nxt;
                 ++tile_it;
-                nxt.next(L, A.causal, G);
+                nxt.next(G.L, A.causal, G);
                 if (!nxt.valid) warp_mma_commit(&sm.q_empty);
             }
             if (!ok) break;
@@ -407,15 +444,15 @@ struct Roles {
             __syncwarp();
             if ((threadIdx.x & 31) == 0) mbar_arrive(&sm.item_empty[b]);
             if (idx < 0) break;
-            const ItemGeom G = item_geom(L, items[idx]);
+            const ItemGeom G = item_geom<kVarlen>(A, L, items[idx]);
             const int a = G.a0[q] + row;
             float m_run = -INFINITY, l = 0.f;
             int n_act = 0;
             for (int s = A.s_begin; s < A.s_end && ok; ++s) {
-                const int j = ring_block32(G.i, s, L.N);
-                const int nt = tiles_for(L, A.causal, G, q, j);
+                const int j = ring_block32(G.i, s, G.L.N);
+                const int nt = tiles_for(G.L, A.causal, G, q, j);
                 if (nt == 0) continue;
-                const int cnt = visible_keys(L, A.causal, G.i, a, j);
+                const int cnt = visible_keys(G.L, A.causal, G.i, a, j);
                 for (int kt = 0; kt < nt; ++kt) {
                     if (!wait_all(&sm.s_full[q], s_cnt & 1)) break;
                     ++s_cnt;
@@ -532,18 +569,19 @@ struct Roles {
     template <typename Wait>
     __device__ void epilogue(int q, const ItemGeom& G, int a, int n_act, float m_run, float l,
                              uint32_t tO, bool& ok, Wait& wait_all, uint32_t& items_act) {
-        const bool row_ok = a < L.S_loc;
+        const bool row_ok = a < G.L.S_loc;
         const float inv_l = l > 0.f ? 1.f / l : 0.f;
         const float lse = l > 0.f ? (m_run + log2f(l)) * kLn2 : -INFINITY;
         const int64_t H = A.H, S = A.L.S;
         float* lse_dst;
         uint8_t* row_dst;
         if (A.out_mode == kOutFinal) {
-            const int64_t g = row_ok ? global_position(L, G.i, a) : 0;
+            // token on the (packed) axis: the sequence's first token plus the position inside it
+            const int64_t g = G.base + (row_ok ? global_position(G.L, G.i, a) : 0);
             row_dst = static_cast<uint8_t*>(A.out) + (((G.b * S + g) * H + G.h) * kD) * 2;
             lse_dst = A.lse + (G.b * H + G.h) * S + g;
         } else {
-            const int64_t rr = (((int64_t)G.b * L.N + G.i) * L.S_loc + a) * H + G.h;
+            const int64_t rr = (((int64_t)G.b * G.L.N + G.i) * G.L.S_loc + a) * H + G.h;
             row_dst = static_cast<uint8_t*>(A.out) + rr * kD * 4;
             lse_dst = A.lse + rr;
         }
@@ -592,7 +630,7 @@ struct Roles {
     }
 };
 
-template <int kD>
+template <int kD, bool kVarlen>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const AttnArgs A,
@@ -637,10 +675,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     tc_fence_after();
 
-    Roles<kD> roles{sm, A, items, n_items, timeout_ns, status, &sm.abort, sm.tmem_base, narrow(A.L), counter};
-    // register split: 256 softmax threads x 184 + 128 producer/MMA threads x 112 = 61440 <= 384 x 168
+    Roles<kD, kVarlen> roles{sm, A, items, n_items, timeout_ns, status, &sm.abort, sm.tmem_base, narrow(A.L), counter};
     if (warp >= 8) {
-        setmaxnreg_dec112();
+        setmaxnreg_dec<kRegsOther>();
         if (warp == kLoadWarp) {
             roles.producer(&tm_q, &tm_k, &tm_v, debug);
             __syncwarp();
@@ -649,7 +686,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             __syncwarp();
         }
     } else {
-        setmaxnreg_inc184();
+        setmaxnreg_inc<kRegsSoftmax>();
         roles.softmax(warp >> 2, warp, threadIdx.x & 127);
     }
 
@@ -670,7 +707,8 @@ size_t tc_smem_bytes(int64_t D) {
 cudaError_t launch_attn_tc(const AttnArgs& a, const TcLaunch& t, cudaStream_t stream) {
     if (t.n_items == 0) return cudaSuccess;
     const size_t smem = tc_smem_bytes(a.D);
-    auto kern = (a.D == 64) ? attn_tc_kernel<64> : attn_tc_kernel<128>;
+    auto kern = a.seqs ? ((a.D == 64) ? attn_tc_kernel<64, true> : attn_tc_kernel<128, true>)
+                       : ((a.D == 64) ? attn_tc_kernel<64, false> : attn_tc_kernel<128, false>);
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     kern<<<t.grid, kThreads, smem, stream>>>(t.tm_q, t.tm_k, t.tm_v, a, t.items, t.n_items, t.counter,

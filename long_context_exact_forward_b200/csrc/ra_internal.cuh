@@ -24,6 +24,11 @@ struct AttnArgs {
     void* out;            // kOutFinal: [B, S, H, D] dtype; kOutPartial: fp32 [rows, D]
     float* lse;           // kOutFinal: [B, H, S]; kOutPartial: [rows]
     float scale;          // 1 / sqrt(D)
+    // Packed sequences (tensor-core kernel, fused, B = 1): work item x indexes `seqs`, each entry
+    // {S_k, first token of sequence k}; L then describes the whole packed axis (S = S_total) and
+    // every sequence is split into L.N shards with L.kind.  Null: batch mode (item x = batch b).
+    const int2* seqs;
+    int varlen_striped;   // packed sequences with the striped layout inside each sequence
 };
 
 // permute.cu

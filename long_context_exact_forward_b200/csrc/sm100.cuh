@@ -288,8 +288,11 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
     return d;
 }
 
-__device__ __forceinline__ void setmaxnreg_inc184() { asm volatile("setmaxnreg.inc.sync.aligned.u32 184;"); }
-__device__ __forceinline__ void setmaxnreg_dec112() { asm volatile("setmaxnreg.dec.sync.aligned.u32 112;"); }
+// Per-thread register budget of the calling warpgroup (a multiple of 8 in [24, 256]).
+template <int kRegs>
+__device__ __forceinline__ void setmaxnreg_inc() { asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegs)); }
+template <int kRegs>
+__device__ __forceinline__ void setmaxnreg_dec() { asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegs)); }
 
 }  // namespace sm100
 }  // namespace ra

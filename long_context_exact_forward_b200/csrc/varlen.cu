@@ -1,0 +1,148 @@
+// varlen.cu -- ra_forward_varlen: the fused tensor-core ring forward pass over packed sequences.
+//
+// Several sequences of different lengths are packed one after another on the token axis; a query
+// attends only to the keys of its own sequence (and, causal, to those at or before it).  Each
+// sequence is split into the same n_ring shards with the requested layout, and its items
+// (sequence, head, shard, query-tile pair) join one work list, ordered longest first across all
+// sequences (troisinh.com "Ring Attention", "Trade-off thuc te": load balancing with sequences of
+// different lengths is the challenge; one list over every sequence lets the persistent kernel's
+// dynamic scheduler balance it).  The kernel reads the packed tensors in place through TMA maps over
+// the whole packed axis; rows past a sequence's end that a tile box still covers are masked by the
+// per-row key counts of that sequence.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <vector>
+
+#include "ra.h"
+#include "ra_internal.cuh"
+
+namespace {
+
+constexpr int kTileRows = 128;
+constexpr int kPairRows = 256;
+
+size_t align256(size_t x) { return (x + 255) / 256 * 256; }
+
+// Live 128-key tiles of block j for the query tile starting at local row a0 of shard i.
+int64_t live_tiles(const ra::Layout& L, int causal, int64_t i, int64_t a0, int64_t j) {
+    if (a0 >= L.S_loc) return 0;
+    const int64_t last = std::min(a0 + kTileRows - 1, L.S_loc - 1);
+    return (ra::visible_keys(L, causal, i, last, j) + kTileRows - 1) / kTileRows;
+}
+
+struct Item {
+    int4 it;
+    int64_t cost;
+};
+
+}  // namespace
+
+extern "C" int ra_forward_varlen(const void* q, const void* k, const void* v, void* out, float* lse,
+                                 const int64_t* cu_seqlens, int n_seqs, int64_t H, int64_t D, int n_ring,
+                                 int causal, int layout, void* stream_handle) {
+    if (!q || !k || !v || !out || !lse || !cu_seqlens || n_seqs < 1 || H < 1 || n_ring < 1) return RA_ERR_INVALID_ARG;
+    if (layout != RA_LAYOUT_CONTIGUOUS && layout != RA_LAYOUT_STRIPED) {
+        ra::host_set_error("ra_forward_varlen: contiguous or striped layout");
+        return RA_ERR_UNSUPPORTED;
+    }
+    if (D != 64 && D != 128) return RA_ERR_UNSUPPORTED;
+    if (cu_seqlens[0] != 0) return RA_ERR_INVALID_ARG;
+    for (int s = 0; s < n_seqs; ++s) {
+        const int64_t len = cu_seqlens[s + 1] - cu_seqlens[s];
+        if (len < 0) return RA_ERR_INVALID_ARG;
+        if (len % n_ring) return RA_ERR_SHAPE;
+    }
+    const int64_t S_total = cu_seqlens[n_seqs];
+    if (S_total >= (int64_t(1) << 31) || H * D * 2 % 16) return RA_ERR_SHAPE;
+    auto a16 = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; };
+    if (!a16(q) || !a16(k) || !a16(v) || !a16(out) || (reinterpret_cast<uintptr_t>(lse) & 3u)) return RA_ERR_ALIGN;
+    int sms = 0;
+    bool sm100 = false;
+    int* status = nullptr;
+    int rc = ra::host_device_facts(&sms, &sm100, &status);
+    if (rc != RA_OK) return rc;
+    if (!sm100) return RA_ERR_UNSUPPORTED;
+    if (S_total == 0) return RA_OK;
+
+    // work list: every (sequence, head, shard, pair), longest first (ties in list order)
+    const int64_t N = n_ring;
+    std::vector<Item> items;
+    std::vector<int2> seqs(n_seqs);
+    for (int s = 0; s < n_seqs; ++s) {
+        const int64_t len = cu_seqlens[s + 1] - cu_seqlens[s];
+        seqs[s] = make_int2((int)len, (int)cu_seqlens[s]);
+        if (len == 0) continue;
+        const ra::Layout L{len, N, len / N, layout};
+        const int64_t pairs = (L.S_loc + kPairRows - 1) / kPairRows;
+        for (int64_t i = 0; i < N; ++i)
+            for (int64_t p = 0; p < pairs; ++p) {
+                int64_t cost = 0;
+                for (int64_t st = 0; st < N; ++st) {
+                    const int64_t j = ra::ring_block(i, st, N);
+                    cost += live_tiles(L, causal, i, p * kPairRows, j) + live_tiles(L, causal, i, p * kPairRows + kTileRows, j);
+                }
+                for (int64_t h = 0; h < H; ++h) items.push_back({make_int4(s, (int)h, (int)i, (int)p), cost});
+            }
+    }
+    std::stable_sort(items.begin(), items.end(), [](const Item& a, const Item& b) { return a.cost > b.cost; });
+    std::vector<int4> list(items.size());
+    for (size_t t = 0; t < items.size(); ++t) list[t] = items[t].it;
+    if (list.size() > (size_t)INT32_MAX) return RA_ERR_SHAPE;
+
+    cudaStream_t stream = static_cast<cudaStream_t>(stream_handle);
+    const size_t off_seqs = 256, off_items = off_seqs + align256(seqs.size() * sizeof(int2));
+    const size_t bytes = off_items + align256(list.size() * sizeof(int4));
+    uint8_t* ws = nullptr;
+    cudaError_t e = cudaMallocAsync(reinterpret_cast<void**>(&ws), bytes, stream);
+    if (e != cudaSuccess) return ra::host_cuda_fail(e, "cudaMallocAsync(varlen scratch)");
+    auto finish = [&](int r) {
+        const cudaError_t ef = cudaFreeAsync(ws, stream);
+        if (r == RA_OK && ef != cudaSuccess) return ra::host_cuda_fail(ef, "cudaFreeAsync(varlen scratch)");
+        return r;
+    };
+    // pageable sources: each copy returns once its data is staged, so the vectors may go out of scope
+    if ((e = cudaMemsetAsync(ws, 0, sizeof(int), stream)) != cudaSuccess ||
+        (e = cudaMemcpyAsync(ws + off_seqs, seqs.data(), seqs.size() * sizeof(int2), cudaMemcpyHostToDevice,
+                             stream)) != cudaSuccess ||
+        (e = cudaMemcpyAsync(ws + off_items, list.data(), list.size() * sizeof(int4), cudaMemcpyHostToDevice,
+                             stream)) != cudaSuccess)
+        return finish(ra::host_cuda_fail(e, "varlen work list upload"));
+
+    // TMA maps over the packed axis: contiguous (D, H, S_total, 1, 1); striped (D, H, S_total / N, N, 1)
+    // with token = a' * N + i (every sequence starts on a multiple of N)
+    const bool striped = layout == RA_LAYOUT_STRIPED;
+    const ra::Layout Lmap = striped ? ra::Layout{S_total, N, S_total / N, layout} : ra::Layout{S_total, 1, S_total, layout};
+    ra::TcLaunch t{};
+    if ((rc = ra::host_encode_qkv_map(&t.tm_q, q, 1, Lmap, H, D, striped)) != RA_OK ||
+        (rc = ra::host_encode_qkv_map(&t.tm_k, k, 1, Lmap, H, D, striped)) != RA_OK ||
+        (rc = ra::host_encode_qkv_map(&t.tm_v, v, 1, Lmap, H, D, striped)) != RA_OK)
+        return finish(rc);
+    t.items = reinterpret_cast<const int4*>(ws + off_items);
+    t.n_items = (int)list.size();
+    t.counter = reinterpret_cast<int*>(ws);
+    t.grid = (int)std::min<int64_t>((int64_t)list.size(), sms);
+    t.timeout_ns = 2000000000ull;
+    t.debug = 0;
+    t.status = status;
+
+    ra::AttnArgs a{};
+    a.L = ra::Layout{S_total, N, S_total / N, layout};  // S = S_total; N and the kind apply per sequence
+    a.B = 1;
+    a.H = H;
+    a.D = D;
+    a.causal = causal ? 1 : 0;
+    a.dtype = RA_DTYPE_BF16;
+    a.s_begin = 0;
+    a.s_end = n_ring;
+    a.out_mode = ra::kOutFinal;
+    a.out = out;
+    a.lse = lse;
+    a.scale = (float)(1.0 / std::sqrt((double)D));
+    a.seqs = reinterpret_cast<const int2*>(ws + off_seqs);
+    a.varlen_striped = striped ? 1 : 0;
+    if ((e = ra::launch_attn_tc(a, t, stream)) != cudaSuccess) return finish(ra::host_cuda_fail(e, "attention launch"));
+    return finish(RA_OK);
+}
