@@ -35,6 +35,23 @@ METRIC = "ring-attn fwd TFLOP/s (bf16, causal) and % of B200 dense BF16 tensor p
 # --backward runs: gradient flops counted as 2.5x the forward flops (five S x S x D products:
 # the recomputed scores, dP, dV, dQ, dK), halved for causal like the forward
 METRIC_BWD = "ring-attn bwd TFLOP/s (causal; 2.5x forward flops)"
+# --varlen runs: packed sequences, flops summed per sequence (4 * H * len^2 * D, halved for causal)
+METRIC_VARLEN = "ring-attn fwd TFLOP/s over packed variable-length sequences (bf16, causal)"
+
+
+def varlen_lengths(S, n_ring, seed):
+    """A seeded mix of sequence lengths that fills S tokens: multiples of 128 * n_ring between
+    S / 64 and S / 4 (the last one takes what is left)."""
+    import random
+    rng = random.Random(seed)
+    unit = 128 * n_ring
+    lo, hi = max(1, S // 64 // unit), max(1, S // 4 // unit)
+    out, left = [], S
+    while left > 0:
+        n = min(rng.randint(lo, hi) * unit, left)
+        out.append(n)
+        left -= n
+    return out
 UNIT = "TFLOP/s"
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
@@ -215,6 +232,7 @@ def config_dict(w, args):
         "l2": f"inputs (3 x B*S*H*D {args.dtype}) larger than the 126 MB L2; no flush"
               if 3 * w.B * w.S * w.H * w.D * (4 if args.dtype == "fp32" else 2) > 126e6
               else "inputs smaller than the 126 MB L2 (kernel-level runs; not the headline)",
+        **({"varlen_lengths": varlen_lengths(w.S, w.n_ring, w.seed)} if getattr(args, "varlen", False) else {}),
     }
 
 
@@ -288,6 +306,21 @@ def run_ours(args, w):
     def step(ev=None):
         ra.forward(q, k, v, N, True, args.layout, variant=args.variant, kernel=args.kernel, out=out,
                    lse=lse, workspace=ws, stream=stream, events=ev)
+
+    if args.varlen:
+        lengths = varlen_lengths(S, N, w.seed)
+        cu = [0]
+        for n in lengths:
+            cu.append(cu[-1] + n)
+        lse_v = torch.empty((H, S), dtype=torch.float32, device=dev)
+        flops = sum(attention_flops(1, H, n, D, True) for n in lengths)
+
+        def step(ev=None):
+            if ev is not None:
+                ev[0].record(stream)
+            ra.forward_varlen(q[0], k[0], v[0], cu, N, True, args.layout, out=out[0], lse=lse_v, stream=stream)
+            if ev is not None:
+                ev[1].record(stream)
 
     if args.backward:
         # one forward pass outside the timed region supplies out and lse; a step is one ra_backward
@@ -435,11 +468,13 @@ def run_ours(args, w):
         roofline = {
             "bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
             "traffic": (args.traffic_bytes if args.traffic_bytes is not None
-                        else None if args.backward else recorded_traffic(args)),
+                        else None if (args.backward or args.varlen) else recorded_traffic(args)),
             "peak_kind": f"bf16 dense cuBLAS, sustained ({peak_src})",
             "frac_of_burst_peak": achieved / peaks["bf16_tflops"],
             "kernel": ("bwd_dq_tc_kernel + bwd_dkv_tc_kernel (tcgen05), timed as one ra_backward call"
-                       if args.backward else "attn_tc_kernel<128> (fused ring, tcgen05)"),
+                       if args.backward else
+                       "attn_tc_kernel<128, varlen> (fused ring, tcgen05), timed as one ra_forward_varlen call"
+                       if args.varlen else "attn_tc_kernel<128> (fused ring, tcgen05)"),
             "kernel_ms": k_ms,
             "algorithmic_flops_per_launch": flops,
         }
@@ -461,7 +496,7 @@ def run_ours(args, w):
     if args.backward:
         launches_per_step = 3  # Delta, dq, dk/dv
     line = {
-        "metric": METRIC_BWD if args.backward else METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "metric": METRIC_BWD if args.backward else METRIC_VARLEN if args.varlen else METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f32" if fp32 else "bf16", "data": "synthetic",
         "config": config_dict(w, args),
@@ -492,6 +527,9 @@ def main():
     ap.add_argument("--dtype", default="bf16", choices=["bf16", "fp32"])
     ap.add_argument("--bwd-kernel", default="auto", choices=["auto", "tc", "simt"],
                     help="backward path for --backward runs (auto: tensor cores where they apply)")
+    ap.add_argument("--varlen", action="store_true",
+                    help="time ra_forward_varlen over a seeded mix of packed sequences filling the workload's "
+                         "tokens (needs --no-e2e --no-cpu-baseline; not the headline)")
     ap.add_argument("--backward", action="store_true",
                     help="time ra_backward (needs --no-e2e and --no-cpu-baseline; not the headline)")
     ap.add_argument("--no-e2e", action="store_true")
@@ -502,8 +540,10 @@ def main():
     ap.add_argument("--traffic-bytes", type=float, default=None,
                     help="DRAM bytes per attention launch from an ncu capture of this kernel")
     args = ap.parse_args()
-    if args.backward and not (args.no_e2e and args.no_cpu_baseline):
-        ap.error("--backward runs time the device call only: add --no-e2e --no-cpu-baseline")
+    if (args.backward or args.varlen) and not (args.no_e2e and args.no_cpu_baseline):
+        ap.error("--backward / --varlen runs time the device call only: add --no-e2e --no-cpu-baseline")
+    if args.backward and args.varlen:
+        ap.error("--backward and --varlen are separate runs")
     if args.kernel == "tc" and args.dtype == "fp32":
         ap.error("the tensor-core kernel takes bf16 inputs; fp32 runs on --kernel simt")
     w = inputs.WORKLOADS[args.workload]
