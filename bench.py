@@ -58,7 +58,7 @@ PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # DRAM bytes (read + write) per attention launch on s128k striped, from an ncu capture of the
 # 4-head case scaled by heads (profiles/attn_tc_fused_s128k_striped.md); valid only while
 # sha256(attn_tc.cu + api.cu) starts with the recorded prefix -- otherwise traffic is null.
-TRAFFIC_RECORD = {"source_sha256_prefix": "7caf598abf792ad0", "bytes_per_launch": 3.645195e9 * 8}
+TRAFFIC_RECORD = {"source_sha256_prefix": "19d20a87f3c3cd75", "bytes_per_launch": 3.634440e9 * 8}
 # the files whose concatenation the record's hash covers: the kernel, the helpers it inlines and
 # the host code that decides the layout it reads
 TRAFFIC_SOURCES = ("attn_tc.cu", "sm100.cuh", "layout.cuh", "api.cu")
