@@ -79,3 +79,25 @@ def test_workspace_size_grows_with_per_step_and_permute():
 def test_workspace_size_rejects_bad_shape():
     with pytest.raises(ra.RAError):
         ra.workspace_size(1, 1, 10, 16, 3, False, "contiguous", 0)
+
+
+def test_backward_rope_and_varlen_validate_before_any_cuda_call():
+    lib = ra.lib()
+    # ra_backward_ex: S not divisible by n_ring; bad kernel code; head dim above 128
+    assert lib.ra_backward_ex(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1, 2, 63, 16, 4, 1, 0, 0,
+                              0, 0, 0, None) == -2
+    assert lib.ra_backward_ex(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1, 2, 64, 16, 4, 1, 0, 0,
+                              9, 0, 0, None) == -1
+    assert lib.ra_backward_ex(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1, 2, 64, 256, 4, 1, 0, 1,
+                              0, 0, 0, None) == -4
+    # ra_rope: odd head dim, negative offset, misaligned pointer
+    assert lib.ra_rope(FAKE, FAKE, 1, 4, 1, 3, 0, 10000.0, 0, None) == -1
+    assert lib.ra_rope(FAKE, FAKE, 1, 4, 1, 4, -1, 10000.0, 0, None) == -1
+    assert lib.ra_rope(FAKE + 2, FAKE, 1, 4, 1, 4, 0, 10000.0, 0, None) == -3
+    # ra_forward_varlen: a length not divisible by n_ring, zigzag, cu[0] != 0
+    cu = np.array([0, 50, 100], dtype=np.int64)
+    assert lib.ra_forward_varlen(FAKE, FAKE, FAKE, FAKE, FAKE, cu.ctypes.data, 2, 1, 128, 4, 1, 0, None) == -2
+    cu = np.array([0, 64, 128], dtype=np.int64)
+    assert lib.ra_forward_varlen(FAKE, FAKE, FAKE, FAKE, FAKE, cu.ctypes.data, 2, 1, 128, 4, 1, 2, None) == -4
+    cu = np.array([4, 64, 128], dtype=np.int64)
+    assert lib.ra_forward_varlen(FAKE, FAKE, FAKE, FAKE, FAKE, cu.ctypes.data, 2, 1, 128, 4, 1, 0, None) == -1
