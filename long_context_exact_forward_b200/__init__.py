@@ -1,4 +1,4 @@
-"""Ring Attention exact forward on NVIDIA B200 (sm_100a).
+"""Ring Attention exact forward (and backward) on NVIDIA B200 (sm_100a).
 
 A thin ctypes binding over the C ABI of ``include/ra.h`` (``libra_b200.so``, built in-tree by
 ``python -m long_context_exact_forward_b200._build``).  Every step of the computation runs in the
@@ -8,6 +8,10 @@ device is not a CUDA device the calls raise.
 
 Entry points (same names as the C ABI):
     forward(q, k, v, n_ring, causal, layout, ...)   -> (out, lse)      ra_forward_ex
+    forward_noalloc(q, k, v, n_ring, causal, layout) -> (out, lse)      ra_forward_noalloc
+    forward_varlen(q, k, v, cu_seqlens, n_ring, ...) -> (out, lse)      ra_forward_varlen
+    backward(q, k, v, out, lse, dout, n_ring, ...)   -> (dq, dk, dv)    ra_backward_ex
+    rope(x, pos_offset, base)                        -> tensor          ra_rope
     workspace_size(...)                              -> int             ra_workspace_size
     permute(x, n_ring, layout) / unpermute(...)      -> tensor          ra_permute / ra_unpermute
     merge_partials(O_run, lse_run, O_step, lse_step)                     ra_merge_partials
