@@ -72,3 +72,40 @@ def test_noalloc_rejects_problems_beyond_its_scratch():
     q2, k2, v2 = inputs.make_qkv(1, 256, 1, 96, torch.bfloat16, "cuda", seed=2)
     rc, _, _ = call_noalloc(q2, k2, v2, 2, True, "contiguous")
     assert rc == -4  # RA_ERR_UNSUPPORTED: head dim outside the tensor-core kernel
+
+
+def test_noalloc_call_replays_from_a_cuda_graph():
+    # the use the entry point exists for: record it once in a CUDA graph, then replay the graph on
+    # new inputs copied into the same buffers; each replay matches the allocating entry point
+    B, H, S, D, N = 1, 2, 4 * 512, 128, 4
+    q, k, v = inputs.make_qkv(B, S, H, D, torch.bfloat16, "cuda", seed=7)
+    out = torch.empty_like(q)
+    lse = torch.empty((B, H, S), dtype=torch.float32, device="cuda")
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        # the first call on the device looks up the scratch array; it happens before the capture
+        rc = ra.lib().ra_forward_noalloc(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                                         lse.data_ptr(), B, H, S, D, N, 1, ra.LAYOUTS["striped"],
+                                         ctypes.c_void_p(side.cuda_stream))
+        assert rc == 0
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        rc = ra.lib().ra_forward_noalloc(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                                         lse.data_ptr(), B, H, S, D, N, 1, ra.LAYOUTS["striped"],
+                                         ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+    assert rc == 0
+    for seed in (8, 9):
+        nq, nk, nv = inputs.make_qkv(B, S, H, D, torch.bfloat16, "cuda", seed=seed)
+        q.copy_(nq)
+        k.copy_(nk)
+        v.copy_(nv)
+        graph.replay()
+        ref, ref_lse = ra.forward(q, k, v, N, True, "striped")
+        torch.cuda.synchronize()
+        assert ra.get_device_status() == 0
+        d = (out.float() - ref.float()).abs()
+        assert d.max().item() <= 2e-2 and d.mean().item() <= 2e-3
+        assert (lse - ref_lse).abs().max().item() <= 1e-3
