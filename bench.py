@@ -202,18 +202,19 @@ def run_reference(args, w):
         return
     q, k, v = inputs.make_qkv(w.B, w.S, w.H, w.D, torch.bfloat16, "cpu", w.seed)
     rows_per_head = args.ref_rows
+    causal = causal_of(args)
     for _ in range(args.warmup):
-        oracle_sample(q, k, v, True, rows_per_head)
+        oracle_sample(q, k, v, causal, rows_per_head)
     tot_f, tot_t = 0.0, 0.0
     for _ in range(args.steps):
-        f, dt, threads, n = oracle_sample(q, k, v, True, rows_per_head)
+        f, dt, threads, n = oracle_sample(q, k, v, causal, rows_per_head)
         tot_f += f
         tot_t += dt
     value = tot_f / tot_t / 1e12
-    sample = (f"{rows_per_head} query rows per head x {w.H} heads of {w.name} (causal), "
+    sample = (f"{rows_per_head} query rows per head x {w.H} heads of {w.name} ({mask_word(args)}), "
               f"{tot_f / args.steps:.3e} flops per step")
     line = {
-        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "impl": "reference", "metric": metric_of(args), "value": value, "unit": UNIT, "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": tot_t / args.steps * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic", "config": config_dict(w, args),
@@ -223,11 +224,27 @@ def run_reference(args, w):
     print(json.dumps(line), flush=True)
 
 
+def causal_of(args):
+    return not getattr(args, "non_causal", False)
+
+
+def mask_word(args):
+    return "causal" if causal_of(args) else "non-causal"
+
+
+def metric_of(args):
+    """The metric named by the run: the headline forward metric, or that of a --backward /
+    --varlen run; "causal" becomes "non-causal" under --non-causal."""
+    m = METRIC_BWD if getattr(args, "backward", False) else METRIC_VARLEN if getattr(args, "varlen", False) else METRIC
+    return m if causal_of(args) else m.replace("causal", "non-causal")
+
+
 def config_dict(w, args):
     return {
         "workload": f"{w.name}: batch {w.B}, {w.H} heads, head dim {w.D}, {w.S} tokens in {w.n_ring} "
-                    f"shards of {w.S_loc}, {args.dtype}, causal, {args.layout} layout",
-        "B": w.B, "H": w.H, "S": w.S, "D": w.D, "n_ring": w.n_ring, "causal": True,
+                    f"shards of {w.S_loc}, {args.dtype}, {'causal' if causal_of(args) else 'non-causal'}, "
+                    f"{args.layout} layout",
+        "B": w.B, "H": w.H, "S": w.S, "D": w.D, "n_ring": w.n_ring, "causal": causal_of(args),
         "layout": args.layout, "variant": args.variant, "kernel": args.kernel,
         "l2": f"inputs (3 x B*S*H*D {args.dtype}) larger than the 126 MB L2; no flush"
               if 3 * w.B * w.S * w.H * w.D * (4 if args.dtype == "fp32" else 2) > 126e6
@@ -298,13 +315,14 @@ def run_ours(args, w):
     q, k, v = inputs.make_qkv(B, S, H, D, torch.float32 if fp32 else torch.bfloat16, dev, w.seed + rank)
     out = torch.empty_like(q)
     lse = torch.empty((B, H, S), dtype=torch.float32, device=dev)
-    ws = torch.empty(ra.workspace_size(B, H, S, D, N, True, args.layout, 0 if fp32 else 1,
+    causal = causal_of(args)
+    ws = torch.empty(ra.workspace_size(B, H, S, D, N, causal, args.layout, 0 if fp32 else 1,
                                        variant=args.variant, kernel=args.kernel),
                      dtype=torch.uint8, device=dev)
-    flops = attention_flops(B, H, S, D, True)
+    flops = attention_flops(B, H, S, D, causal)
 
     def step(ev=None):
-        ra.forward(q, k, v, N, True, args.layout, variant=args.variant, kernel=args.kernel, out=out,
+        ra.forward(q, k, v, N, causal, args.layout, variant=args.variant, kernel=args.kernel, out=out,
                    lse=lse, workspace=ws, stream=stream, events=ev)
 
     if args.varlen:
@@ -313,12 +331,12 @@ def run_ours(args, w):
         for n in lengths:
             cu.append(cu[-1] + n)
         lse_v = torch.empty((H, S), dtype=torch.float32, device=dev)
-        flops = sum(attention_flops(1, H, n, D, True) for n in lengths)
+        flops = sum(attention_flops(1, H, n, D, causal) for n in lengths)
 
         def step(ev=None):
             if ev is not None:
                 ev[0].record(stream)
-            ra.forward_varlen(q[0], k[0], v[0], cu, N, True, args.layout, out=out[0], lse=lse_v, stream=stream)
+            ra.forward_varlen(q[0], k[0], v[0], cu, N, causal, args.layout, out=out[0], lse=lse_v, stream=stream)
             if ev is not None:
                 ev[1].record(stream)
 
@@ -328,12 +346,12 @@ def run_ours(args, w):
         dout = torch.randn(q.shape, generator=gen, device=dev, dtype=torch.float32).to(q.dtype)
         step()
         dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
-        flops = 2.5 * attention_flops(B, H, S, D, True)
+        flops = 2.5 * attention_flops(B, H, S, D, causal)
 
         def step(ev=None):
             if ev is not None:
                 ev[0].record(stream)
-            ra.backward(q, k, v, out, lse, dout, N, True, args.layout, kernel=args.bwd_kernel, dq=dq, dk=dk,
+            ra.backward(q, k, v, out, lse, dout, N, causal, args.layout, kernel=args.bwd_kernel, dq=dq, dk=dk,
                         dv=dv, stream=stream)
             if ev is not None:
                 ev[1].record(stream)
@@ -394,7 +412,7 @@ def run_ours(args, w):
                 stream.wait_event(ev_in[b])
                 if st >= 2:
                     stream.wait_event(ev_free_out[b])
-                ra.forward(dq[b][0], dq[b][1], dq[b][2], N, True, args.layout, variant=args.variant, kernel=args.kernel,
+                ra.forward(dq[b][0], dq[b][1], dq[b][2], N, causal, args.layout, variant=args.variant, kernel=args.kernel,
                            out=do[b], lse=dl[b], workspace=ws, stream=stream)
                 ev_free_in[b].record(stream)
                 ev_done[b].record(stream)
@@ -417,7 +435,7 @@ def run_ours(args, w):
         def serial_step():
             for dst, src in zip(dq[0], (qh, kh, vh)):
                 dst.copy_(src, non_blocking=True)
-            ra.forward(dq[0][0], dq[0][1], dq[0][2], N, True, args.layout, variant=args.variant, kernel=args.kernel,
+            ra.forward(dq[0][0], dq[0][1], dq[0][2], N, causal, args.layout, variant=args.variant, kernel=args.kernel,
                        out=do[0], lse=dl[0], workspace=ws, stream=stream)
             oh[0].copy_(do[0], non_blocking=True)
             lh[0].copy_(dl[0], non_blocking=True)
@@ -483,9 +501,9 @@ def run_ours(args, w):
     cpu = None
     if not args.no_cpu_baseline and world == 1 and rank == 0:
         qc, kc, vc = q.cpu(), k.cpu(), v.cpu()
-        f, dt, threads, n = oracle_sample(qc, kc, vc, True, args.cpu_rows)
+        f, dt, threads, n = oracle_sample(qc, kc, vc, causal, args.cpu_rows)
         cpu = {"value": f / dt / 1e12, "unit": UNIT, "cores": threads, "kind": "oracle",
-               "sample": f"{args.cpu_rows} query rows per head x {H} heads of {w.name} (causal), "
+               "sample": f"{args.cpu_rows} query rows per head x {H} heads of {w.name} ({mask_word(args)}), "
                          f"{f:.3e} flops in {dt:.1f} s"}
 
     # our kernels per step: the zigzag permute (striped and contiguous are read in place) and the
@@ -496,7 +514,7 @@ def run_ours(args, w):
     if args.backward:
         launches_per_step = 3  # Delta, dq, dk/dv
     line = {
-        "metric": METRIC_BWD if args.backward else METRIC_VARLEN if args.varlen else METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "metric": metric_of(args), "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f32" if fp32 else "bf16", "data": "synthetic",
         "config": config_dict(w, args),
@@ -525,6 +543,8 @@ def main():
     ap.add_argument("--kernel", default="tc", choices=["tc", "simt"],
                     help="tc: the tcgen05 kernel (the headline); simt: the fp32 CUDA-core kernel")
     ap.add_argument("--dtype", default="bf16", choices=["bf16", "fp32"])
+    ap.add_argument("--non-causal", action="store_true",
+                    help="no causal mask (flops not halved; not the headline)")
     ap.add_argument("--bwd-kernel", default="auto", choices=["auto", "tc", "simt"],
                     help="backward path for --backward runs (auto: tensor cores where they apply)")
     ap.add_argument("--varlen", action="store_true",
