@@ -122,3 +122,37 @@ def test_work_list_groups_shards_when_a_head_exceeds_l2():
     # below the threshold the plain heaviest-first order is kept
     small = ra.plan_items(1, 1, 65536, 16, True, "striped", D=128)
     assert (np.diff(small[:, 4]) <= 0).all()
+
+
+def test_random_shapes_layouts_and_tiles_against_brute_force():
+    # seeded random shapes beyond the fixed list: every (query, key) pair of the tile classes agrees
+    # with the mask computed from the oracle's positions, and the work list covers each item once
+    rng = np.random.default_rng(2024)
+    for _ in range(25):
+        N = int(rng.integers(1, 7))
+        layout = ["contiguous", "striped", "zigzag"][int(rng.integers(3))]
+        unit = 2 * N if layout == "zigzag" else N
+        S = unit * int(rng.integers(1, 12))
+        tile = int(rng.integers(1, 9))
+        causal = bool(rng.integers(2))
+        pos = oracle.layout_positions(S, N, layout)
+        np.testing.assert_array_equal(ra.layout_positions(S, N, layout), pos)
+        S_loc = S // N
+        nt = -(-S_loc // tile)
+        cls = ra.plan_tiles(S, N, layout, causal, tile)
+        for i in range(N):
+            for s in range(N):
+                j = (i - s) % N
+                for qt in range(nt):
+                    qa = np.arange(qt * tile, min((qt + 1) * tile, S_loc))
+                    for kt in range(nt):
+                        ka = np.arange(kt * tile, min((kt + 1) * tile, S_loc))
+                        gq, gk = pos[i, qa][:, None], pos[j, ka][None, :]
+                        allowed = (gk <= gq) if causal else np.ones((qa.size, ka.size), dtype=bool)
+                        c = cls[i, s, qt, kt]
+                        if c == 0:
+                            assert not allowed.any(), (S, N, layout, causal, tile, i, s, qt, kt)
+                        elif c == 1:
+                            assert allowed.all() and ka.size == tile, (S, N, layout, causal, tile, i, s, qt, kt)
+                        else:
+                            assert allowed.any(), (S, N, layout, causal, tile, i, s, qt, kt)
