@@ -57,7 +57,8 @@ PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 
 # DRAM bytes (read + write) per attention launch on s128k striped, from an ncu capture of the
 # 4-head case scaled by heads (profiles/attn_tc_fused_s128k_striped.md); valid only while
-# sha256(attn_tc.cu + api.cu) starts with the recorded prefix -- otherwise traffic is null.
+# the sha256 of the TRAFFIC_SOURCES files, concatenated in that order, starts with the recorded
+# prefix -- otherwise traffic is null.
 TRAFFIC_RECORD = {"source_sha256_prefix": "19d20a87f3c3cd75", "bytes_per_launch": 3.634440e9 * 8}
 # the files whose concatenation the record's hash covers: the kernel, the helpers it inlines and
 # the host code that decides the layout it reads

@@ -254,8 +254,15 @@ RA_API int ra_rope(const void* x, void* y, int64_t B, int64_t S, int64_t H, int6
 /* ra_status_string: static description of a status code. */
 RA_API const char* ra_status_string(int status);
 
-/* ra_last_error_string: description of the last RA_ERR_CUDA on the calling host thread. */
+/* ra_last_error_string: the message of the last error recorded on the calling host thread: every
+ * RA_ERR_CUDA records one, and so do the validation failures whose code alone is ambiguous (for
+ * example RA_ERR_NO_WORKSPACE of ra_forward_noalloc).  Messages persist until the next one or until
+ * ra_clear_last_error; the string is owned by the library and valid until the thread's next call. */
 RA_API const char* ra_last_error_string(void);
+
+/* ra_clear_last_error: empty the calling host thread's message, so that a non-empty message after a
+ * failing call belongs to that call. */
+RA_API void ra_clear_last_error(void);
 
 /* ra_get_device_status: read and clear the status word that the kernels of this library set on
  * the current device (RA_OK, or RA_ERR_DEVICE_TIMEOUT after a bounded wait ran out).  Call it

@@ -97,6 +97,8 @@ def lib():
         L.ra_last_error_string.restype = ctypes.c_char_p
         L.ra_last_error_string.argtypes = []
         L.ra_get_device_status.argtypes = []
+        L.ra_clear_last_error.argtypes = []
+        L.ra_clear_last_error.restype = None
         for name in ("ra_forward", "ra_forward_ex", "ra_forward_noalloc", "ra_workspace_size", "ra_permute",
                      "ra_unpermute", "ra_merge_partials", "ra_layout_positions", "ra_plan_tiles",
                      "ra_plan_items", "ra_get_device_status", "ra_backward", "ra_backward_ex", "ra_rope", "ra_forward_varlen"):
@@ -105,10 +107,30 @@ def lib():
     return _lib
 
 
+def _last_error():
+    return lib().ra_last_error_string().decode()
+
+
+def _clear_error():
+    """Empty the library's per-thread message before a call, so that whatever it holds after a
+    failure was recorded by that call."""
+    lib().ra_clear_last_error()
+
+
 def _check(rc, where):
+    """Raise RAError for a non-zero status, with the library's message when the call left one."""
     if rc != RA_OK:
-        detail = lib().ra_last_error_string().decode() if rc == -6 else ""
-        raise RAError(rc, where, detail)
+        raise RAError(rc, where, _last_error())
+
+
+def _check_out(t, shape, dtype, name, like=None):
+    """A caller-supplied output tensor must match the shape and dtype the kernels write, live on
+    the inputs' device and be contiguous; otherwise the kernels would write outside it."""
+    _check_cuda(t)
+    if tuple(t.shape) != tuple(shape) or t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype} {list(shape)}, got {t.dtype} {list(t.shape)}")
+    if like is not None and t.device != like.device:
+        raise ValueError(f"{name} must be on {like.device}")
 
 
 def _torch():
@@ -142,6 +164,7 @@ def _check_cuda(*ts):
 
 def workspace_size(B, H, S, D, n_ring, causal, layout, dtype_code, variant="auto", kernel="auto"):
     n = ctypes.c_size_t(0)
+    _clear_error()
     _check(lib().ra_workspace_size(B, H, S, D, n_ring, int(bool(causal)), LAYOUTS[layout],
                                    dtype_code, VARIANTS[variant], KERNELS[kernel], ctypes.byref(n)),
            "ra_workspace_size")
@@ -168,7 +191,8 @@ def forward(q, k, v, n_ring, causal=True, layout="contiguous", *, variant="auto"
         out = torch.empty_like(q)
     if lse is None:
         lse = torch.empty((B, H, S), dtype=torch.float32, device=q.device)
-    _check_cuda(out, lse)
+    _check_out(out, q.shape, q.dtype, "out", q)
+    _check_out(lse, (B, H, S), torch.float32, "lse", q)
     opt = Options()
     opt.variant = VARIANTS[variant]
     opt.kernel = KERNELS[kernel]
@@ -184,6 +208,7 @@ def forward(q, k, v, n_ring, causal=True, layout="contiguous", *, variant="auto"
                 ev.record(stream if stream is not None else torch.cuda.current_stream())
         opt.attn_events[0] = events[0].cuda_event
         opt.attn_events[1] = events[1].cuda_event
+    _clear_error()
     with torch.cuda.device(q.device):
         rc = lib().ra_forward_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
                                  lse.data_ptr(), B, H, S, D, int(n_ring), int(bool(causal)),
@@ -201,12 +226,16 @@ def forward_noalloc(q, k, v, n_ring, causal=True, layout="contiguous", *, out=No
     _check_cuda(q, k, v)
     if q.dtype != torch.bfloat16 or k.dtype != q.dtype or v.dtype != q.dtype:
         raise TypeError("forward_noalloc takes bf16 q, k, v")
+    if q.dim() != 4 or q.shape != k.shape or q.shape != v.shape:
+        raise ValueError("q, k, v must all be [B, S, H, D]")
     B, S, H, D = q.shape
     if out is None:
         out = torch.empty_like(q)
     if lse is None:
         lse = torch.empty((B, H, S), dtype=torch.float32, device=q.device)
-    _check_cuda(out, lse)
+    _check_out(out, q.shape, q.dtype, "out", q)
+    _check_out(lse, (B, H, S), torch.float32, "lse", q)
+    _clear_error()
     with torch.cuda.device(q.device):
         rc = lib().ra_forward_noalloc(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
                                       lse.data_ptr(), B, H, S, D, int(n_ring), int(bool(causal)),
@@ -233,7 +262,9 @@ def backward(q, k, v, out, lse, dout, n_ring, causal=True, layout="contiguous", 
     dq = torch.empty_like(q) if dq is None else dq
     dk = torch.empty_like(k) if dk is None else dk
     dv = torch.empty_like(v) if dv is None else dv
-    _check_cuda(dq, dk, dv)
+    for name, g in (("dq", dq), ("dk", dk), ("dv", dv)):
+        _check_out(g, q.shape, q.dtype, name, q)
+    _clear_error()
     with torch.cuda.device(q.device):
         rc = lib().ra_backward_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
                                   dout.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, H, S, D,
@@ -253,11 +284,17 @@ def forward_varlen(q, k, v, cu_seqlens, n_ring, causal=True, layout="contiguous"
     _check_cuda(q, k, v)
     if q.dim() != 3 or q.shape != k.shape or q.shape != v.shape:
         raise ValueError("q, k, v must all be [S_total, H, D]")
+    if q.dtype != torch.bfloat16 or k.dtype != q.dtype or v.dtype != q.dtype:
+        raise TypeError("forward_varlen takes bf16 q, k, v")
     S, H, D = q.shape
     cu = np.ascontiguousarray(np.asarray(cu_seqlens, dtype=np.int64))
+    if cu.ndim != 1 or cu.size < 2 or cu[-1] != S:
+        raise ValueError("cu_seqlens must hold n_seqs + 1 offsets ending at S_total")
     out = torch.empty_like(q) if out is None else out
     lse = torch.empty((H, S), dtype=torch.float32, device=q.device) if lse is None else lse
-    _check_cuda(out, lse)
+    _check_out(out, q.shape, q.dtype, "out", q)
+    _check_out(lse, (H, S), torch.float32, "lse", q)
+    _clear_error()
     with torch.cuda.device(q.device):
         rc = lib().ra_forward_varlen(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
                                      cu.ctypes.data, int(cu.size - 1), H, D, int(n_ring), int(bool(causal)),
@@ -274,8 +311,9 @@ def rope(x, pos_offset=0, base=10000.0, out=None, stream=None):
     if x.dim() != 4:
         raise ValueError("x must be [B, S, H, D]")
     out = torch.empty_like(x) if out is None else out
-    _check_cuda(out)
+    _check_out(out, x.shape, x.dtype, "out", x)
     B, S, H, D = x.shape
+    _clear_error()
     with torch.cuda.device(x.device):
         rc = lib().ra_rope(x.data_ptr(), out.data_ptr(), B, S, H, D, int(pos_offset), float(base),
                            _dtype_code(x), _stream_handle(stream))
@@ -287,11 +325,17 @@ def permute(x, n_ring, layout, out=None, stream=None, inverse=False):
     """Natural order [B, S, H, D] -> shard-major [B, n_ring, S/n_ring, H, D] (or back)."""
     torch = _torch()
     _check_cuda(x)
+    if x.dim() != (5 if inverse else 4) or int(n_ring) < 1:
+        raise ValueError("permute takes x [B, S, H, D], unpermute [B, n_ring, S_loc, H, D]; n_ring >= 1")
+    if inverse and x.shape[1] != n_ring:
+        raise ValueError("unpermute: x.shape[1] must equal n_ring")
     B, S, H, D = (x.shape[0], x.shape[1] * x.shape[2], x.shape[3], x.shape[4]) if inverse else x.shape
+    shape = (B, S, H, D) if inverse else (B, n_ring, S // n_ring, H, D)
     if out is None:
-        out = (torch.empty((B, S, H, D), dtype=x.dtype, device=x.device) if inverse else
-               torch.empty((B, n_ring, S // n_ring, H, D), dtype=x.dtype, device=x.device))
+        out = torch.empty(shape, dtype=x.dtype, device=x.device)
+    _check_out(out, shape, x.dtype, "out", x)
     fn = lib().ra_unpermute if inverse else lib().ra_permute
+    _clear_error()
     with torch.cuda.device(x.device):
         rc = fn(x.data_ptr(), out.data_ptr(), B, S, H, D, int(n_ring), LAYOUTS[layout],
                 _dtype_code(x), _stream_handle(stream))
@@ -312,6 +356,9 @@ def merge_partials(O_run, lse_run, O_step, lse_step, stream=None):
             raise TypeError("merge_partials works on fp32 tensors")
     D = O_run.shape[-1]
     rows = O_run.numel() // D
+    if O_step.shape != O_run.shape or lse_run.numel() != rows or lse_step.numel() != rows:
+        raise ValueError("O_step must match O_run, and lse_run, lse_step hold one value per row of O_run")
+    _clear_error()
     with torch.cuda.device(O_run.device):
         rc = lib().ra_merge_partials(O_run.data_ptr(), lse_run.data_ptr(), O_step.data_ptr(),
                                      lse_step.data_ptr(), rows, D, _stream_handle(stream))
@@ -321,14 +368,18 @@ def merge_partials(O_run, lse_run, O_step, lse_step, stream=None):
 
 def layout_positions(S, n_ring, layout):
     pos = np.empty(S, dtype=np.int64)
+    _clear_error()
     _check(lib().ra_layout_positions(S, n_ring, LAYOUTS[layout], pos.ctypes.data),
            "ra_layout_positions")
     return pos.reshape(n_ring, S // n_ring)
 
 
 def plan_tiles(S, n_ring, layout, causal, tile):
+    if n_ring < 1 or tile < 1:
+        raise ValueError("n_ring and tile must be >= 1")
     nt = -(-(S // n_ring) // tile)
     cls = np.empty((n_ring, n_ring, nt, nt), dtype=np.int8)
+    _clear_error()
     _check(lib().ra_plan_tiles(S, n_ring, LAYOUTS[layout], int(bool(causal)), tile,
                                cls.ctypes.data), "ra_plan_tiles")
     return cls
@@ -336,6 +387,7 @@ def plan_tiles(S, n_ring, layout, causal, tile):
 
 def plan_items(B, H, S, n_ring, causal, layout, D=128):
     n = ctypes.c_int64(0)
+    _clear_error()
     _check(lib().ra_plan_items(B, H, S, D, n_ring, int(bool(causal)), LAYOUTS[layout], None, 0,
                                ctypes.byref(n)), "ra_plan_items")
     items = np.empty((n.value, 5), dtype=np.int32)

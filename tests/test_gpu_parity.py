@@ -198,3 +198,21 @@ def test_caller_workspace_and_events():
         with pytest.raises(ra.RAError) as e:
             ra.forward(q, k, v, N, True, layout, variant=variant, workspace=small)
         assert e.value.code == -5
+
+
+def test_caller_outputs_of_the_wrong_size_are_refused_before_launch():
+    B, H, S, D, N = 1, 2, 512, 128, 4
+    q, k, v = inputs.make_qkv(B, S, H, D, dtype=torch.bfloat16, device="cuda", seed=11)
+    short = torch.empty((B, S - 128, H, D), dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(ValueError):
+        ra.forward(q, k, v, N, True, "striped", out=short)
+    with pytest.raises(ValueError):
+        ra.forward(q, k, v, N, True, "striped", lse=torch.empty((B, H, S - 1), device="cuda"))
+    with pytest.raises(ValueError):
+        ra.backward(q, k, v, q, torch.zeros((B, H, S), device="cuda"), q, N, True, "striped", dq=short)
+    with pytest.raises(ValueError):
+        ra.rope(q, out=short)
+    with pytest.raises(TypeError):
+        ra.forward_varlen(q[0].float(), k[0].float(), v[0].float(), [0, S], N)
+    torch.cuda.synchronize()
+    assert ra.get_device_status() == 0
