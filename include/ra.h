@@ -244,7 +244,8 @@ RA_API int ra_forward_varlen(const void* q, const void* k, const void* v, void* 
  * wherever its block travels on the ring).  x, y: [B, S, H, D] in natural token order, dtype fp32 or
  * bf16; the token at natural index g takes the position m = g + pos_offset (so a later chunk of a
  * sequence passes the length before it).  The pair (x[2p], x[2p+1]) is rotated by m * theta_p,
- * theta_p = base^(-2p/D) (10000 is the usual base).  y may equal x (in place).  D even, <= 256;
+ * theta_p = base^(-2p/D) (10000 is the usual base).  y may equal x (in place) but must not overlap it
+ * otherwise.  D even, <= 256; H * D <= 2^28 (RA_ERR_SHAPE otherwise);
  * pos_offset >= 0; base > 0; pointers aligned to their element size.  The angle is reduced in fp64,
  * the rotation is fp32, the result rounds to the dtype.  Asynchronous on `stream`; returns RA_OK
  * or a validation error before anything is enqueued. */

@@ -131,6 +131,7 @@ extern "C" int ra_rope(const void* x, void* y, int64_t B, int64_t S, int64_t H, 
     const uintptr_t esize = dtype == RA_DTYPE_FP32 ? 4 : 2;
     if ((reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(y)) % esize) return RA_ERR_ALIGN;
     if (B * S * H == 0) return RA_OK;
+    if (H * D > (int64_t(1) << 28)) return RA_ERR_SHAPE;  // per-token element counts are int in the kernel
     ra::RopeArgs A{};
     A.pairs = (int)(D / 2);
     for (int p = 0; p < A.pairs; ++p) A.theta[p] = std::pow(base, -2.0 * p / (double)D);

@@ -94,6 +94,7 @@ def test_backward_rope_and_varlen_validate_before_any_cuda_call():
     assert lib.ra_rope(FAKE, FAKE, 1, 4, 1, 3, 0, 10000.0, 0, None) == -1
     assert lib.ra_rope(FAKE, FAKE, 1, 4, 1, 4, -1, 10000.0, 0, None) == -1
     assert lib.ra_rope(FAKE + 2, FAKE, 1, 4, 1, 4, 0, 10000.0, 0, None) == -3
+    assert lib.ra_rope(FAKE, FAKE, 1, 4, 1 << 21, 256, 0, 10000.0, 0, None) == -2  # H * D above 2^28
     # ra_forward_varlen: a length not divisible by n_ring, zigzag, cu[0] != 0
     cu = np.array([0, 50, 100], dtype=np.int64)
     assert lib.ra_forward_varlen(FAKE, FAKE, FAKE, FAKE, FAKE, cu.ctypes.data, 2, 1, 128, 4, 1, 0, None) == -2
