@@ -196,6 +196,18 @@ def oracle_sample(q, k, v, causal, rows_per_head, seed_base=7000):
     return flops, dt, threads, rows.size
 
 
+def oracle_single_thread(q, k, v, causal, n_rows, seed=7000):
+    """The same oracle on one host thread: `n_rows` uniformly drawn query rows of head 0."""
+    import oracle  # test-side fp64 reference: only this CPU-baseline leg runs it
+    B, S, H, D = q.shape
+    rows = np.sort(np.random.default_rng(seed).choice(S, n_rows, replace=False))
+    q0, k0, v0 = (t[:, :, :1].contiguous() for t in (q, k, v))
+    flops = B * sum(4.0 * D * ((r + 1) if causal else S) for r in rows)
+    t0 = time.perf_counter()
+    oracle.attention(q0, k0, v0, causal, rows=rows, threads=1)
+    return flops, time.perf_counter() - t0
+
+
 def run_reference(args, w):
     """Reference arm: the fp64 oracle, as it stands, on the host cores (rank 0 only)."""
     world, rank, _ = dist_env()
@@ -506,6 +518,11 @@ def run_ours(args, w):
         cpu = {"value": f / dt / 1e12, "unit": UNIT, "cores": threads, "kind": "oracle",
                "sample": f"{args.cpu_rows} query rows per head x {H} heads of {w.name} ({mask_word(args)}), "
                          f"{f:.3e} flops in {dt:.1f} s"}
+        if args.cpu_rows_single > 0:
+            f1, dt1 = oracle_single_thread(qc, kc, vc, causal, min(args.cpu_rows_single, w.S))
+            cpu["single_thread"] = {"value": f1 / dt1 / 1e12, "unit": UNIT, "cores": 1,
+                                    "sample": f"{min(args.cpu_rows_single, w.S)} query rows of head 0 of "
+                                              f"{w.name} ({mask_word(args)}), {f1:.3e} flops in {dt1:.1f} s"}
 
     # our kernels per step: the zigzag permute (striped and contiguous are read in place) and the
     # attention launch(es) -- per-step: N attention launches and N - 1 merges (2 kernels each,
@@ -557,6 +574,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-hbm-kernels", action="store_true")
     ap.add_argument("--cpu-rows", type=int, default=256, help="oracle rows per head for cpu_baseline")
+    ap.add_argument("--cpu-rows-single", type=int, default=64,
+                    help="oracle rows of one head for cpu_baseline's single-thread rate (0: skip)")
     ap.add_argument("--ref-rows", type=int, default=64, help="oracle rows per head per reference step")
     ap.add_argument("--traffic-bytes", type=float, default=None,
                     help="DRAM bytes per attention launch from an ncu capture of this kernel")
