@@ -231,9 +231,11 @@ RA_API int ra_backward_ex(const void* q, const void* k, const void* v, const voi
  * fused tensor-core kernel.
  *   q, k, v, out: [S_total, H, D] bf16 (batch 1), natural order; lse: [H, S_total] fp32, natural log.
  *   cu_seqlens: HOST array of n_seqs + 1 int64 offsets, cu[0] = 0, non-decreasing, cu[n_seqs] =
- *     S_total; every length a multiple of n_ring (RA_ERR_SHAPE otherwise); empty sequences allowed.
- *   layout: contiguous or striped (zigzag: RA_ERR_UNSUPPORTED); D in {64, 128}; sm_100; q, k, v, out
- *   16-byte aligned.  Scratch (work list, sequence table, counter) is allocated stream-ordered.
+ *     S_total; every length a multiple of n_ring, of 2 n_ring for zigzag (RA_ERR_SHAPE otherwise);
+ *     empty sequences allowed.
+ *   layout: contiguous, striped or zigzag, applied inside each sequence; D in {64, 128}; sm_100;
+ *   q, k, v, out 16-byte aligned.  Scratch (work list, sequence table, counter; for zigzag also
+ *   shard-major copies of q, k, v, 3 x S_total*H*D bf16) is allocated stream-ordered.
  *   Asynchronous on `stream`; bounded waits report through ra_get_device_status. */
 RA_API int ra_forward_varlen(const void* q, const void* k, const void* v, void* out, float* lse,
                              const int64_t* cu_seqlens, int n_seqs, int64_t H, int64_t D, int n_ring,

@@ -277,8 +277,8 @@ def backward(q, k, v, out, lse, dout, n_ring, causal=True, layout="contiguous", 
 def forward_varlen(q, k, v, cu_seqlens, n_ring, causal=True, layout="contiguous", *, out=None, lse=None,
                    stream=None):
     """ra_forward_varlen: attention over sequences packed on the token axis of q, k, v [S_total, H, D]
-    (bf16); cu_seqlens: n_seqs + 1 offsets (a host sequence of ints).  Returns (out [S_total, H, D],
-    lse [H, S_total])."""
+    (bf16); cu_seqlens: n_seqs + 1 offsets (a host sequence of ints); layout "contiguous", "striped"
+    or "zigzag" inside each sequence.  Returns (out [S_total, H, D], lse [H, S_total])."""
     torch = _torch()
     import numpy as np
     _check_cuda(q, k, v)

@@ -8,7 +8,9 @@
 // different lengths is the challenge; one list over every sequence lets the persistent kernel's
 // dynamic scheduler balance it).  The kernel reads the packed tensors in place through TMA maps over
 // the whole packed axis; rows past a sequence's end that a tile box still covers are masked by the
-// per-row key counts of that sequence.
+// per-row key counts of that sequence.  For the zigzag layout each sequence is first gathered into its
+// own shard-major order (shard i's tokens at sequence start + i * S_loc), which the kernel addresses
+// like the contiguous layout while it masks, and places its output, by the zigzag positions.
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -38,22 +40,54 @@ struct Item {
     int64_t cost;
 };
 
+constexpr int kRowsPerBlock = 8;  // one warp per token row
+
+struct PackArgs {
+    const uint4* src[3];
+    uint4* dst[3];
+};
+
+// Gather each packed sequence of q, k, v (grid.y) into its shard-major order: destination token t of
+// sequence s (first token base_s, length len_s, S_loc = len_s / N) is local token a = u mod S_loc of
+// shard i = u / S_loc, u = t - base_s, and comes from token base_s + g(i, a) of the source.  One warp
+// copies one token row (row_vecs 16-byte vectors); HBM-bound, each row read once and written once.
+__global__ void __launch_bounds__(256) pack_shard_major(PackArgs args, const int2* __restrict__ seqs, int n_seqs,
+                                                        int64_t S_total, int N, int kind, int64_t row_vecs) {
+    const int tensor = blockIdx.y;
+    const int64_t t = (int64_t)blockIdx.x * kRowsPerBlock + (threadIdx.x >> 5);
+    if (t >= S_total) return;
+    // the sequence holding t: the last entry whose first token is <= t (starts are non-decreasing;
+    // an empty sequence shares its start with the next entry, so it is never the last such entry)
+    int lo = 0, hi = n_seqs - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (seqs[mid].y <= t) lo = mid;
+        else hi = mid - 1;
+    }
+    const int64_t len = seqs[lo].x, base = seqs[lo].y;
+    const int64_t S_loc = len / N, u = t - base;
+    const ra::Layout L{len, N, S_loc, kind};
+    const int64_t src_row = base + ra::global_position(L, u / S_loc, u % S_loc);
+    const uint4* __restrict__ s = args.src[tensor] + src_row * row_vecs;
+    uint4* __restrict__ d = args.dst[tensor] + t * row_vecs;
+    for (int64_t c = threadIdx.x & 31; c < row_vecs; c += 32) d[c] = __ldcs(s + c);
+}
+
 }  // namespace
 
 extern "C" int ra_forward_varlen(const void* q, const void* k, const void* v, void* out, float* lse,
                                  const int64_t* cu_seqlens, int n_seqs, int64_t H, int64_t D, int n_ring,
                                  int causal, int layout, void* stream_handle) {
     if (!q || !k || !v || !out || !lse || !cu_seqlens || n_seqs < 1 || H < 1 || n_ring < 1) return RA_ERR_INVALID_ARG;
-    if (layout != RA_LAYOUT_CONTIGUOUS && layout != RA_LAYOUT_STRIPED) {
-        ra::host_set_error("ra_forward_varlen: contiguous or striped layout");
-        return RA_ERR_UNSUPPORTED;
-    }
+    if (layout != RA_LAYOUT_CONTIGUOUS && layout != RA_LAYOUT_STRIPED && layout != RA_LAYOUT_ZIGZAG)
+        return RA_ERR_INVALID_ARG;
     if (D != 64 && D != 128) return RA_ERR_UNSUPPORTED;
     if (cu_seqlens[0] != 0) return RA_ERR_INVALID_ARG;
+    const int64_t unit = layout == RA_LAYOUT_ZIGZAG ? 2 * (int64_t)n_ring : n_ring;  // zigzag: 2N chunks
     for (int s = 0; s < n_seqs; ++s) {
         const int64_t len = cu_seqlens[s + 1] - cu_seqlens[s];
         if (len < 0) return RA_ERR_INVALID_ARG;
-        if (len % n_ring) return RA_ERR_SHAPE;
+        if (len % unit) return RA_ERR_SHAPE;
     }
     const int64_t S_total = cu_seqlens[n_seqs];
     if (S_total >= (int64_t(1) << 31) || H * D * 2 % 16) return RA_ERR_SHAPE;
@@ -93,8 +127,11 @@ extern "C" int ra_forward_varlen(const void* q, const void* k, const void* v, vo
     if (list.size() > (size_t)INT32_MAX) return RA_ERR_SHAPE;
 
     cudaStream_t stream = static_cast<cudaStream_t>(stream_handle);
+    const bool zigzag = layout == RA_LAYOUT_ZIGZAG;
+    const size_t tensor_bytes = align256((size_t)S_total * (size_t)H * (size_t)D * 2);
     const size_t off_seqs = 256, off_items = off_seqs + align256(seqs.size() * sizeof(int2));
-    const size_t bytes = off_items + align256(list.size() * sizeof(int4));
+    const size_t off_perm = off_items + align256(list.size() * sizeof(int4));  // zigzag: q, k, v copies
+    const size_t bytes = off_perm + (zigzag ? 3 * tensor_bytes : 0);
     uint8_t* ws = nullptr;
     cudaError_t e = cudaMallocAsync(reinterpret_cast<void**>(&ws), bytes, stream);
     if (e != cudaSuccess) return ra::host_cuda_fail(e, "cudaMallocAsync(varlen scratch)");
@@ -111,14 +148,33 @@ extern "C" int ra_forward_varlen(const void* q, const void* k, const void* v, vo
                              stream)) != cudaSuccess)
         return finish(ra::host_cuda_fail(e, "varlen work list upload"));
 
-    // TMA maps over the packed axis: contiguous (D, H, S_total, 1, 1); striped (D, H, S_total / N, N, 1)
-    // with token = a' * N + i (every sequence starts on a multiple of N)
+    // zigzag: gather every sequence into its shard-major order; the kernel then reads the copies with
+    // contiguous addressing (sequence start + i * S_loc + a)
+    const void *qs = q, *ks = k, *vs = v;
+    if (zigzag) {
+        PackArgs pa{};
+        const void* src[3] = {q, k, v};
+        for (int x = 0; x < 3; ++x) {
+            pa.src[x] = static_cast<const uint4*>(src[x]);
+            pa.dst[x] = reinterpret_cast<uint4*>(ws + off_perm + x * tensor_bytes);
+        }
+        const dim3 grid((unsigned)((S_total + kRowsPerBlock - 1) / kRowsPerBlock), 3);
+        pack_shard_major<<<grid, 256, 0, stream>>>(pa, reinterpret_cast<const int2*>(ws + off_seqs), n_seqs,
+                                                   S_total, n_ring, layout, H * D * 2 / 16);
+        if ((e = cudaGetLastError()) != cudaSuccess) return finish(ra::host_cuda_fail(e, "varlen permute launch"));
+        qs = pa.dst[0];
+        ks = pa.dst[1];
+        vs = pa.dst[2];
+    }
+
+    // TMA maps over the packed axis: contiguous and zigzag copies (D, H, S_total, 1, 1); striped
+    // (D, H, S_total / N, N, 1) with token = a' * N + i (every sequence starts on a multiple of N)
     const bool striped = layout == RA_LAYOUT_STRIPED;
     const ra::Layout Lmap = striped ? ra::Layout{S_total, N, S_total / N, layout} : ra::Layout{S_total, 1, S_total, layout};
     ra::TcLaunch t{};
-    if ((rc = ra::host_encode_qkv_map(&t.tm_q, q, 1, Lmap, H, D, striped)) != RA_OK ||
-        (rc = ra::host_encode_qkv_map(&t.tm_k, k, 1, Lmap, H, D, striped)) != RA_OK ||
-        (rc = ra::host_encode_qkv_map(&t.tm_v, v, 1, Lmap, H, D, striped)) != RA_OK)
+    if ((rc = ra::host_encode_qkv_map(&t.tm_q, qs, 1, Lmap, H, D, striped)) != RA_OK ||
+        (rc = ra::host_encode_qkv_map(&t.tm_k, ks, 1, Lmap, H, D, striped)) != RA_OK ||
+        (rc = ra::host_encode_qkv_map(&t.tm_v, vs, 1, Lmap, H, D, striped)) != RA_OK)
         return finish(rc);
     t.items = reinterpret_cast<const int4*>(ws + off_items);
     t.n_items = (int)list.size();

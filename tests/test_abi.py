@@ -95,10 +95,13 @@ def test_backward_rope_and_varlen_validate_before_any_cuda_call():
     assert lib.ra_rope(FAKE, FAKE, 1, 4, 1, 4, -1, 10000.0, 0, None) == -1
     assert lib.ra_rope(FAKE + 2, FAKE, 1, 4, 1, 4, 0, 10000.0, 0, None) == -3
     assert lib.ra_rope(FAKE, FAKE, 1, 4, 1 << 21, 256, 0, 10000.0, 0, None) == -2  # H * D above 2^28
-    # ra_forward_varlen: a length not divisible by n_ring, zigzag, cu[0] != 0
+    # ra_forward_varlen: a length not divisible by n_ring; under zigzag one not divisible by 2 n_ring;
+    # an unknown layout; cu[0] != 0
     cu = np.array([0, 50, 100], dtype=np.int64)
     assert lib.ra_forward_varlen(FAKE, FAKE, FAKE, FAKE, FAKE, cu.ctypes.data, 2, 1, 128, 4, 1, 0, None) == -2
+    cu = np.array([0, 64, 132], dtype=np.int64)
+    assert lib.ra_forward_varlen(FAKE, FAKE, FAKE, FAKE, FAKE, cu.ctypes.data, 2, 1, 128, 4, 1, 2, None) == -2
     cu = np.array([0, 64, 128], dtype=np.int64)
-    assert lib.ra_forward_varlen(FAKE, FAKE, FAKE, FAKE, FAKE, cu.ctypes.data, 2, 1, 128, 4, 1, 2, None) == -4
+    assert lib.ra_forward_varlen(FAKE, FAKE, FAKE, FAKE, FAKE, cu.ctypes.data, 2, 1, 128, 4, 1, 3, None) == -1
     cu = np.array([4, 64, 128], dtype=np.int64)
     assert lib.ra_forward_varlen(FAKE, FAKE, FAKE, FAKE, FAKE, cu.ctypes.data, 2, 1, 128, 4, 1, 0, None) == -1

@@ -1,8 +1,6 @@
 """Checks of the Python binding's own argument handling that need no GPU: caller-supplied output
 tensors are matched against what the kernels write before any launch, and library messages are
 attached to errors only when the failing call produced them."""
-import ctypes
-
 import numpy as np
 import pytest
 import torch
@@ -58,22 +56,27 @@ def test_plan_tiles_rejects_zero_ring_and_tile():
         ra.plan_tiles(64, 4, "contiguous", True, 0)
 
 
+def _backward_head_dim_256():
+    """ra_backward_ex with D = 256: refused with RA_ERR_UNSUPPORTED and a message, before any device call."""
+    return ra.lib().ra_backward_ex(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1, 2, 64, 256, 4, 1, 0,
+                                   1, 0, 0, 0, None)
+
+
 def test_error_detail_comes_only_from_the_failing_call():
     lib = ra.lib()
-    cu = np.array([0, 64, 128], dtype=np.int64)
     ra._clear_error()
-    rc = lib.ra_forward_varlen(FAKE, FAKE, FAKE, FAKE, FAKE, cu.ctypes.data, 2, 1, 128, 4, 1, 2, None)
-    with pytest.raises(ra.RAError, match="contiguous or striped"):
-        ra._check(rc, "ra_forward_varlen")
+    rc = _backward_head_dim_256()
+    with pytest.raises(ra.RAError, match="head dims above 128"):
+        ra._check(rc, "ra_backward_ex")
     # the same failure again still carries its message
     ra._clear_error()
-    rc = lib.ra_forward_varlen(FAKE, FAKE, FAKE, FAKE, FAKE, cu.ctypes.data, 2, 1, 128, 4, 1, 2, None)
-    with pytest.raises(ra.RAError, match="contiguous or striped"):
-        ra._check(rc, "ra_forward_varlen")
+    rc = _backward_head_dim_256()
+    with pytest.raises(ra.RAError, match="head dims above 128"):
+        ra._check(rc, "ra_backward_ex")
     # a later failure that records no message does not carry the earlier one
     ra._clear_error()
     assert ra._last_error() == ""
     rc = lib.ra_rope(FAKE, FAKE, 1, 4, 1, 3, 0, 10000.0, 0, None)
     with pytest.raises(ra.RAError) as e:
         ra._check(rc, "ra_rope")
-    assert e.value.code == -1 and "contiguous" not in str(e.value)
+    assert e.value.code == -1 and "head dims" not in str(e.value)

@@ -29,25 +29,30 @@ def run(lengths, H, D, N, causal, layout, seed):
     assert lerr.max() <= 1e-3, lerr.max()
 
 
-@pytest.mark.parametrize("layout", ["contiguous", "striped"])
+@pytest.mark.parametrize("layout", ["contiguous", "striped", "zigzag"])
 @pytest.mark.parametrize("causal", [False, True])
 def test_mixed_lengths(layout, causal):
     run([1024, 256, 4096, 512, 64], 2, 128, 4, causal, layout, seed=1)
 
 
-@pytest.mark.parametrize("layout", ["contiguous", "striped"])
+@pytest.mark.parametrize("layout", ["contiguous", "striped", "zigzag"])
 def test_short_ragged_and_empty_sequences(layout):
-    run([8, 0, 600, 24, 1200, 4], 2, 64, 4, True, layout, seed=2)
+    run([8, 0, 600, 24, 1200, 8], 2, 64, 4, True, layout, seed=2)
+
+
+def test_zigzag_one_long_among_many_short():
+    run([64] * 20 + [8192] + [48] * 10 + [0], 1, 128, 8, True, "zigzag", seed=5)
 
 
 def test_one_long_among_many_short():
     run([64] * 30 + [8192] + [128] * 10, 1, 128, 8, True, "striped", seed=3)
 
 
-def test_single_sequence_equals_the_batch_call():
+@pytest.mark.parametrize("layout", ["striped", "zigzag"])
+def test_single_sequence_equals_the_batch_call(layout):
     q, k, v = inputs.make_qkv(1, 2048, 2, 128, dtype=torch.bfloat16, device="cuda", seed=4)
-    a, la = ra.forward(q, k, v, 4, True, "striped")
-    b, lb = ra.forward_varlen(q[0], k[0], v[0], [0, 2048], 4, True, "striped")
+    a, la = ra.forward(q, k, v, 4, True, layout)
+    b, lb = ra.forward_varlen(q[0], k[0], v[0], [0, 2048], 4, True, layout)
     torch.cuda.synchronize()
     assert torch.equal(a[0], b) and torch.equal(la[0], lb)
 
@@ -56,5 +61,5 @@ def test_varlen_rejects_bad_arguments():
     q = torch.zeros(100, 1, 128, device="cuda", dtype=torch.bfloat16)
     with pytest.raises(ra.RAError):  # length not a multiple of n_ring
         ra.forward_varlen(q, q, q, [0, 50, 100], 4, True)
-    with pytest.raises(ra.RAError):  # zigzag is not offered
-        ra.forward_varlen(q, q, q, [0, 100], 4, True, "zigzag")
+    with pytest.raises(ra.RAError):  # zigzag needs lengths divisible by 2 n_ring
+        ra.forward_varlen(q, q, q, [0, 4, 100], 4, True, "zigzag")
