@@ -530,7 +530,9 @@ def run_ours(args, w):
     launches_per_step = (1 if args.layout == "zigzag" else 0) + (
         1 if args.variant in ("fused", "auto") else N + 2 * (N - 2) + 1)
     if args.backward:
-        launches_per_step = 3  # Delta, dq, dk/dv
+        # Delta, dq, dk/dv; the tensor-core kernels read zigzag from one shard-major permute launch
+        tc_bwd = args.bwd_kernel == "tc" or (args.bwd_kernel == "auto" and args.dtype == "bf16" and D in (64, 128))
+        launches_per_step = 3 + (1 if args.layout == "zigzag" and tc_bwd else 0)
     line = {
         "metric": metric_of(args), "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
