@@ -213,7 +213,8 @@ def run_reference(args, w):
     world, rank, _ = dist_env()
     if rank != 0:
         return
-    q, k, v = inputs.make_qkv(w.B, w.S, w.H, w.D, torch.bfloat16, "cpu", w.seed)
+    q, k, v = inputs.make_qkv(w.B, w.S, w.H, w.D, torch.float32 if args.dtype == "fp32" else torch.bfloat16,
+                              "cpu", w.seed)
     rows_per_head = args.ref_rows
     causal = causal_of(args)
     for _ in range(args.warmup):
@@ -586,6 +587,9 @@ def main():
         ap.error("--backward / --varlen runs time the device call only: add --no-e2e --no-cpu-baseline")
     if args.backward and args.varlen:
         ap.error("--backward and --varlen are separate runs")
+    if args.impl == "reference" and (args.backward or args.varlen):
+        ap.error("--impl reference times the oracle of the batch forward pass; --backward and --varlen "
+                 "have no reference arm")
     if args.kernel == "tc" and args.dtype == "fp32":
         ap.error("the tensor-core kernel takes bf16 inputs; fp32 runs on --kernel simt")
     w = inputs.WORKLOADS[args.workload]
