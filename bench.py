@@ -345,14 +345,12 @@ def run_ours(args, w):
         for n in lengths:
             cu.append(cu[-1] + n)
         lse_v = torch.empty((H, S), dtype=torch.float32, device=dev)
+        ws_v = torch.empty(ra.varlen_workspace_size(cu, H, D, N, args.layout), dtype=torch.uint8, device=dev)
         flops = sum(attention_flops(1, H, n, D, causal) for n in lengths)
 
-        def step(ev=None):
-            if ev is not None:
-                ev[0].record(stream)
-            ra.forward_varlen(q[0], k[0], v[0], cu, N, causal, args.layout, out=out[0], lse=lse_v, stream=stream)
-            if ev is not None:
-                ev[1].record(stream)
+        def step(ev=None):  # ev: recorded by the library around the attention launch
+            ra.forward_varlen(q[0], k[0], v[0], cu, N, causal, args.layout, out=out[0], lse=lse_v, workspace=ws_v,
+                              stream=stream, events=ev)
 
     if args.backward:
         # one forward pass outside the timed region supplies out and lse; a step is one ra_backward
@@ -505,7 +503,7 @@ def run_ours(args, w):
             "frac_of_burst_peak": achieved / peaks["bf16_tflops"],
             "kernel": ("bwd_dq_tc_kernel + bwd_dkv_tc_kernel (tcgen05), timed as one ra_backward call"
                        if args.backward else
-                       "attn_tc_kernel<128, varlen> (fused ring, tcgen05), timed as one ra_forward_varlen call"
+                       "attn_tc_kernel<128, varlen> (fused ring, tcgen05)"
                        if args.varlen else "attn_tc_kernel<128> (fused ring, tcgen05)"),
             "kernel_ms": k_ms,
             "algorithmic_flops_per_launch": flops,

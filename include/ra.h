@@ -241,6 +241,23 @@ RA_API int ra_forward_varlen(const void* q, const void* k, const void* v, void* 
                              const int64_t* cu_seqlens, int n_seqs, int64_t H, int64_t D, int n_ring,
                              int causal, int layout, void* stream);
 
+/* ra_forward_varlen_ex: ra_forward_varlen with options (opt may be NULL for the defaults).
+ *   workspace / workspace_bytes: caller scratch of at least ra_varlen_workspace_size bytes, 256-byte
+ *     aligned (RA_ERR_ALIGN otherwise; RA_ERR_NO_WORKSPACE if smaller); NULL: allocated and freed
+ *     stream-ordered as ra_forward_varlen does.  A caller that keeps the buffer between calls saves
+ *     the allocation, which for zigzag holds the 3 x S_total*H*D bf16 shard-major copies.
+ *   timeout_ns, debug: as for ra_forward_ex.  attn_events: recorded right before and right after the
+ *     attention launch (after the zigzag gather).
+ *   variant must be AUTO or FUSED and kernel AUTO or TC (RA_ERR_UNSUPPORTED otherwise). */
+RA_API int ra_forward_varlen_ex(const void* q, const void* k, const void* v, void* out, float* lse,
+                                const int64_t* cu_seqlens, int n_seqs, int64_t H, int64_t D, int n_ring,
+                                int causal, int layout, void* stream, const ra_options* opt);
+
+/* ra_varlen_workspace_size: scratch bytes ra_forward_varlen_ex needs for these packed sequences,
+ * written to *bytes.  Host only; the arguments are validated as for ra_forward_varlen. */
+RA_API int ra_varlen_workspace_size(const int64_t* cu_seqlens, int n_seqs, int64_t H, int64_t D, int n_ring,
+                                    int layout, size_t* bytes);
+
 /* ra_rope: rotary position embedding with global token positions (troisinh.com "Ring Attention",
  * "RoPE va Position Embedding": a token must be rotated by the angle m theta of its own position m
  * wherever its block travels on the ring).  x, y: [B, S, H, D] in natural token order, dtype fp32 or

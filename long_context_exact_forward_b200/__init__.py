@@ -9,7 +9,8 @@ device is not a CUDA device the calls raise.
 Entry points (same names as the C ABI):
     forward(q, k, v, n_ring, causal, layout, ...)   -> (out, lse)      ra_forward_ex
     forward_noalloc(q, k, v, n_ring, causal, layout) -> (out, lse)      ra_forward_noalloc
-    forward_varlen(q, k, v, cu_seqlens, n_ring, ...) -> (out, lse)      ra_forward_varlen
+    forward_varlen(q, k, v, cu_seqlens, n_ring, ...) -> (out, lse)      ra_forward_varlen_ex
+    varlen_workspace_size(cu_seqlens, H, D, ...)     -> int             ra_varlen_workspace_size
     backward(q, k, v, out, lse, dout, n_ring, ...)   -> (dq, dk, dv)    ra_backward_ex
     rope(x, pos_offset, base)                        -> tensor          ra_rope
     workspace_size(...)                              -> int             ra_workspace_size
@@ -86,6 +87,9 @@ def lib():
         L.ra_backward.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i64, i64, i64, i64, ci, ci, ci,
                                   ci, vp]
         L.ra_forward_varlen.argtypes = [vp, vp, vp, vp, vp, vp, ci, i64, i64, ci, ci, ci, vp]
+        L.ra_forward_varlen_ex.argtypes = [vp, vp, vp, vp, vp, vp, ci, i64, i64, ci, ci, ci, vp,
+                                           ctypes.POINTER(Options)]
+        L.ra_varlen_workspace_size.argtypes = [vp, ci, i64, i64, ci, ci, ctypes.POINTER(ctypes.c_size_t)]
         L.ra_rope.argtypes = [vp, vp, i64, i64, i64, i64, i64, ctypes.c_double, ci, vp]
         L.ra_backward_ex.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i64, i64, i64, i64, ci, ci, ci,
                                      ci, ci, ctypes.c_uint64, ci, vp]
@@ -101,7 +105,8 @@ def lib():
         L.ra_clear_last_error.restype = None
         for name in ("ra_forward", "ra_forward_ex", "ra_forward_noalloc", "ra_workspace_size", "ra_permute",
                      "ra_unpermute", "ra_merge_partials", "ra_layout_positions", "ra_plan_tiles",
-                     "ra_plan_items", "ra_get_device_status", "ra_backward", "ra_backward_ex", "ra_rope", "ra_forward_varlen"):
+                     "ra_plan_items", "ra_get_device_status", "ra_backward", "ra_backward_ex", "ra_rope", "ra_forward_varlen",
+                     "ra_forward_varlen_ex", "ra_varlen_workspace_size"):
             getattr(L, name).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -274,32 +279,71 @@ def backward(q, k, v, out, lse, dout, n_ring, causal=True, layout="contiguous", 
     return dq, dk, dv
 
 
+def _cu_array(cu_seqlens):
+    cu = np.ascontiguousarray(np.asarray(cu_seqlens, dtype=np.int64))
+    if cu.ndim != 1 or cu.size < 2:
+        raise ValueError("cu_seqlens must hold n_seqs + 1 offsets")
+    return cu
+
+
+def varlen_workspace_size(cu_seqlens, H, D, n_ring, layout="contiguous"):
+    """Bytes of scratch forward_varlen needs for these packed sequences (ra_varlen_workspace_size)."""
+    cu = _cu_array(cu_seqlens)
+    n = ctypes.c_size_t(0)
+    _clear_error()
+    _check(lib().ra_varlen_workspace_size(cu.ctypes.data, int(cu.size - 1), H, D, int(n_ring), LAYOUTS[layout],
+                                          ctypes.byref(n)), "ra_varlen_workspace_size")
+    return n.value
+
+
 def forward_varlen(q, k, v, cu_seqlens, n_ring, causal=True, layout="contiguous", *, out=None, lse=None,
-                   stream=None):
-    """ra_forward_varlen: attention over sequences packed on the token axis of q, k, v [S_total, H, D]
+                   workspace=None, stream=None, events=None, timeout_ns=0, debug=0):
+    """ra_forward_varlen_ex: attention over sequences packed on the token axis of q, k, v [S_total, H, D]
     (bf16); cu_seqlens: n_seqs + 1 offsets (a host sequence of ints); layout "contiguous", "striped"
-    or "zigzag" inside each sequence.  Returns (out [S_total, H, D], lse [H, S_total])."""
+    or "zigzag" inside each sequence.  Returns (out [S_total, H, D], lse [H, S_total]).
+
+    `workspace` is an optional uint8 CUDA tensor of at least varlen_workspace_size(...) bytes; without
+    it the scratch comes from torch's caching allocator on the call's stream, so repeated calls do
+    not allocate device memory anew.  `events`: an optional pair of torch.cuda.Event recorded around
+    the attention launch."""
     torch = _torch()
-    import numpy as np
     _check_cuda(q, k, v)
     if q.dim() != 3 or q.shape != k.shape or q.shape != v.shape:
         raise ValueError("q, k, v must all be [S_total, H, D]")
     if q.dtype != torch.bfloat16 or k.dtype != q.dtype or v.dtype != q.dtype:
         raise TypeError("forward_varlen takes bf16 q, k, v")
     S, H, D = q.shape
-    cu = np.ascontiguousarray(np.asarray(cu_seqlens, dtype=np.int64))
-    if cu.ndim != 1 or cu.size < 2 or cu[-1] != S:
-        raise ValueError("cu_seqlens must hold n_seqs + 1 offsets ending at S_total")
+    cu = _cu_array(cu_seqlens)
+    if cu[-1] != S:
+        raise ValueError("cu_seqlens must end at S_total")
     out = torch.empty_like(q) if out is None else out
     lse = torch.empty((H, S), dtype=torch.float32, device=q.device) if lse is None else lse
     _check_out(out, q.shape, q.dtype, "out", q)
     _check_out(lse, (H, S), torch.float32, "lse", q)
+    if workspace is None:
+        n = varlen_workspace_size(cu, H, D, n_ring, layout)
+        with torch.cuda.device(q.device):
+            workspace = torch.empty(n, dtype=torch.uint8, device=q.device)
+        if stream is not None:  # the scratch must outlive the work enqueued on `stream`
+            workspace.record_stream(stream)
+    _check_cuda(workspace)
+    opt = Options()
+    opt.workspace = workspace.data_ptr()
+    opt.workspace_bytes = workspace.numel() * workspace.element_size()
+    opt.timeout_ns = int(timeout_ns)
+    opt.debug = int(debug)
+    if events is not None:
+        for ev in events:  # torch creates the CUDA event lazily, on first record
+            if ev.cuda_event == 0:
+                ev.record(stream if stream is not None else torch.cuda.current_stream())
+        opt.attn_events[0] = events[0].cuda_event
+        opt.attn_events[1] = events[1].cuda_event
     _clear_error()
     with torch.cuda.device(q.device):
-        rc = lib().ra_forward_varlen(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
-                                     cu.ctypes.data, int(cu.size - 1), H, D, int(n_ring), int(bool(causal)),
-                                     LAYOUTS[layout], _stream_handle(stream))
-    _check(rc, "ra_forward_varlen")
+        rc = lib().ra_forward_varlen_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
+                                        cu.ctypes.data, int(cu.size - 1), H, D, int(n_ring), int(bool(causal)),
+                                        LAYOUTS[layout], _stream_handle(stream), ctypes.byref(opt))
+    _check(rc, "ra_forward_varlen_ex")
     return out, lse
 
 

@@ -75,10 +75,13 @@ __global__ void __launch_bounds__(256) pack_shard_major(PackArgs args, const int
 
 }  // namespace
 
-extern "C" int ra_forward_varlen(const void* q, const void* k, const void* v, void* out, float* lse,
-                                 const int64_t* cu_seqlens, int n_seqs, int64_t H, int64_t D, int n_ring,
-                                 int causal, int layout, void* stream_handle) {
-    if (!q || !k || !v || !out || !lse || !cu_seqlens || n_seqs < 1 || H < 1 || n_ring < 1) return RA_ERR_INVALID_ARG;
+namespace {
+
+// Host validation shared by every entry point (nothing touches the device).  On success *S_total is
+// the packed length.
+int check_packed(const int64_t* cu_seqlens, int n_seqs, int64_t H, int64_t D, int n_ring, int layout,
+                 int64_t* S_total) {
+    if (!cu_seqlens || n_seqs < 1 || H < 1 || n_ring < 1) return RA_ERR_INVALID_ARG;
     if (layout != RA_LAYOUT_CONTIGUOUS && layout != RA_LAYOUT_STRIPED && layout != RA_LAYOUT_ZIGZAG)
         return RA_ERR_INVALID_ARG;
     if (D != 64 && D != 128) return RA_ERR_UNSUPPORTED;
@@ -89,14 +92,57 @@ extern "C" int ra_forward_varlen(const void* q, const void* k, const void* v, vo
         if (len < 0) return RA_ERR_INVALID_ARG;
         if (len % unit) return RA_ERR_SHAPE;
     }
-    const int64_t S_total = cu_seqlens[n_seqs];
-    if (S_total >= (int64_t(1) << 31) || H * D * 2 % 16) return RA_ERR_SHAPE;
+    *S_total = cu_seqlens[n_seqs];
+    if (*S_total >= (int64_t(1) << 31) || H * D * 2 % 16) return RA_ERR_SHAPE;
+    return RA_OK;
+}
+
+// Scratch of one call, in this order: work counter (256 B), sequence table {length, first token},
+// work list (int4 per item), and for zigzag the shard-major copies of q, k, v; every part 256-byte
+// aligned.  The item count is known before the list is built: per non-empty sequence,
+// H * N * ceil(S_loc / 256) items.
+struct Scratch {
+    size_t off_seqs, off_items, off_perm, tensor_bytes, bytes;
+    int64_t n_items;
+};
+
+Scratch scratch_layout(const int64_t* cu_seqlens, int n_seqs, int64_t H, int64_t D, int n_ring, int layout,
+                       int64_t S_total) {
+    Scratch w{};
+    for (int s = 0; s < n_seqs; ++s) {
+        const int64_t S_loc = (cu_seqlens[s + 1] - cu_seqlens[s]) / n_ring;
+        w.n_items += H * n_ring * ((S_loc + kPairRows - 1) / kPairRows);
+    }
+    w.tensor_bytes = align256((size_t)S_total * (size_t)H * (size_t)D * 2);
+    w.off_seqs = 256;
+    w.off_items = w.off_seqs + align256((size_t)n_seqs * sizeof(int2));
+    w.off_perm = w.off_items + align256((size_t)w.n_items * sizeof(int4));
+    w.bytes = w.off_perm + (layout == RA_LAYOUT_ZIGZAG ? 3 * w.tensor_bytes : 0);
+    return w;
+}
+
+// The forward pass over packed sequences.  ws == nullptr: the scratch is allocated and freed
+// stream-ordered here; otherwise ws holds at least scratch_layout(...).bytes.
+int varlen_forward(const void* q, const void* k, const void* v, void* out, float* lse, const int64_t* cu_seqlens,
+                   int n_seqs, int64_t H, int64_t D, int n_ring, int causal, int layout, cudaStream_t stream,
+                   uint8_t* ws_given, size_t ws_bytes, uint64_t timeout_ns, int debug, cudaEvent_t ev0,
+                   cudaEvent_t ev1) {
+    if (!q || !k || !v || !out || !lse) return RA_ERR_INVALID_ARG;
+    int64_t S_total = 0;
+    int rc = check_packed(cu_seqlens, n_seqs, H, D, n_ring, layout, &S_total);
+    if (rc != RA_OK) return rc;
     auto a16 = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; };
     if (!a16(q) || !a16(k) || !a16(v) || !a16(out) || (reinterpret_cast<uintptr_t>(lse) & 3u)) return RA_ERR_ALIGN;
+    const Scratch w = scratch_layout(cu_seqlens, n_seqs, H, D, n_ring, layout, S_total);
+    if (w.n_items > (int64_t)INT32_MAX) return RA_ERR_SHAPE;
+    if (ws_given) {
+        if (reinterpret_cast<uintptr_t>(ws_given) & 255u) return RA_ERR_ALIGN;
+        if (ws_bytes < w.bytes) return RA_ERR_NO_WORKSPACE;
+    }
     int sms = 0;
     bool sm100 = false;
     int* status = nullptr;
-    int rc = ra::host_device_facts(&sms, &sm100, &status);
+    rc = ra::host_device_facts(&sms, &sm100, &status);
     if (rc != RA_OK) return rc;
     if (!sm100) return RA_ERR_UNSUPPORTED;
     if (S_total == 0) return RA_OK;
@@ -104,6 +150,7 @@ extern "C" int ra_forward_varlen(const void* q, const void* k, const void* v, vo
     // work list: every (sequence, head, shard, pair), longest first (ties in list order)
     const int64_t N = n_ring;
     std::vector<Item> items;
+    items.reserve((size_t)w.n_items);
     std::vector<int2> seqs(n_seqs);
     for (int s = 0; s < n_seqs; ++s) {
         const int64_t len = cu_seqlens[s + 1] - cu_seqlens[s];
@@ -121,45 +168,47 @@ extern "C" int ra_forward_varlen(const void* q, const void* k, const void* v, vo
                 for (int64_t h = 0; h < H; ++h) items.push_back({make_int4(s, (int)h, (int)i, (int)p), cost});
             }
     }
+    if ((int64_t)items.size() != w.n_items) {  // the scratch was sized by the same count
+        ra::host_set_error("ra_forward_varlen: work list size mismatch");
+        return RA_ERR_INVALID_ARG;
+    }
     std::stable_sort(items.begin(), items.end(), [](const Item& a, const Item& b) { return a.cost > b.cost; });
     std::vector<int4> list(items.size());
     for (size_t t = 0; t < items.size(); ++t) list[t] = items[t].it;
-    if (list.size() > (size_t)INT32_MAX) return RA_ERR_SHAPE;
 
-    cudaStream_t stream = static_cast<cudaStream_t>(stream_handle);
-    const bool zigzag = layout == RA_LAYOUT_ZIGZAG;
-    const size_t tensor_bytes = align256((size_t)S_total * (size_t)H * (size_t)D * 2);
-    const size_t off_seqs = 256, off_items = off_seqs + align256(seqs.size() * sizeof(int2));
-    const size_t off_perm = off_items + align256(list.size() * sizeof(int4));  // zigzag: q, k, v copies
-    const size_t bytes = off_perm + (zigzag ? 3 * tensor_bytes : 0);
-    uint8_t* ws = nullptr;
-    cudaError_t e = cudaMallocAsync(reinterpret_cast<void**>(&ws), bytes, stream);
-    if (e != cudaSuccess) return ra::host_cuda_fail(e, "cudaMallocAsync(varlen scratch)");
+    uint8_t* ws = ws_given;
+    cudaError_t e = cudaSuccess;
+    if (!ws_given) {
+        e = cudaMallocAsync(reinterpret_cast<void**>(&ws), w.bytes, stream);
+        if (e != cudaSuccess) return ra::host_cuda_fail(e, "cudaMallocAsync(varlen scratch)");
+    }
     auto finish = [&](int r) {
+        if (ws_given) return r;
         const cudaError_t ef = cudaFreeAsync(ws, stream);
         if (r == RA_OK && ef != cudaSuccess) return ra::host_cuda_fail(ef, "cudaFreeAsync(varlen scratch)");
         return r;
     };
     // pageable sources: each copy returns once its data is staged, so the vectors may go out of scope
     if ((e = cudaMemsetAsync(ws, 0, sizeof(int), stream)) != cudaSuccess ||
-        (e = cudaMemcpyAsync(ws + off_seqs, seqs.data(), seqs.size() * sizeof(int2), cudaMemcpyHostToDevice,
+        (e = cudaMemcpyAsync(ws + w.off_seqs, seqs.data(), seqs.size() * sizeof(int2), cudaMemcpyHostToDevice,
                              stream)) != cudaSuccess ||
-        (e = cudaMemcpyAsync(ws + off_items, list.data(), list.size() * sizeof(int4), cudaMemcpyHostToDevice,
+        (e = cudaMemcpyAsync(ws + w.off_items, list.data(), list.size() * sizeof(int4), cudaMemcpyHostToDevice,
                              stream)) != cudaSuccess)
         return finish(ra::host_cuda_fail(e, "varlen work list upload"));
 
     // zigzag: gather every sequence into its shard-major order; the kernel then reads the copies with
     // contiguous addressing (sequence start + i * S_loc + a)
+    const bool zigzag = layout == RA_LAYOUT_ZIGZAG;
     const void *qs = q, *ks = k, *vs = v;
     if (zigzag) {
         PackArgs pa{};
         const void* src[3] = {q, k, v};
         for (int x = 0; x < 3; ++x) {
             pa.src[x] = static_cast<const uint4*>(src[x]);
-            pa.dst[x] = reinterpret_cast<uint4*>(ws + off_perm + x * tensor_bytes);
+            pa.dst[x] = reinterpret_cast<uint4*>(ws + w.off_perm + x * w.tensor_bytes);
         }
         const dim3 grid((unsigned)((S_total + kRowsPerBlock - 1) / kRowsPerBlock), 3);
-        pack_shard_major<<<grid, 256, 0, stream>>>(pa, reinterpret_cast<const int2*>(ws + off_seqs), n_seqs,
+        pack_shard_major<<<grid, 256, 0, stream>>>(pa, reinterpret_cast<const int2*>(ws + w.off_seqs), n_seqs,
                                                    S_total, n_ring, layout, H * D * 2 / 16);
         if ((e = cudaGetLastError()) != cudaSuccess) return finish(ra::host_cuda_fail(e, "varlen permute launch"));
         qs = pa.dst[0];
@@ -176,12 +225,12 @@ extern "C" int ra_forward_varlen(const void* q, const void* k, const void* v, vo
         (rc = ra::host_encode_qkv_map(&t.tm_k, ks, 1, Lmap, H, D, striped)) != RA_OK ||
         (rc = ra::host_encode_qkv_map(&t.tm_v, vs, 1, Lmap, H, D, striped)) != RA_OK)
         return finish(rc);
-    t.items = reinterpret_cast<const int4*>(ws + off_items);
+    t.items = reinterpret_cast<const int4*>(ws + w.off_items);
     t.n_items = (int)list.size();
     t.counter = reinterpret_cast<int*>(ws);
     t.grid = (int)std::min<int64_t>((int64_t)list.size(), sms);
-    t.timeout_ns = 2000000000ull;
-    t.debug = 0;
+    t.timeout_ns = timeout_ns ? timeout_ns : 2000000000ull;
+    t.debug = debug;
     t.status = status;
 
     ra::AttnArgs a{};
@@ -197,8 +246,43 @@ extern "C" int ra_forward_varlen(const void* q, const void* k, const void* v, vo
     a.out = out;
     a.lse = lse;
     a.scale = (float)(1.0 / std::sqrt((double)D));
-    a.seqs = reinterpret_cast<const int2*>(ws + off_seqs);
+    a.seqs = reinterpret_cast<const int2*>(ws + w.off_seqs);
     a.varlen_striped = striped ? 1 : 0;
+    if (ev0 && (e = cudaEventRecord(ev0, stream)) != cudaSuccess) return finish(ra::host_cuda_fail(e, "cudaEventRecord"));
     if ((e = ra::launch_attn_tc(a, t, stream)) != cudaSuccess) return finish(ra::host_cuda_fail(e, "attention launch"));
+    if (ev1 && (e = cudaEventRecord(ev1, stream)) != cudaSuccess) return finish(ra::host_cuda_fail(e, "cudaEventRecord"));
     return finish(RA_OK);
+}
+
+}  // namespace
+
+extern "C" int ra_forward_varlen(const void* q, const void* k, const void* v, void* out, float* lse,
+                                 const int64_t* cu_seqlens, int n_seqs, int64_t H, int64_t D, int n_ring,
+                                 int causal, int layout, void* stream_handle) {
+    return varlen_forward(q, k, v, out, lse, cu_seqlens, n_seqs, H, D, n_ring, causal, layout,
+                          static_cast<cudaStream_t>(stream_handle), nullptr, 0, 0, RA_DEBUG_NONE, nullptr, nullptr);
+}
+
+extern "C" int ra_forward_varlen_ex(const void* q, const void* k, const void* v, void* out, float* lse,
+                                    const int64_t* cu_seqlens, int n_seqs, int64_t H, int64_t D, int n_ring,
+                                    int causal, int layout, void* stream_handle, const ra_options* opt) {
+    ra_options o{};
+    if (opt) o = *opt;
+    if (o.variant != RA_VARIANT_AUTO && o.variant != RA_VARIANT_FUSED) return RA_ERR_UNSUPPORTED;
+    if (o.kernel != RA_KERNEL_AUTO && o.kernel != RA_KERNEL_TC) return RA_ERR_UNSUPPORTED;
+    if (o.debug != RA_DEBUG_NONE && o.debug != RA_DEBUG_STALL_LOADS) return RA_ERR_INVALID_ARG;
+    return varlen_forward(q, k, v, out, lse, cu_seqlens, n_seqs, H, D, n_ring, causal, layout,
+                          static_cast<cudaStream_t>(stream_handle), static_cast<uint8_t*>(o.workspace),
+                          o.workspace_bytes, o.timeout_ns, o.debug, static_cast<cudaEvent_t>(o.attn_events[0]),
+                          static_cast<cudaEvent_t>(o.attn_events[1]));
+}
+
+extern "C" int ra_varlen_workspace_size(const int64_t* cu_seqlens, int n_seqs, int64_t H, int64_t D, int n_ring,
+                                        int layout, size_t* bytes) {
+    if (!bytes) return RA_ERR_INVALID_ARG;
+    int64_t S_total = 0;
+    const int rc = check_packed(cu_seqlens, n_seqs, H, D, n_ring, layout, &S_total);
+    if (rc != RA_OK) return rc;
+    *bytes = scratch_layout(cu_seqlens, n_seqs, H, D, n_ring, layout, S_total).bytes;
+    return RA_OK;
 }

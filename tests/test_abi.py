@@ -105,3 +105,31 @@ def test_backward_rope_and_varlen_validate_before_any_cuda_call():
     assert lib.ra_forward_varlen(FAKE, FAKE, FAKE, FAKE, FAKE, cu.ctypes.data, 2, 1, 128, 4, 1, 3, None) == -1
     cu = np.array([4, 64, 128], dtype=np.int64)
     assert lib.ra_forward_varlen(FAKE, FAKE, FAKE, FAKE, FAKE, cu.ctypes.data, 2, 1, 128, 4, 1, 0, None) == -1
+
+
+def test_varlen_workspace_size_and_options_validate_on_the_host():
+    lib = ra.lib()
+    lengths = [1024, 0, 600 * 8, 48, 4096]
+    cu = np.concatenate([[0], np.cumsum(lengths)]).astype(np.int64)
+    H, D, N = 3, 128, 8
+    a256 = lambda x: -(-x // 256) * 256
+    items = sum(H * N * -(-(n // N) // 256) for n in lengths)
+    base = 256 + a256(len(lengths) * 8) + a256(items * 16)
+    assert ra.varlen_workspace_size(cu, H, D, N, "contiguous") == base
+    assert ra.varlen_workspace_size(cu, H, D, N, "striped") == base
+    assert ra.varlen_workspace_size(cu, H, D, N, "zigzag") == base + 3 * a256(int(cu[-1]) * H * D * 2)
+    with pytest.raises(ra.RAError):  # 600 * 8 + 4 is not a multiple of 2N
+        ra.varlen_workspace_size([0, 600 * 8 + 4], H, D, N, "zigzag")
+
+    def ex(variant=0, kernel=0, ws=None, nbytes=0, debug=0):
+        opt = ra.Options()
+        opt.variant, opt.kernel, opt.debug = variant, kernel, debug
+        opt.workspace, opt.workspace_bytes = ws, nbytes
+        return lib.ra_forward_varlen_ex(FAKE, FAKE, FAKE, FAKE, FAKE, cu.ctypes.data, len(lengths), H, D, N, 1, 2,
+                                        None, ctypes.byref(opt))
+    assert ex(variant=2) == -4                        # per-step variant not offered
+    assert ex(kernel=2) == -4                         # CUDA-core kernel not offered
+    assert ex(debug=9) == -1
+    need = ra.varlen_workspace_size(cu, H, D, N, "zigzag")
+    assert ex(ws=FAKE + 16, nbytes=need) == -3        # workspace not 256-byte aligned
+    assert ex(ws=FAKE, nbytes=need - 1) == -5         # workspace too small
