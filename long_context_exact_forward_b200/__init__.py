@@ -253,8 +253,9 @@ def backward(q, k, v, out, lse, dout, n_ring, causal=True, layout="contiguous", 
              dk=None, dv=None, stream=None, timeout_ns=0, debug=0):
     """ra_backward_ex: gradients (dq, dk, dv) of forward(q, k, v, n_ring, causal, layout) for the
     upstream gradient dout, recomputed block by block in ring order from the saved out and lse.
-    kernel: "auto" (tensor cores for bf16 with D in {64, 128} and the contiguous or striped layout,
-    else CUDA cores), "tc" or "simt".  All tensors [B, S, H, D] in q's dtype except lse."""
+    kernel: "auto" (tensor cores for bf16 with D in {64, 128} and 16-byte aligned tensors, any layout --
+    zigzag through shard-major copies -- else CUDA cores), "tc" or "simt".  All tensors [B, S, H, D] in
+    q's dtype except lse."""
     torch = _torch()
     _check_cuda(q, k, v, out, lse, dout)
     if not (q.shape == k.shape == v.shape == out.shape == dout.shape) or q.dim() != 4:
