@@ -160,11 +160,15 @@ def _stream_handle(stream):
 
 
 def _check_cuda(*ts):
+    """Every tensor of one call lives on the same CUDA device (the kernels run on that device and
+    dereference every pointer there) and is contiguous."""
     for t in ts:
         if not t.is_cuda:
             raise ValueError("tensors must live on a CUDA device")
         if not t.is_contiguous():
             raise ValueError("tensors must be contiguous")
+        if t.device != ts[0].device:
+            raise ValueError(f"tensors of one call must share a device ({ts[0].device} and {t.device})")
 
 
 def workspace_size(B, H, S, D, n_ring, causal, layout, dtype_code, variant="auto", kernel="auto"):
@@ -202,7 +206,7 @@ def forward(q, k, v, n_ring, causal=True, layout="contiguous", *, variant="auto"
     opt.variant = VARIANTS[variant]
     opt.kernel = KERNELS[kernel]
     if workspace is not None:
-        _check_cuda(workspace)
+        _check_cuda(q, workspace)
         opt.workspace = workspace.data_ptr()
         opt.workspace_bytes = workspace.numel() * workspace.element_size()
     opt.timeout_ns = int(timeout_ns)
@@ -327,7 +331,7 @@ def forward_varlen(q, k, v, cu_seqlens, n_ring, causal=True, layout="contiguous"
             workspace = torch.empty(n, dtype=torch.uint8, device=q.device)
         if stream is not None:  # the scratch must outlive the work enqueued on `stream`
             workspace.record_stream(stream)
-    _check_cuda(workspace)
+    _check_cuda(q, workspace)
     opt = Options()
     opt.workspace = workspace.data_ptr()
     opt.workspace_bytes = workspace.numel() * workspace.element_size()

@@ -41,6 +41,13 @@ def test_check_out_rejects_what_the_kernels_would_overrun(t):
         ra._check_out(t, like.shape, torch.bfloat16, "out", like)
 
 
+def test_tensors_of_one_call_must_share_a_device():
+    a, b = FakeCuda((4, 8), torch.bfloat16), FakeCuda((4, 8), torch.bfloat16, device="cuda:1")
+    ra._check_cuda(a, FakeCuda((4, 8), torch.bfloat16))
+    with pytest.raises(ValueError, match="share a device"):
+        ra._check_cuda(a, b)
+
+
 def test_cpu_tensors_are_refused_before_the_library():
     q = torch.zeros(1, 64, 2, 16)
     with pytest.raises(ValueError, match="CUDA"):
