@@ -158,8 +158,9 @@ RA_API int ra_plan_items(int64_t B, int64_t H, int64_t S, int64_t D, int n_ring,
                          int layout, int32_t* items, int64_t cap, int64_t* n_items);
 
 /* RA_NOALLOC_SCRATCH_BYTES: size of the fixed device array that ra_forward_noalloc uses as
- * scratch.  Every GPU that loads the library holds this much device memory until the process
- * exits. */
+ * scratch.  The array is part of the library's device code: a GPU holds it from the moment that
+ * code is loaded there (the first use of the library on the device under CUDA's default lazy
+ * module loading; context creation with CUDA_MODULE_LOADING=EAGER) until the process exits. */
 #define RA_NOALLOC_SCRATCH_BYTES (64u << 20)
 
 /* ra_forward_noalloc: the pages have no counterpart to this call; it exists for callers that
@@ -169,14 +170,15 @@ RA_API int ra_plan_items(int64_t B, int64_t H, int64_t S, int64_t D, int n_ring,
  * tensor-core ring), but takes its scratch (work list and counter; shard-major copies of q, k, v
  * for the zigzag layout) from one fixed device array of RA_NOALLOC_SCRATCH_BYTES instead of
  * allocating.  Arguments as for ra_forward (dtype is bf16 implicitly).
- *   - The first call on a device looks up the array's address with that device current; make it
- *     before any stream capture.
+ *   - The first call on a device, with that device current, looks up the array's address and
+ *     loads the code of every kernel the call launches (both head dims, every layout), so that no
+ *     later call loads module code; make that first call before any stream capture.
  *   - All calls on a device share the array and leave their data in it; calls whose GPU work
  *     overlaps (other streams, other host threads) race on it.
  *   - A problem whose scratch does not fit (B*H*n_ring*ceil(S_loc/256) work items of 16 bytes,
- *     plus 3*B*S*H*D*2 bytes for zigzag and 256 bytes of counter, at most 11264 items per
- *     head) is rejected with
- *     RA_ERR_NO_WORKSPACE and a message in ra_last_error_string; nothing is enqueued.
+ *     plus 3*B*S*H*D*2 bytes for zigzag and 256 bytes of counter), or whose work list the device
+ *     builder cannot hold ((n_ring*ceil(S_loc/256) + n_ring) * 4 bytes above 48 KB), is rejected
+ *     with RA_ERR_NO_WORKSPACE and a message in ra_last_error_string; nothing is enqueued.
  *   - Other dtypes or head dims return RA_ERR_UNSUPPORTED. */
 RA_API int ra_forward_noalloc(const void* q, const void* k, const void* v, void* out, float* lse,
                               int64_t B, int64_t H, int64_t S, int64_t D, int n_ring, int causal,
@@ -270,6 +272,56 @@ RA_API int ra_varlen_workspace_size(const int64_t* cu_seqlens, int n_seqs, int64
  * or a validation error before anything is enqueued. */
 RA_API int ra_rope(const void* x, void* y, int64_t B, int64_t S, int64_t H, int64_t D, int64_t pos_offset,
                    double base, int dtype, void* stream);
+
+/* ---- One ring step on one device's own buffers (a real multi-device ring).
+ *
+ * On a real ring device i keeps its query block Q_i and, at step s, holds the key/value block of
+ * device j = (i - s) mod n_ring, which its left neighbour sent it during the previous step; it
+ * computes the partial attention of Q_i against that block and merges it into its running result
+ * (jisaku.com "Ring Attention", 処理フロー and 通信計算オーバーラップ; ultralytics.com "Ring
+ * Attention", "how ring attention works").  These calls are the per-device compute of that loop;
+ * moving the blocks between devices is the caller's (for example NCCL send/recv into a local
+ * buffer -- the kernels only ever read memory of the current device).
+ *
+ * Local buffers hold one shard each, in the layout's local order: q_i[b, a] is global token
+ * g(i, a) and k_j[b, a], v_j[b, a] are global token g(j, a), with g the layout map described at the
+ * top of this file; every buffer is [B, S_loc, H, D], S_loc = S / n_ring.  The causal mask still
+ * compares global positions, so the result of n_ring steps equals rows g(i, 0..S_loc-1) of
+ * ra_forward on the whole sequence.
+ *
+ * ra_ring_step: step `step` (0 <= step < n_ring) of query shard `shard`, whose key/value block is
+ * j = (shard - step) mod n_ring.
+ *   q_i, k_j, v_j: [B, S_loc, H, D] in dtype (bf16 with D in {64, 128} on sm_100 runs on the tensor
+ *     cores and needs 16-byte aligned pointers; other cases run the fp32 CUDA-core kernel).
+ *   O_acc: [B, S_loc, H, D] fp32, 16-byte aligned; lse_acc: [B, S_loc, H] fp32.  The running
+ *     result: O normalised by its own sum and its log-sum-exp.  Step 0 writes it (nothing is read);
+ *     a later step merges its partial into it with the log-sum-exp form of the merge identities
+ *     (troisinh.com "Ring Attention", "Tai sao no hoat dong").  Every step must see the same
+ *     B, H, S, D, n_ring, causal, layout, dtype and shard.  A later step whose whole block is
+ *     masked for every query of the shard enqueues nothing.
+ *   sms_reserved: SMs the persistent tensor-core kernel leaves free (0 <= sms_reserved < SM count),
+ *     so that a transfer kernel running at the same time (an NCCL send/recv of the next block) finds
+ *     room on the GPU instead of waiting for the attention kernel to end; the CUDA-core kernel
+ *     ignores it.
+ *   workspace: device scratch of at least ra_ring_step_workspace_size bytes, 256-byte aligned
+ *     (work list, counter, and the step's partial result); NULL: allocated and freed
+ *     stream-ordered on `stream`.
+ *   Asynchronous on `stream`; bounded in-kernel waits report through ra_get_device_status. */
+RA_API int ra_ring_step(const void* q_i, const void* k_j, const void* v_j, float* O_acc, float* lse_acc,
+                        int64_t B, int64_t H, int64_t S, int64_t D, int n_ring, int causal, int layout,
+                        int dtype, int shard, int step, int sms_reserved, void* workspace,
+                        size_t workspace_bytes, void* stream);
+
+/* ra_ring_step_workspace_size: scratch bytes that suffice for ra_ring_step at every (shard, step) of
+ * these arguments, written to *bytes.  Host only. */
+RA_API int ra_ring_step_workspace_size(int64_t B, int64_t H, int64_t S, int64_t D, int n_ring, int causal,
+                                       int layout, int dtype, size_t* bytes);
+
+/* ra_ring_finalize: write the running result of a shard after its last step: out [B, S_loc, H, D] in
+ * dtype (bf16 rounded to nearest even) and lse [B, H, S_loc] fp32, both in the shard's local token
+ * order.  O_acc and out 16-byte aligned.  Asynchronous on `stream`. */
+RA_API int ra_ring_finalize(const float* O_acc, const float* lse_acc, void* out, float* lse, int64_t B,
+                            int64_t H, int64_t S_loc, int64_t D, int dtype, void* stream);
 
 /* ra_status_string: static description of a status code. */
 RA_API const char* ra_status_string(int status);

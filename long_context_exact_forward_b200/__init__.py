@@ -13,6 +13,9 @@ Entry points (same names as the C ABI):
     varlen_workspace_size(cu_seqlens, H, D, ...)     -> int             ra_varlen_workspace_size
     backward(q, k, v, out, lse, dout, n_ring, ...)   -> (dq, dk, dv)    ra_backward_ex
     rope(x, pos_offset, base)                        -> tensor          ra_rope
+    ring_step(q_i, k_j, v_j, O_acc, lse_acc, ...)                        ra_ring_step
+    ring_step_workspace_size(...)                    -> int             ra_ring_step_workspace_size
+    ring_finalize(O_acc, lse_acc)                    -> (out, lse)      ra_ring_finalize
     workspace_size(...)                              -> int             ra_workspace_size
     permute(x, n_ring, layout) / unpermute(...)      -> tensor          ra_permute / ra_unpermute
     merge_partials(O_run, lse_run, O_step, lse_step)                     ra_merge_partials
@@ -93,6 +96,11 @@ def lib():
         L.ra_rope.argtypes = [vp, vp, i64, i64, i64, i64, i64, ctypes.c_double, ci, vp]
         L.ra_backward_ex.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i64, i64, i64, i64, ci, ci, ci,
                                      ci, ci, ctypes.c_uint64, ci, vp]
+        L.ra_ring_step.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i64, ci, ci, ci, ci, ci, ci, ci, vp,
+                                   ctypes.c_size_t, vp]
+        L.ra_ring_step_workspace_size.argtypes = [i64, i64, i64, i64, ci, ci, ci, ci,
+                                                  ctypes.POINTER(ctypes.c_size_t)]
+        L.ra_ring_finalize.argtypes = [vp, vp, vp, vp, i64, i64, i64, i64, ci, vp]
         L.ra_layout_positions.argtypes = [i64, ci, ci, vp]
         L.ra_plan_tiles.argtypes = [i64, ci, ci, ci, ci, vp]
         L.ra_plan_items.argtypes = [i64, i64, i64, i64, ci, ci, ci, vp, i64, ctypes.POINTER(ctypes.c_int64)]
@@ -106,7 +114,8 @@ def lib():
         for name in ("ra_forward", "ra_forward_ex", "ra_forward_noalloc", "ra_workspace_size", "ra_permute",
                      "ra_unpermute", "ra_merge_partials", "ra_layout_positions", "ra_plan_tiles",
                      "ra_plan_items", "ra_get_device_status", "ra_backward", "ra_backward_ex", "ra_rope", "ra_forward_varlen",
-                     "ra_forward_varlen_ex", "ra_varlen_workspace_size"):
+                     "ra_forward_varlen_ex", "ra_varlen_workspace_size", "ra_ring_step",
+                     "ra_ring_step_workspace_size", "ra_ring_finalize"):
             getattr(L, name).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -368,6 +377,74 @@ def rope(x, pos_offset=0, base=10000.0, out=None, stream=None):
                            _dtype_code(x), _stream_handle(stream))
     _check(rc, "ra_rope")
     return out
+
+
+def ring_step_workspace_size(B, H, S, D, n_ring, causal, layout, dtype_code):
+    """Scratch bytes that suffice for ring_step at every (shard, step) of these arguments."""
+    n = ctypes.c_size_t(0)
+    _clear_error()
+    _check(lib().ra_ring_step_workspace_size(B, H, S, D, int(n_ring), int(bool(causal)), LAYOUTS[layout],
+                                             dtype_code, ctypes.byref(n)), "ra_ring_step_workspace_size")
+    return n.value
+
+
+def ring_step(q_i, k_j, v_j, O_acc, lse_acc, n_ring, shard, step, causal=True, layout="contiguous", *,
+              sms_reserved=0, workspace=None, stream=None):
+    """ra_ring_step: one ring step of query shard `shard` against the key/value block
+    j = (shard - step) mod n_ring held in this device's own buffers.
+
+    q_i, k_j, v_j: [B, S_loc, H, D] (fp32 or bf16) in the layout's local token order; O_acc fp32
+    [B, S_loc, H, D] and lse_acc fp32 [B, S_loc, H] hold the running result (written at step 0,
+    merged into afterwards).  `workspace`: an optional uint8 CUDA tensor of at least
+    ring_step_workspace_size(...) bytes; without it the scratch comes from torch's caching
+    allocator.  `sms_reserved`: SMs the tensor-core kernel leaves free for a concurrent transfer."""
+    torch = _torch()
+    _check_cuda(q_i, k_j, v_j, O_acc, lse_acc)
+    if q_i.dim() != 4 or q_i.shape != k_j.shape or q_i.shape != v_j.shape:
+        raise ValueError("q_i, k_j, v_j must all be [B, S_loc, H, D]")
+    if not (q_i.dtype == k_j.dtype == v_j.dtype):
+        raise TypeError("q_i, k_j, v_j must share a dtype")
+    B, S_loc, H, D = q_i.shape
+    _check_out(O_acc, q_i.shape, torch.float32, "O_acc", q_i)
+    _check_out(lse_acc, (B, S_loc, H), torch.float32, "lse_acc", q_i)
+    S = S_loc * int(n_ring)
+    if workspace is None:
+        n = ring_step_workspace_size(B, H, S, D, n_ring, causal, layout, _dtype_code(q_i))
+        with torch.cuda.device(q_i.device):
+            workspace = torch.empty(n, dtype=torch.uint8, device=q_i.device)
+        if stream is not None:  # the scratch must outlive the work enqueued on `stream`
+            workspace.record_stream(stream)
+    _check_cuda(q_i, workspace)
+    _clear_error()
+    with torch.cuda.device(q_i.device):
+        rc = lib().ra_ring_step(q_i.data_ptr(), k_j.data_ptr(), v_j.data_ptr(), O_acc.data_ptr(),
+                                lse_acc.data_ptr(), B, H, S, D, int(n_ring), int(bool(causal)), LAYOUTS[layout],
+                                _dtype_code(q_i), int(shard), int(step), int(sms_reserved), workspace.data_ptr(),
+                                workspace.numel(), _stream_handle(stream))
+    _check(rc, "ra_ring_step")
+    return O_acc, lse_acc
+
+
+def ring_finalize(O_acc, lse_acc, out=None, lse=None, dtype=None, stream=None):
+    """ra_ring_finalize: the shard's result after its last ring step, out [B, S_loc, H, D] in `dtype`
+    (default bf16) and lse [B, H, S_loc] fp32, in the shard's local token order."""
+    torch = _torch()
+    _check_cuda(O_acc, lse_acc)
+    if O_acc.dim() != 4 or O_acc.dtype != torch.float32:
+        raise ValueError("O_acc must be fp32 [B, S_loc, H, D]")
+    B, S_loc, H, D = O_acc.shape
+    _check_out(lse_acc, (B, S_loc, H), torch.float32, "lse_acc", O_acc)
+    dtype = dtype or (out.dtype if out is not None else torch.bfloat16)
+    out = torch.empty(O_acc.shape, dtype=dtype, device=O_acc.device) if out is None else out
+    lse = torch.empty((B, H, S_loc), dtype=torch.float32, device=O_acc.device) if lse is None else lse
+    _check_out(out, O_acc.shape, dtype, "out", O_acc)
+    _check_out(lse, (B, H, S_loc), torch.float32, "lse", O_acc)
+    _clear_error()
+    with torch.cuda.device(O_acc.device):
+        rc = lib().ra_ring_finalize(O_acc.data_ptr(), lse_acc.data_ptr(), out.data_ptr(), lse.data_ptr(), B, H,
+                                    S_loc, D, _dtype_code(out), _stream_handle(stream))
+    _check(rc, "ra_ring_finalize")
+    return out, lse
 
 
 def permute(x, n_ring, layout, out=None, stream=None, inverse=False):

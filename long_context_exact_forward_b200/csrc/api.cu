@@ -20,9 +20,13 @@
 #include <cstdio>
 #include <cstring>
 #include <map>
+#include <memory>
 #include <mutex>
 #include <tuple>
+#include <utility>
 #include <vector>
+
+#include <nvtx3/nvToolsExt.h>
 
 #include "ra.h"
 #include "ra_internal.cuh"
@@ -34,6 +38,12 @@ namespace {
 using ra::Layout;
 
 thread_local char g_last_error[512] = "";
+
+// Close the NVTX range an entry point opened and pass its status through (early returns).
+int nvtx_pop(int status) {
+    nvtxRangePop();
+    return status;
+}
 
 int cuda_fail(cudaError_t e, const char* what) {
     snprintf(g_last_error, sizeof g_last_error, "%s: %s (%s)", what, cudaGetErrorString(e),
@@ -112,34 +122,83 @@ struct PlanKey {
     int64_t B, H, S;
     int n_ring, causal, layout, s_begin, s_end;
     int64_t D;
+    int shard;  // -1: every shard; otherwise the items of this query shard only
     bool operator<(const PlanKey& o) const {
-        return std::tie(B, H, S, n_ring, causal, layout, s_begin, s_end, D) <
-               std::tie(o.B, o.H, o.S, o.n_ring, o.causal, o.layout, o.s_begin, o.s_end, o.D);
+        return std::tie(B, H, S, n_ring, causal, layout, s_begin, s_end, D, shard) <
+               std::tie(o.B, o.H, o.S, o.n_ring, o.causal, o.layout, o.s_begin, o.s_end, o.D, o.shard);
     }
+};
+
+// A map from problem shape to a planned object, bounded to kCacheEntries entries: inserting
+// beyond that drops the least recently used one.  Entries are shared_ptr, so a caller still
+// holding a dropped entry keeps it alive until it lets go.  The cache objects themselves are
+// created with new and never destroyed, so no CUDA call runs during static destruction.
+constexpr size_t kCacheEntries = 64;
+
+template <class K, class V>
+class LruCache {
+  public:
+    std::shared_ptr<V> get(const K& key) {
+        std::lock_guard<std::mutex> lock(mu_);
+        auto it = map_.find(key);
+        if (it == map_.end()) return nullptr;
+        it->second.first = ++tick_;
+        return it->second.second;
+    }
+    // Insert unless another thread got there first; returns the entry that is cached.
+    std::shared_ptr<V> put(const K& key, std::shared_ptr<V> value) {
+        std::shared_ptr<V> dropped;  // released after the lock, so its destructor runs unlocked
+        std::lock_guard<std::mutex> lock(mu_);
+        auto it = map_.find(key);
+        if (it != map_.end()) return it->second.second;
+        map_.emplace(key, std::make_pair(++tick_, value));
+        if (map_.size() > kCacheEntries) {
+            auto oldest = map_.begin();
+            for (auto jt = map_.begin(); jt != map_.end(); ++jt)
+                if (jt->second.first < oldest->second.first) oldest = jt;
+            dropped = std::move(oldest->second.second);
+            map_.erase(oldest);
+        }
+        return value;
+    }
+    size_t size() {
+        std::lock_guard<std::mutex> lock(mu_);
+        return map_.size();
+    }
+
+  private:
+    std::mutex mu_;
+    std::map<K, std::pair<uint64_t, std::shared_ptr<V>>> map_;
+    uint64_t tick_ = 0;
 };
 
 struct PlanItem {
     int32_t b, h, i, p, cost;
 };
 
+using ItemList = std::vector<PlanItem>;
+
+LruCache<PlanKey, const ItemList>& plan_cache() {
+    static auto* cache = new LruCache<PlanKey, const ItemList>();
+    return *cache;
+}
+
 // Work list of the tensor-core kernel for ring steps [s_begin, s_end): one item per
-// (b, h, shard i, pair of 128-row query tiles), cost = live (query tile, key tile) pairs.
+// (b, h, shard i, pair of 128-row query tiles), cost = live (query tile, key tile) pairs; with
+// shard >= 0 only the items of that query shard (a ring step on one device's local buffers).
 // Order: (b, h) major so that CTAs running at the same time share one head's keys and values in
 // L2; inside a head, heaviest first (LPT) so the short items fill the tail -- or, when one head's
 // K/V exceeds L2 (plan_groups_by_shard), shard groups heaviest first and LPT inside a group.
-const std::vector<PlanItem>& plan_items(int64_t B, int64_t H, const Layout& L, int64_t D_for_plan,
-                                        int causal, int s_begin, int s_end) {
-    static std::mutex mu;
-    static std::map<PlanKey, std::vector<PlanItem>> cache;
-    PlanKey key{B, H, L.S, (int)L.N, causal, L.kind, s_begin, s_end, D_for_plan};
-    std::lock_guard<std::mutex> lock(mu);
-    auto it = cache.find(key);
-    if (it != cache.end()) return it->second;
+std::shared_ptr<const ItemList> plan_items(int64_t B, int64_t H, const Layout& L, int64_t D_for_plan,
+                                           int causal, int s_begin, int s_end, int shard = -1) {
+    const PlanKey key{B, H, L.S, (int)L.N, causal, L.kind, s_begin, s_end, D_for_plan, shard};
+    if (auto hit = plan_cache().get(key)) return hit;
     const int64_t pairs = (L.S_loc + kTcPairRows - 1) / kTcPairRows;
     std::vector<PlanItem> head;
     head.reserve((size_t)(L.N * pairs));
     for (int64_t i = 0; i < L.N; ++i)
         for (int64_t p = 0; p < pairs; ++p) {
+            if (shard >= 0 && i != shard) continue;
             int64_t cost = 0;
             for (int s = s_begin; s < s_end; ++s) {
                 const int64_t j = ra::ring_block(i, s, L.N);
@@ -164,59 +223,111 @@ const std::vector<PlanItem>& plan_items(int64_t B, int64_t H, const Layout& L, i
         std::stable_sort(head.begin(), head.end(),
                          [](const PlanItem& x, const PlanItem& y) { return x.cost > y.cost; });
     }
-    std::vector<PlanItem> all;
-    all.reserve(head.size() * (size_t)(B * H));
+    auto all = std::make_shared<ItemList>();
+    all->reserve(head.size() * (size_t)(B * H));
     for (int64_t b = 0; b < B; ++b)
         for (int64_t h = 0; h < H; ++h)
             for (PlanItem x : head) {
                 x.b = (int32_t)b;
                 x.h = (int32_t)h;
-                all.push_back(x);
+                all->push_back(x);
             }
-    return cache.emplace(key, std::move(all)).first->second;
+    return plan_cache().put(key, std::move(all));
 }
 
-// All lists of one call flattened into pinned host memory (kept for the life of the process, so
-// the asynchronous upload never reads freed or pageable memory).  offsets[s] .. offsets[s + 1]
-// delimit the list of step s (per-step) or the single list (fused).
+// All lists of one call flattened into pinned host memory, so that the upload is a true
+// asynchronous copy.  offsets[s] .. offsets[s + 1] delimit the list of step s (per-step) or the
+// single list (fused).  Pinned memory may only be freed once no copy from it is pending: every
+// upload records an event on its stream, and the destructor (run when the bounded cache drops
+// the entry and no call holds it any more) waits for those events first.  An upload recorded
+// into a CUDA graph reads the buffer at every replay, for as long as the graph lives, which the
+// library cannot see; such a buffer is never freed.
 struct FlatList {
     int4* data = nullptr;
     size_t count = 0;
     std::vector<int> offsets;
+    std::mutex mu;
+    std::vector<std::pair<cudaStream_t, cudaEvent_t>> uploads;  // latest upload per stream
+    bool in_graph = false;
+
+    FlatList() = default;
+    FlatList(const FlatList&) = delete;
+    FlatList& operator=(const FlatList&) = delete;
+    ~FlatList() {
+        if (in_graph) return;  // a captured graph may still copy from data
+        for (auto& u : uploads) {
+            cudaEventSynchronize(u.second);
+            cudaEventDestroy(u.second);
+        }
+        if (data) cudaFreeHost(data);
+    }
+
+    // Upload [first, first + n) items to dst on `stream`, and remember the copy.
+    cudaError_t upload(void* dst, size_t first, size_t n, cudaStream_t stream) {
+        cudaError_t e = cudaMemcpyAsync(dst, data + first, n * sizeof(int4), cudaMemcpyHostToDevice, stream);
+        if (e != cudaSuccess) return e;
+        cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+        if ((e = cudaStreamIsCapturing(stream, &cap)) != cudaSuccess) return e;
+        std::lock_guard<std::mutex> lock(mu);
+        if (cap != cudaStreamCaptureStatusNone) {
+            in_graph = true;
+            return cudaSuccess;
+        }
+        cudaEvent_t ev = nullptr;
+        for (auto& u : uploads)
+            if (u.first == stream) ev = u.second;
+        if (!ev) {
+            if ((e = cudaEventCreateWithFlags(&ev, cudaEventDisableTiming)) != cudaSuccess) return e;
+            uploads.emplace_back(stream, ev);
+        }
+        return cudaEventRecord(ev, stream);
+    }
 };
 
+struct FlatKey {
+    PlanKey plan;
+    bool per_step;
+    int device;
+    bool operator<(const FlatKey& o) const {
+        return std::tie(plan, per_step, device) < std::tie(o.plan, o.per_step, o.device);
+    }
+};
+
+LruCache<FlatKey, FlatList>& flat_cache() {
+    static auto* cache = new LruCache<FlatKey, FlatList>();
+    return *cache;
+}
+
+// shard >= 0: the list of that query shard for the single step s_begin (a ring step on local
+// buffers); otherwise every shard, for all steps (fused) or one list per step (per_step).
 int flat_items(int64_t B, int64_t H, const Layout& L, int64_t D, int causal, bool per_step,
-               const FlatList** out) {
-    static std::mutex mu;
-    static std::map<std::pair<PlanKey, bool>, FlatList> cache;
-    const PlanKey key{B, H, L.S, (int)L.N, causal, L.kind, 0, (int)L.N, D};
-    {
-        std::lock_guard<std::mutex> lock(mu);
-        auto it = cache.find({key, per_step});
-        if (it != cache.end()) {
-            *out = &it->second;
-            return RA_OK;
-        }
-    }
-    FlatList f;
+               std::shared_ptr<FlatList>* out, int shard = -1, int step = 0) {
+    int device = 0;
+    cudaError_t e = cudaGetDevice(&device);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    const PlanKey pk = shard >= 0 ? PlanKey{B, H, L.S, (int)L.N, causal, L.kind, step, step + 1, D, shard}
+                                  : PlanKey{B, H, L.S, (int)L.N, causal, L.kind, 0, (int)L.N, D, -1};
+    const FlatKey key{pk, per_step, device};
+    if ((*out = flat_cache().get(key))) return RA_OK;
+    auto f = std::make_shared<FlatList>();
     std::vector<int4> flat;
-    const int n_lists = per_step ? (int)L.N : 1;
+    const int n_lists = (per_step && shard < 0) ? (int)L.N : 1;
     for (int s = 0; s < n_lists; ++s) {
-        f.offsets.push_back((int)flat.size());
-        const auto& items = per_step ? plan_items(B, H, L, D, causal, s, s + 1) : plan_items(B, H, L, D, causal, 0, (int)L.N);
-        for (const PlanItem& x : items) flat.push_back(make_int4(x.b, x.h, x.i, x.p));
+        f->offsets.push_back((int)flat.size());
+        std::shared_ptr<const ItemList> items =
+            shard >= 0 ? plan_items(B, H, L, D, causal, step, step + 1, shard)
+            : per_step ? plan_items(B, H, L, D, causal, s, s + 1)
+                       : plan_items(B, H, L, D, causal, 0, (int)L.N);
+        for (const PlanItem& x : *items) flat.push_back(make_int4(x.b, x.h, x.i, x.p));
     }
-    f.offsets.push_back((int)flat.size());
-    f.count = flat.size();
-    if (f.count) {
-        cudaError_t e = cudaHostAlloc(reinterpret_cast<void**>(&f.data), f.count * sizeof(int4), cudaHostAllocPortable);
+    f->offsets.push_back((int)flat.size());
+    f->count = flat.size();
+    if (f->count) {
+        e = cudaHostAlloc(reinterpret_cast<void**>(&f->data), f->count * sizeof(int4), cudaHostAllocPortable);
         if (e != cudaSuccess) return cuda_fail(e, "cudaHostAlloc(work list)");
-        std::memcpy(f.data, flat.data(), f.count * sizeof(int4));
+        std::memcpy(f->data, flat.data(), f->count * sizeof(int4));
     }
-    std::lock_guard<std::mutex> lock(mu);
-    auto ins = cache.emplace(std::make_pair(key, per_step), std::move(f));
-    if (!ins.second && f.data) cudaFreeHost(f.data);  // another thread won the race
-    *out = &ins.first->second;
+    *out = flat_cache().put(key, std::move(f));
     return RA_OK;
 }
 
@@ -241,9 +352,9 @@ Workspace carve(int64_t B, int64_t H, const Layout& L, int64_t D, int causal, in
     w.per_step = per_step && L.N > 1;
     if (kernel == kTC) {
         if (w.per_step) {
-            for (int s = 0; s < (int)L.N; ++s) w.n_items_total += plan_items(B, H, L, D, causal, s, s + 1).size();
+            for (int s = 0; s < (int)L.N; ++s) w.n_items_total += plan_items(B, H, L, D, causal, s, s + 1)->size();
         } else {
-            w.n_items_total = plan_items(B, H, L, D, causal, 0, (int)L.N).size();
+            w.n_items_total = plan_items(B, H, L, D, causal, 0, (int)L.N)->size();
         }
         w.counters = off;
         w.n_counters = w.per_step ? (size_t)L.N : 1;
@@ -398,8 +509,10 @@ int run_forward(const Call& c, const ra_options& opt) {
         if (w.permute) {
             const void* src[3] = {c.q, c.k, c.v};
             void* dst[3] = {ws + w.qp, ws + w.kp, ws + w.vp};
-            if ((e = ra::launch_permute(src, dst, 3, c.B, L, c.H, c.D, 2, false, c.stream)) != cudaSuccess)
-                return finish(cuda_fail(e, "permute launch"));
+            nvtxRangePushA("ra_forward permute");
+            e = ra::launch_permute(src, dst, 3, c.B, L, c.H, c.D, 2, false, c.stream);
+            nvtxRangePop();
+            if (e != cudaSuccess) return finish(cuda_fail(e, "permute launch"));
             q = dst[0];
             k = dst[1];
             v = dst[2];
@@ -409,12 +522,10 @@ int run_forward(const Call& c, const ra_options& opt) {
         if ((rc = encode_qkv_map(&tc.tm_k, k, c.B, L, c.H, c.D, striped_natural)) != RA_OK) return finish(rc);
         if ((rc = encode_qkv_map(&tc.tm_v, v, c.B, L, c.H, c.D, striped_natural)) != RA_OK) return finish(rc);
         // upload the work list(s) from the cached pinned copy
-        const FlatList* fl = nullptr;
+        std::shared_ptr<FlatList> fl;
         if ((rc = flat_items(c.B, c.H, L, c.D, args.causal, w.per_step, &fl)) != RA_OK) return finish(rc);
         step_item_offset = fl->offsets;
-        if (fl->count > 0 &&
-            (e = cudaMemcpyAsync(ws + w.items, fl->data, fl->count * sizeof(int4),
-                                 cudaMemcpyHostToDevice, c.stream)) != cudaSuccess)
+        if (fl->count > 0 && (e = fl->upload(ws + w.items, 0, fl->count, c.stream)) != cudaSuccess)
             return finish(cuda_fail(e, "work list upload"));
         if ((e = cudaMemsetAsync(ws + w.counters, 0, w.n_counters * sizeof(int), c.stream)) != cudaSuccess)
             return finish(cuda_fail(e, "work counter reset"));
@@ -444,24 +555,34 @@ int run_forward(const Call& c, const ra_options& opt) {
 
     if (ev0 && (e = cudaEventRecord(ev0, c.stream)) != cudaSuccess) return finish(cuda_fail(e, "cudaEventRecord"));
     if (!w.per_step) {
-        if ((e = attention(0, (int)L.N, ra::kOutFinal, c.out, c.lse)) != cudaSuccess)
-            return finish(cuda_fail(e, "attention launch"));
+        // the unpermute is fused into the attention kernel's epilogue (natural-order stores)
+        nvtxRangePushA("ra_forward attention (fused ring, unpermute in the epilogue)");
+        e = attention(0, (int)L.N, ra::kOutFinal, c.out, c.lse);
+        nvtxRangePop();
+        if (e != cudaSuccess) return finish(cuda_fail(e, "attention launch"));
     } else {
         float* O_run = reinterpret_cast<float*>(ws + w.O_run);
         float* lse_run = reinterpret_cast<float*>(ws + w.lse_run);
         float* O_step = reinterpret_cast<float*>(ws + w.O_step);
         float* lse_step = reinterpret_cast<float*>(ws + w.lse_step);
         const int64_t rows = c.B * c.S * c.H;
-        if ((e = attention(0, 1, ra::kOutPartial, O_run, lse_run)) != cudaSuccess)
-            return finish(cuda_fail(e, "attention launch (step 0)"));
+        nvtxRangePushA("ra_forward attention (ring step 0)");
+        e = attention(0, 1, ra::kOutPartial, O_run, lse_run);
+        nvtxRangePop();
+        if (e != cudaSuccess) return finish(cuda_fail(e, "attention launch (step 0)"));
         for (int s = 1; s < (int)L.N; ++s) {
-            if ((e = attention(s, s + 1, ra::kOutPartial, O_step, lse_step)) != cudaSuccess)
-                return finish(cuda_fail(e, "attention launch (step)"));
+            nvtxRangePushA("ra_forward attention (ring step)");
+            e = attention(s, s + 1, ra::kOutPartial, O_step, lse_step);
+            nvtxRangePop();
+            if (e != cudaSuccess) return finish(cuda_fail(e, "attention launch (step)"));
+            // the last merge also unpermutes: it writes out and lse in natural order
+            nvtxRangePushA(s + 1 < (int)L.N ? "ra_forward merge" : "ra_forward merge + unpermute");
             if (s + 1 < (int)L.N)
                 e = ra::launch_merge_inplace(O_run, lse_run, O_step, lse_step, rows, c.D, c.stream);
             else
                 e = ra::launch_merge_final(O_run, lse_run, O_step, lse_step, c.out, c.lse, c.dtype, c.B,
                                            L, c.H, c.D, c.stream);
+            nvtxRangePop();
             if (e != cudaSuccess) return finish(cuda_fail(e, "merge launch"));
         }
     }
@@ -536,8 +657,10 @@ int ra_permute(const void* x, void* y, int64_t B, int64_t S, int64_t H, int64_t 
     if (!x || !y) return RA_ERR_INVALID_ARG;
     const void* src[1] = {x};
     void* dst[1] = {y};
+    nvtxRangePushA("ra_permute");
     cudaError_t e = ra::launch_permute(src, dst, 1, B, make_layout(S, n_ring, layout), H, D,
                                        dtype == RA_DTYPE_BF16 ? 2 : 4, false, static_cast<cudaStream_t>(stream));
+    nvtxRangePop();
     return e == cudaSuccess ? RA_OK : cuda_fail(e, "permute launch");
 }
 
@@ -548,8 +671,10 @@ int ra_unpermute(const void* x, void* y, int64_t B, int64_t S, int64_t H, int64_
     if (!x || !y) return RA_ERR_INVALID_ARG;
     const void* src[1] = {x};
     void* dst[1] = {y};
+    nvtxRangePushA("ra_unpermute");
     cudaError_t e = ra::launch_permute(src, dst, 1, B, make_layout(S, n_ring, layout), H, D,
                                        dtype == RA_DTYPE_BF16 ? 2 : 4, true, static_cast<cudaStream_t>(stream));
+    nvtxRangePop();
     return e == cudaSuccess ? RA_OK : cuda_fail(e, "unpermute launch");
 }
 
@@ -557,8 +682,10 @@ int ra_merge_partials(float* O_run, float* lse_run, const float* O_step, const f
                       int64_t rows, int64_t D, void* stream) {
     if (!O_run || !lse_run || !O_step || !lse_step || rows < 0 || D < 1) return RA_ERR_INVALID_ARG;
     if (D % 4 == 0 && (!aligned16(O_run) || !aligned16(O_step))) return RA_ERR_ALIGN;
+    nvtxRangePushA("ra_merge_partials");
     cudaError_t e = ra::launch_merge_inplace(O_run, lse_run, O_step, lse_step, rows, D,
                                              static_cast<cudaStream_t>(stream));
+    nvtxRangePop();
     return e == cudaSuccess ? RA_OK : cuda_fail(e, "merge launch");
 }
 
@@ -604,10 +731,10 @@ int ra_plan_items(int64_t B, int64_t H, int64_t S, int64_t D, int n_ring, int ca
     int rc = check_shape(B, H, S, D, n_ring, layout, RA_DTYPE_FP32);
     if (rc != RA_OK) return rc;
     const Layout L = make_layout(S, n_ring, layout);
-    const auto& list = plan_items(B, H, L, D, causal ? 1 : 0, 0, n_ring);
-    *n_items = (int64_t)list.size();
-    for (int64_t t = 0; t < std::min<int64_t>(cap, (int64_t)list.size()); ++t) {
-        const PlanItem& x = list[(size_t)t];
+    const auto list = plan_items(B, H, L, D, causal ? 1 : 0, 0, n_ring);
+    *n_items = (int64_t)list->size();
+    for (int64_t t = 0; t < std::min<int64_t>(cap, (int64_t)list->size()); ++t) {
+        const PlanItem& x = (*list)[(size_t)t];
         int32_t* d = items + 5 * t;
         d[0] = x.b;
         d[1] = x.h;
@@ -616,6 +743,180 @@ int ra_plan_items(int64_t B, int64_t H, int64_t S, int64_t D, int n_ring, int ca
         d[4] = x.cost;
     }
     return RA_OK;
+}
+
+}  // extern "C"
+
+// ------------------------------------------------------------------ one ring step on local buffers
+namespace {
+
+struct RingWorkspace {
+    size_t counter = 0, items = 0, O_s = 0, lse_s = 0, total = 0;
+    size_t n_items = 0;
+};
+
+RingWorkspace ring_carve(int64_t B, int64_t H, const Layout& L, int64_t D, int causal, int shard, int step,
+                         bool tc) {
+    RingWorkspace w;
+    size_t off = 0;
+    if (tc) {
+        w.n_items = plan_items(B, H, L, D, causal, step, step + 1, shard)->size();
+        w.counter = off;
+        off = align_up(off + sizeof(int));
+        w.items = off;
+        off = align_up(off + w.n_items * sizeof(int4));
+    }
+    const size_t rows = (size_t)(B * L.S_loc * H);
+    w.O_s = off;
+    off = align_up(off + rows * (size_t)D * 4);
+    w.lse_s = off;
+    off = align_up(off + rows * 4);
+    w.total = std::max<size_t>(off, kAlign);
+    return w;
+}
+
+bool ring_kernel_tc(const DeviceInfo& dev, int dtype, int64_t D) {
+    return dev.sm100 && dtype == RA_DTYPE_BF16 && (D == 64 || D == 128);
+}
+
+int ring_check(int64_t B, int64_t H, int64_t S, int64_t D, int n_ring, int layout, int dtype, int shard, int step) {
+    const int rc = check_shape(B, H, S, D, n_ring, layout, dtype);
+    if (rc != RA_OK) return rc;
+    if (shard < 0 || shard >= n_ring || step < 0 || step >= n_ring) return RA_ERR_INVALID_ARG;
+    return RA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int ra_ring_step_workspace_size(int64_t B, int64_t H, int64_t S, int64_t D, int n_ring, int causal, int layout,
+                                int dtype, size_t* bytes) {
+    if (!bytes) return RA_ERR_INVALID_ARG;
+    const int rc = ring_check(B, H, S, D, n_ring, layout, dtype, 0, 0);
+    if (rc != RA_OK) return rc;
+    // host only: the tensor-core carve-up (a superset) whenever it could apply; the largest
+    // work list over every (shard, step) is one item per query-tile pair of each (b, h)
+    const bool tc = dtype == RA_DTYPE_BF16 && (D == 64 || D == 128);
+    const Layout L = make_layout(S, n_ring, layout);
+    const int64_t pairs = (L.S_loc + kTcPairRows - 1) / kTcPairRows;
+    size_t off = 0;
+    if (tc) off = align_up(sizeof(int)) + align_up((size_t)(B * H * pairs) * sizeof(int4));
+    const size_t rows = (size_t)(B * L.S_loc * H);
+    off = align_up(off + rows * (size_t)D * 4);
+    off = align_up(off + rows * 4);
+    *bytes = std::max<size_t>(off, kAlign);
+    (void)causal;
+    return RA_OK;
+}
+
+int ra_ring_step(const void* q_i, const void* k_j, const void* v_j, float* O_acc, float* lse_acc, int64_t B,
+                 int64_t H, int64_t S, int64_t D, int n_ring, int causal, int layout, int dtype, int shard,
+                 int step, int sms_reserved, void* workspace, size_t workspace_bytes, void* stream_handle) {
+    int rc = ring_check(B, H, S, D, n_ring, layout, dtype, shard, step);
+    if (rc != RA_OK) return rc;
+    if (sms_reserved < 0) return RA_ERR_INVALID_ARG;
+    if (!q_i || !k_j || !v_j || !O_acc || !lse_acc) return RA_ERR_INVALID_ARG;
+    const size_t esize = dtype == RA_DTYPE_BF16 ? 2 : 4;
+    auto aligned = [](const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; };
+    if (!aligned(O_acc, 16) || !aligned(lse_acc, 4)) return RA_ERR_ALIGN;
+    DeviceInfo dev;
+    if ((rc = device_info(&dev)) != RA_OK) return rc;
+    if (sms_reserved >= dev.sms) return RA_ERR_INVALID_ARG;
+    const bool tc = ring_kernel_tc(dev, dtype, D);
+    const size_t qkv_align = tc ? 16 : esize;
+    if (!aligned(q_i, qkv_align) || !aligned(k_j, qkv_align) || !aligned(v_j, qkv_align)) return RA_ERR_ALIGN;
+    cudaStream_t stream = static_cast<cudaStream_t>(stream_handle);
+    const Layout L = make_layout(S, n_ring, layout);
+    const int j = (int)ra::ring_block(shard, step, n_ring);
+    // a later step whose whole block lies in the future of every query of the shard adds nothing
+    if (step > 0 && ra::visible_keys(L, causal ? 1 : 0, shard, L.S_loc - 1, j) == 0) return RA_OK;
+
+    const RingWorkspace w = ring_carve(B, H, L, D, causal ? 1 : 0, shard, step, tc);
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    bool own_ws = false;
+    if (ws) {
+        if (workspace_bytes < w.total) return RA_ERR_NO_WORKSPACE;
+        if (reinterpret_cast<uintptr_t>(ws) % kAlign) return RA_ERR_ALIGN;
+    } else {
+        cudaError_t e = cudaMallocAsync(reinterpret_cast<void**>(&ws), w.total, stream);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaMallocAsync(ring step workspace)");
+        own_ws = true;
+    }
+    auto finish = [&](int status) {
+        if (own_ws) {
+            cudaError_t e = cudaFreeAsync(ws, stream);
+            if (e != cudaSuccess && status == RA_OK) status = cuda_fail(e, "cudaFreeAsync(ring step workspace)");
+        }
+        return status;
+    };
+
+    ra::AttnArgs a{};
+    a.L = L;
+    a.B = B;
+    a.H = H;
+    a.D = D;
+    a.causal = causal ? 1 : 0;
+    a.dtype = dtype;
+    a.s_begin = step;
+    a.s_end = step + 1;
+    a.out_mode = ra::kOutPartial;
+    a.local = 1;
+    a.q_shard = shard;
+    a.scale = (float)(1.0 / std::sqrt((double)D));
+    // step 0 starts the running result; later steps write a partial that is merged into it
+    float* O_s = step == 0 ? O_acc : reinterpret_cast<float*>(ws + w.O_s);
+    float* lse_s = step == 0 ? lse_acc : reinterpret_cast<float*>(ws + w.lse_s);
+    a.out = O_s;
+    a.lse = lse_s;
+    cudaError_t e;
+    nvtxRangePushA("ra_ring_step attention");
+    if (tc) {
+        ra::TcLaunch t{};
+        const Layout Lloc{L.S_loc, 1, L.S_loc, RA_LAYOUT_CONTIGUOUS};  // one shard per buffer
+        if ((rc = encode_qkv_map(&t.tm_q, q_i, B, Lloc, H, D, false)) != RA_OK) return nvtx_pop(finish(rc));
+        if ((rc = encode_qkv_map(&t.tm_k, k_j, B, Lloc, H, D, false)) != RA_OK) return nvtx_pop(finish(rc));
+        if ((rc = encode_qkv_map(&t.tm_v, v_j, B, Lloc, H, D, false)) != RA_OK) return nvtx_pop(finish(rc));
+        std::shared_ptr<FlatList> fl;
+        if ((rc = flat_items(B, H, L, D, a.causal, false, &fl, shard, step)) != RA_OK) return nvtx_pop(finish(rc));
+        if (fl->count > 0 && (e = fl->upload(ws + w.items, 0, fl->count, stream)) != cudaSuccess)
+            return nvtx_pop(finish(cuda_fail(e, "work list upload")));
+        if ((e = cudaMemsetAsync(ws + w.counter, 0, sizeof(int), stream)) != cudaSuccess)
+            return nvtx_pop(finish(cuda_fail(e, "work counter reset")));
+        t.items = reinterpret_cast<const int4*>(ws + w.items);
+        t.n_items = (int)fl->count;
+        t.counter = reinterpret_cast<int*>(ws + w.counter);
+        t.grid = std::max(1, std::min(t.n_items, dev.sms - sms_reserved));
+        t.timeout_ns = 2000000000ull;
+        t.status = dev.status;
+        e = ra::launch_attn_tc(a, t, stream);
+    } else {
+        e = ra::launch_attn_simt(q_i, k_j, v_j, a, stream);
+    }
+    nvtxRangePop();
+    if (e != cudaSuccess) return finish(cuda_fail(e, "ring step attention launch"));
+    if (step > 0) {
+        nvtxRangePushA("ra_ring_step merge");
+        e = ra::launch_merge_inplace(O_acc, lse_acc, O_s, lse_s, B * L.S_loc * H, D, stream);
+        nvtxRangePop();
+        if (e != cudaSuccess) return finish(cuda_fail(e, "ring step merge launch"));
+    }
+    return finish(RA_OK);
+}
+
+int ra_ring_finalize(const float* O_acc, const float* lse_acc, void* out, float* lse, int64_t B, int64_t H,
+                     int64_t S_loc, int64_t D, int dtype, void* stream) {
+    if (!O_acc || !lse_acc || !out || !lse) return RA_ERR_INVALID_ARG;
+    if (B < 1 || H < 1 || S_loc < 1 || D < 1 || D > 256) return RA_ERR_INVALID_ARG;
+    if (dtype != RA_DTYPE_FP32 && dtype != RA_DTYPE_BF16) return RA_ERR_INVALID_ARG;
+    auto aligned = [](const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; };
+    if (!aligned(O_acc, 16) || !aligned(out, 16) || !aligned(lse_acc, 4) || !aligned(lse, 4)) return RA_ERR_ALIGN;
+    const Layout Lloc{S_loc, 1, S_loc, RA_LAYOUT_CONTIGUOUS};
+    nvtxRangePushA("ra_ring_finalize");
+    cudaError_t e = ra::launch_merge_final(O_acc, lse_acc, nullptr, nullptr, out, lse, dtype, B, Lloc, H, D,
+                                           static_cast<cudaStream_t>(stream));
+    nvtxRangePop();
+    return e == cudaSuccess ? RA_OK : cuda_fail(e, "ring finalize launch");
 }
 
 const char* ra_status_string(int status) {

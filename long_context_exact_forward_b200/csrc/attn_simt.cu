@@ -47,13 +47,19 @@ __device__ __forceinline__ __nv_bfloat16 from_float<__nv_bfloat16>(float x) { re
 // as fp32 into shared memory, transposed: dst[d * kB + r].  Rows past the shard end and columns
 // d >= D read as zero.  Thread t takes row t % kB and 4 consecutive columns at a time, so
 // consecutive threads write consecutive words and each thread reads whole sectors of its row.
+// Token row of local token a of shard `shard`: natural order through the layout map, or, for a
+// ring step on local buffers, row a of the one-shard buffer.
+__device__ __forceinline__ int64_t token_row(const Layout& L, int local, int64_t b, int64_t shard, int64_t a) {
+    return local ? b * L.S_loc + a : b * L.S + global_position(L, shard, a);
+}
+
 template <typename T, int kDMax, int kB>
-__device__ void load_transposed(float* dst, const T* __restrict__ src, const Layout& L, int64_t b,
+__device__ void load_transposed(float* dst, const T* __restrict__ src, const Layout& L, int local, int64_t b,
                                 int64_t h, int64_t H, int64_t D, int64_t shard, int64_t a0) {
     const int r = threadIdx.x % kB;
     const int64_t a = a0 + r;
     const T* row = nullptr;
-    if (a < L.S_loc) row = src + ((b * L.S + global_position(L, shard, a)) * H + h) * D;
+    if (a < L.S_loc) row = src + (token_row(L, local, b, shard, a) * H + h) * D;
     for (int d4 = 4 * (threadIdx.x / kB); d4 < kDMax; d4 += 4 * (kThreads / kB)) {
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
@@ -65,14 +71,14 @@ __device__ void load_transposed(float* dst, const T* __restrict__ src, const Lay
 
 // Same rows, row-major: dst[r * kDMax + d].  Consecutive threads take consecutive columns.
 template <typename T, int kDMax, int kB>
-__device__ void load_rowmajor(float* dst, const T* __restrict__ src, const Layout& L, int64_t b,
+__device__ void load_rowmajor(float* dst, const T* __restrict__ src, const Layout& L, int local, int64_t b,
                               int64_t h, int64_t H, int64_t D, int64_t shard, int64_t a0) {
     for (int idx = threadIdx.x; idx < kB * kDMax; idx += kThreads) {
         const int r = idx / kDMax, d = idx % kDMax;
         const int64_t a = a0 + r;
         float x = 0.f;
         if (a < L.S_loc && d < D)
-            x = to_float<T>(src[((b * L.S + global_position(L, shard, a)) * H + h) * D + d]);
+            x = to_float<T>(src[(token_row(L, local, b, shard, a) * H + h) * D + d]);
         dst[idx] = x;
     }
 }
@@ -100,14 +106,14 @@ __global__ void __launch_bounds__(kThreads, kDMax <= 128 ? 2 : 1)
     const int64_t D = args.D, H = args.H;
     // heaviest shards first: under the causal mask with the contiguous layout shard i meets i + 1
     // live blocks, so the CTAs of the last shards are launched first (a longest-first order)
-    const int64_t i = L.N - 1 - blockIdx.y;
+    const int64_t i = args.local ? args.q_shard : L.N - 1 - blockIdx.y;
     const int64_t bh = blockIdx.z;
     const int64_t b = bh / H, h = bh % H;
     const int64_t a0 = (int64_t)blockIdx.x * kBQ;
     const int ty = threadIdx.x >> 4, tx = threadIdx.x & 15;
     const int64_t a_last = (a0 + kBQ - 1 < L.S_loc - 1) ? a0 + kBQ - 1 : L.S_loc - 1;
 
-    load_transposed<T, kDMax, kBQ>(Qt, q, L, b, h, H, D, i, a0);
+    load_transposed<T, kDMax, kBQ>(Qt, q, L, args.local, b, h, H, D, i, a0);
 
     float m[4], l[4], o[4][kOC];
 #pragma unroll
@@ -129,8 +135,8 @@ __global__ void __launch_bounds__(kThreads, kDMax <= 128 ? 2 : 1)
         const int64_t n_vis_cta = visible_keys(L, args.causal, i, a_last, j);  // the CTA's widest
         for (int64_t b0 = 0; b0 < n_vis_cta; b0 += kBK) {
             __syncthreads();  // previous tile consumed (and Q loaded on the first pass)
-            load_transposed<T, kDMax, kBK>(Kt, k, L, b, h, H, D, j, b0);
-            load_rowmajor<T, kDMax, kBK>(Vs, v, L, b, h, H, D, j, b0);
+            load_transposed<T, kDMax, kBK>(Kt, k, L, args.local, b, h, H, D, j, b0);
+            load_rowmajor<T, kDMax, kBK>(Vs, v, L, args.local, b, h, H, D, j, b0);
             __syncthreads();
 
             // S block: rows 4ty + r, keys 4tx + c
@@ -221,7 +227,7 @@ __global__ void __launch_bounds__(kThreads, kDMax <= 128 ? 2 : 1)
             }
             if (tx == 0) args.lse[(b * H + h) * L.S + g] = lse;
         } else {
-            const int64_t row = ((b * L.N + i) * L.S_loc + a) * H + h;
+            const int64_t row = args.local ? (b * L.S_loc + a) * H + h : ((b * L.N + i) * L.S_loc + a) * H + h;
             float* dst = static_cast<float*>(args.out) + row * D;
 #pragma unroll
             for (int c = 0; c < kOC; ++c) {
@@ -240,7 +246,7 @@ cudaError_t launch_typed(const void* q, const void* k, const void* v, const Attn
     auto kern = attn_simt_kernel<T, kDMax>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    dim3 grid((unsigned)((a.L.S_loc + kBQ - 1) / kBQ), (unsigned)a.L.N, (unsigned)(a.B * a.H));
+    dim3 grid((unsigned)((a.L.S_loc + kBQ - 1) / kBQ), a.local ? 1u : (unsigned)a.L.N, (unsigned)(a.B * a.H));
     kern<<<grid, kThreads, smem, stream>>>(static_cast<const T*>(q), static_cast<const T*>(k),
                                            static_cast<const T*>(v), a);
     return cudaGetLastError();

@@ -163,7 +163,7 @@ __device__ __forceinline__ ItemGeom item_geom(const AttnArgs& A, const Layout32&
 // map is (token / N, token mod N) and sequences start on multiples of N.
 template <bool kVarlen>
 __device__ __forceinline__ int2 tma_rows(const AttnArgs& A, const ItemGeom& G, int shard, int a) {
-    if (!kVarlen) return make_int2(a, shard);
+    if (!kVarlen) return make_int2(a, A.local ? 0 : shard);
     if (A.varlen_striped) return make_int2(G.base / G.L.N + a, shard);
     return make_int2(G.base + shard * G.L.S_loc + a, 0);
 }
@@ -581,7 +581,8 @@ struct Roles {
             row_dst = static_cast<uint8_t*>(A.out) + (((G.b * S + g) * H + G.h) * kD) * 2;
             lse_dst = A.lse + (G.b * H + G.h) * S + g;
         } else {
-            const int64_t rr = (((int64_t)G.b * G.L.N + G.i) * G.L.S_loc + a) * H + G.h;
+            const int64_t rr = A.local ? ((int64_t)G.b * G.L.S_loc + a) * H + G.h
+                                       : (((int64_t)G.b * G.L.N + G.i) * G.L.S_loc + a) * H + G.h;
             row_dst = static_cast<uint8_t*>(A.out) + rr * kD * 4;
             lse_dst = A.lse + rr;
         }
@@ -699,6 +700,15 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 }  // namespace
+
+cudaError_t preload_attn_tc() {
+    cudaFuncAttributes fa;
+    cudaError_t e = cudaFuncGetAttributes(&fa, attn_tc_kernel<64, false>);
+    if (e == cudaSuccess) e = cudaFuncGetAttributes(&fa, attn_tc_kernel<128, false>);
+    if (e == cudaSuccess) e = cudaFuncGetAttributes(&fa, attn_tc_kernel<64, true>);
+    if (e == cudaSuccess) e = cudaFuncGetAttributes(&fa, attn_tc_kernel<128, true>);
+    return e;
+}
 
 size_t tc_smem_bytes(int64_t D) {
     return (D == 64 ? sizeof(TcSmem<64>) : sizeof(TcSmem<128>)) + 1024;

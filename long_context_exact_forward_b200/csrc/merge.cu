@@ -66,6 +66,8 @@ __global__ void __launch_bounds__(256) merge_inplace_scalar(float* __restrict__ 
 }
 
 // Final merge: rows are shard-major (b, i, a, h); the result goes to natural position g(i, a).
+// With O_s and lse_s null, the running result alone is converted and written (the last step of a
+// ring whose partials were already merged).
 template <typename T>
 __device__ __forceinline__ void store4(T* p, float4 v);
 template <>
@@ -98,15 +100,16 @@ __global__ void __launch_bounds__(256) merge_final(const float* __restrict__ O_r
     const int64_t a = r % L.S_loc, bi = r / L.S_loc;
     const int64_t i = bi % L.N, b = bi / L.N;
     const int64_t g = global_position(L, i, a);
-    const Weights w = merge_weights(lse_r[row], __ldcs(lse_s + row));
+    // without a step partial (lse_s null) the running result is written as it is
+    const Weights w = lse_s ? merge_weights(lse_r[row], __ldcs(lse_s + row)) : Weights{1.f, 0.f, lse_r[row]};
     T* dst = out + ((b * L.S + g) * H + h) * D;
     if (kVec) {
         const float4 x = reinterpret_cast<const float4*>(O_r)[t];
-        const float4 y = __ldcs(reinterpret_cast<const float4*>(O_s) + t);
+        const float4 y = lse_s ? __ldcs(reinterpret_cast<const float4*>(O_s) + t) : make_float4(0.f, 0.f, 0.f, 0.f);
         store4<T>(dst + 4 * c, make_float4(w.wr * x.x + w.ws * y.x, w.wr * x.y + w.ws * y.y,
                                            w.wr * x.z + w.ws * y.z, w.wr * x.w + w.ws * y.w));
     } else {
-        const float x = w.wr * O_r[t] + w.ws * O_s[t];
+        const float x = w.wr * O_r[t] + (lse_s ? w.ws * O_s[t] : 0.f);
         if constexpr (sizeof(T) == 4) {
             dst[c] = x;
         } else {

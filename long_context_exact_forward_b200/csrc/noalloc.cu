@@ -6,13 +6,17 @@
 // allocate device memory at all: code recording a CUDA graph (an allocation inside stream capture
 // either fails or becomes part of the graph), engines that own every byte of the GPU through
 // their own allocator and budget, and latency-critical loops where an allocator call may stall.
-// This entry point serves them: its scratch lives in one fixed array in device memory that the
-// library reserves when it is loaded (NOALLOC_SCRATCH_BYTES on every GPU that loads it, held
-// until the process exits), so the call itself allocates nothing.
+// This entry point serves them: its scratch lives in one fixed array in device memory
+// (RA_NOALLOC_SCRATCH_BYTES), part of the library's device code.  The array comes into being on a
+// device when the library's code is loaded there -- at the first use of the library on that
+// device under CUDA's default lazy module loading, at context creation otherwise -- and stays
+// until the process exits.  The call itself allocates nothing.
 //
 // Rules of use.
-//   * The first call on a device looks up the array's device address (cudaGetSymbolAddress) with
-//     that device current; make that first call before any stream capture.
+//   * The first call on a device, with that device current, looks up the array's device address
+//     (cudaGetSymbolAddress) and loads every kernel this entry point launches (both head-dim
+//     instantiations of the attention kernel, the permute kernels and the list builder), so that
+//     no later call loads module code.  Make that first call before any stream capture.
 //   * Every call on a device shares the one array and leaves its contents behind.  The one part
 //     that must start at zero, the kernel's work counter, is cleared by each call on its stream
 //     (cudaMemsetAsync, no allocation); everything else is rewritten before it is read.  Calls
@@ -35,11 +39,18 @@ using ra::Layout;
 constexpr size_t kScratchBytes = (size_t)RA_NOALLOC_SCRATCH_BYTES;
 constexpr int kTileRows = 128;
 constexpr int kPairRows = 256;
-constexpr int kMaxItemsPerHead = 11264;  // shared-memory tables of the list builder (< 48 KB)
+// The list builder keeps one cost per item of a head and one total per shard in shared memory;
+// it is launched without an opt-in above the default 48 KB of dynamic shared memory, so
+// (items per head + shards) * 4 bytes must stay within 48 KB.
+constexpr size_t kBuilderSmemBytes = 48 * 1024;
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kScratchBytes];
 
-// Device address of g_noalloc_scratch on the current device, looked up once per device.
+__global__ void build_work_list(int4* __restrict__ items, int64_t BH, int64_t H, Layout L, int causal,
+                                int pairs, int by_shard);
+
+// Device address of g_noalloc_scratch on the current device, looked up once per device; the same
+// first call loads every kernel the entry point launches on this device.
 int scratch_address(unsigned char** out) {
     static std::mutex mu;
     static std::map<int, unsigned char*> addr;
@@ -52,6 +63,11 @@ int scratch_address(unsigned char** out) {
         void* p = nullptr;
         e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
         if (e != cudaSuccess) return ra::host_cuda_fail(e, "cudaGetSymbolAddress(noalloc scratch)");
+        cudaFuncAttributes fa;
+        if ((e = cudaFuncGetAttributes(&fa, build_work_list)) != cudaSuccess)
+            return ra::host_cuda_fail(e, "loading the work-list builder");
+        if ((e = ra::preload_attn_tc()) != cudaSuccess) return ra::host_cuda_fail(e, "loading the attention kernel");
+        if ((e = ra::preload_permute()) != cudaSuccess) return ra::host_cuda_fail(e, "loading the permute kernel");
         it = addr.emplace(dev, static_cast<unsigned char*>(p)).first;
     }
     *out = it->second;
@@ -140,9 +156,15 @@ extern "C" int ra_forward_noalloc(const void* q, const void* k, const void* v, v
     const size_t counter_bytes = 256;  // the persistent kernel's work counter, zeroed every call
     const size_t items_bytes = align256((size_t)n_items * sizeof(int4));
     const size_t need = counter_bytes + items_bytes + (permute ? 3 * align256(tensor_bytes) : 0);
-    if (per_head > kMaxItemsPerHead || need > kScratchBytes || n_items > INT32_MAX) {
+    const size_t builder_smem = (size_t)(per_head + L.N) * sizeof(int);
+    if (builder_smem > kBuilderSmemBytes) {
+        ra::host_set_error("ra_forward_noalloc: too many work items per head for the device list "
+                           "builder ((items per head + n_ring) * 4 bytes must stay within 48 KB)");
+        return RA_ERR_NO_WORKSPACE;
+    }
+    if (need > kScratchBytes || n_items > INT32_MAX) {
         ra::host_set_error("ra_forward_noalloc: problem needs more scratch than the fixed "
-                           "RA_NOALLOC_SCRATCH_BYTES array (or more than 11264 work items per head)");
+                           "RA_NOALLOC_SCRATCH_BYTES array");
         return RA_ERR_NO_WORKSPACE;
     }
     unsigned char* scratch = nullptr;
@@ -153,8 +175,7 @@ extern "C" int ra_forward_noalloc(const void* q, const void* k, const void* v, v
     int4* items = reinterpret_cast<int4*>(scratch + counter_bytes);
     cudaError_t e = cudaMemsetAsync(counter, 0, sizeof(int), stream);
     if (e != cudaSuccess) return ra::host_cuda_fail(e, "work counter reset");
-    const size_t smem = (size_t)(per_head + L.N) * sizeof(int);
-    build_work_list<<<1, 1024, smem, stream>>>(items, B * H, H, L, causal ? 1 : 0, pairs,
+    build_work_list<<<1, 1024, builder_smem, stream>>>(items, B * H, H, L, causal ? 1 : 0, pairs,
                                                 ra::plan_groups_by_shard(S, D) ? 1 : 0);
     e = cudaGetLastError();
     if (e != cudaSuccess) return ra::host_cuda_fail(e, "work list launch");

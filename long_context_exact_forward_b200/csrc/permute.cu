@@ -82,4 +82,12 @@ cudaError_t launch_permute(const void* const* src, void* const* dst, int n_tenso
     return cudaGetLastError();
 }
 
+cudaError_t preload_permute() {
+    cudaFuncAttributes fa;
+    cudaError_t e = cudaFuncGetAttributes(&fa, permute_rows_vec16);
+    if (e == cudaSuccess) e = cudaFuncGetAttributes(&fa, permute_rows_elem<float>);
+    if (e == cudaSuccess) e = cudaFuncGetAttributes(&fa, permute_rows_elem<unsigned short>);
+    return e;
+}
+
 }  // namespace ra

@@ -29,6 +29,12 @@ struct AttnArgs {
     // every sequence is split into L.N shards with L.kind.  Null: batch mode (item x = batch b).
     const int2* seqs;
     int varlen_striped;   // packed sequences with the striped layout inside each sequence
+    // One ring step on one device's local buffers (kOutPartial only): q holds query shard
+    // q_shard alone and k, v hold key block (q_shard - s_begin) mod N alone, each [B, S_loc, H, D]
+    // in the layout's local order.  Masks and positions use the true shard indices; addresses use
+    // shard 0 of a one-shard buffer, and the partial rows are local, ((b * S_loc + a) * H + h).
+    int local;
+    int q_shard;
 };
 
 // permute.cu
@@ -37,7 +43,8 @@ cudaError_t launch_permute(const void* const* src, void* const* dst, int n_tenso
                            cudaStream_t stream);
 
 // merge.cu: fold (O_s, lse_s) into (O_r, lse_r) in place, or (final) write the merged result
-// to out (natural order, dtype) and lse natural [B, H, S].
+// to out (natural order, dtype) and lse natural [B, H, S]; launch_merge_final with O_s and lse_s
+// null writes (O_r, lse_r) alone.
 cudaError_t launch_merge_inplace(float* O_r, float* lse_r, const float* O_s, const float* lse_s,
                                  int64_t rows, int64_t D, cudaStream_t stream);
 cudaError_t launch_merge_final(const float* O_r, const float* lse_r, const float* O_s,
@@ -60,6 +67,12 @@ struct TcLaunch {
     int* status;           // device status word, set to RA_ERR_DEVICE_TIMEOUT on a give-up
 };
 size_t tc_smem_bytes(int64_t D);
+
+// Load the module code of every instantiation of a kernel family on the current device now
+// (cudaFuncGetAttributes forces it), so that a later launch -- possibly inside a stream capture --
+// never triggers lazy module loading.
+cudaError_t preload_attn_tc();
+cudaError_t preload_permute();
 
 // api.cu: host helpers shared by the entry points.
 int host_check_shape(int64_t B, int64_t H, int64_t S, int64_t D, int n_ring, int layout, int dtype);

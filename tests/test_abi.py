@@ -133,3 +133,33 @@ def test_varlen_workspace_size_and_options_validate_on_the_host():
     need = ra.varlen_workspace_size(cu, H, D, N, "zigzag")
     assert ex(ws=FAKE + 16, nbytes=need) == -3        # workspace not 256-byte aligned
     assert ex(ws=FAKE, nbytes=need - 1) == -5         # workspace too small
+
+
+def test_ring_step_validates_before_any_cuda_call():
+    lib = ra.lib()
+
+    def step(S=64, n_ring=4, shard=0, step=0, reserved=0, q=FAKE, O=FAKE, layout=1):
+        return lib.ra_ring_step(q, FAKE, FAKE, O, FAKE, 1, 2, S, 64, n_ring, 1, layout, 1, shard, step, reserved,
+                                None, 0, None)
+    assert step(S=63) == -2             # S % n_ring
+    assert step(shard=4) == -1          # query shard outside the ring
+    assert step(shard=-1) == -1
+    assert step(step=4) == -1           # ring step outside [0, n_ring)
+    assert step(reserved=-1) == -1
+    assert step(q=0) == -1
+    assert step(O=FAKE + 8) == -3       # running output must be 16-byte aligned
+    assert step(layout=5) == -1
+    assert lib.ra_ring_finalize(FAKE, FAKE, FAKE, FAKE, 1, 2, 0, 64, 1, None) == -1
+    assert lib.ra_ring_finalize(FAKE, FAKE, FAKE + 4, FAKE, 1, 2, 16, 64, 1, None) == -3
+
+
+def test_ring_step_workspace_covers_every_shard_and_step():
+    B, H, D, N = 2, 3, 128, 8
+    S = N * 1000
+    n = ra.ring_step_workspace_size(B, H, S, D, N, True, "zigzag", 1)
+    a256 = lambda x: -(-x // 256) * 256
+    rows = B * (S // N) * H
+    pairs = -(-(S // N) // 256)
+    assert n == 256 + a256(B * H * pairs * 16) + a256(rows * D * 4) + a256(rows * 4)
+    simt = ra.ring_step_workspace_size(B, H, S, 40, N, True, "zigzag", 0)
+    assert simt == a256(rows * 40 * 4) + a256(rows * 4)

@@ -1,8 +1,14 @@
 """GPU parity at full workload sizes, on sampled query rows the oracle computes one by one.
 
-Rows per head: row 0, row S-1, the first and last token of every shard (under the layout run),
-then uniform draws without replacement (numpy default_rng(1000 + h)) up to RA_ROWS_PER_HEAD
-(default 128; 4096 reproduces the full per-head check).  Tolerances as in test_gpu_parity.
+Every large workload is checked on 4096 rows per head (RA_ROWS_PER_HEAD overrides the count):
+row 0, row S-1, the first and last token of every shard under EVERY layout the workload is run
+with, then uniform draws without replacement (numpy default_rng(1000 + h)) until 4096 distinct
+rows.  The oracle depends only on the inputs and the mask, not on the layout or the kernel
+variant, so it is computed once per (workload, causal) and every run of that workload -- each
+layout, fused and per-step -- is compared with the same fp64 rows.  That keeps the oracle's cost
+(about 4.4e12 flops for s128k and for s1m) to one pass per workload.
+
+Bars as in test_gpu_parity: max |err| <= 2e-2, mean |err| <= 2e-3, |lse err| <= 1e-3.
 """
 import os
 
@@ -16,9 +22,10 @@ from long_context_exact_forward_b200 import inputs
 
 pytestmark = pytest.mark.gpu
 
-ROWS = int(os.environ.get("RA_ROWS_PER_HEAD", "128"))
+ROWS = int(os.environ.get("RA_ROWS_PER_HEAD", "4096"))
 THREADS = os.cpu_count() or 1
 
+# (workload, causal, layout, variant); runs of one (workload, causal) share one oracle pass
 CASES = [
     ("s32k", False, "contiguous", "fused"),
     ("s32k", True, "contiguous", "fused"),
@@ -27,34 +34,55 @@ CASES = [
     ("s128k", True, "striped", "fused"),
     ("s128k", True, "zigzag", "fused"),
     ("s128k", True, "striped", "per_step"),
+    ("s128k", True, "zigzag", "per_step"),
     ("s1m", True, "striped", "fused"),
+    ("s1m", True, "striped", "per_step"),
 ]
 
+_REFERENCE = {}
 
-def boundary_rows(S, N, layout):
-    pos = oracle.layout_positions(S, N, layout)
-    return [0, S - 1, *pos[:, 0].tolist(), *pos[:, -1].tolist()]
+
+def boundary_rows(S, N, layouts):
+    """Row 0, row S-1 and the first and last token of every shard under each layout."""
+    rows = [0, S - 1]
+    for layout in layouts:
+        pos = oracle.layout_positions(S, N, layout)
+        rows += pos[:, 0].tolist() + pos[:, -1].tolist()
+    return rows
+
+
+def reference(name, causal):
+    """(rows [H, n], out [H, n, D], lse [H, n]) of the fp64 oracle for a workload, computed once."""
+    key = (name, causal)
+    if key not in _REFERENCE:
+        _REFERENCE.clear()  # workloads run one after another; keep one in host memory
+        w = inputs.WORKLOADS[name]
+        layouts = sorted({c[2] for c in CASES if c[0] == name})
+        rows = inputs.sample_rows(w.S, w.H, ROWS, boundary_rows(w.S, w.n_ring, layouts))
+        q, k, v = inputs.workload_qkv(w)
+        qc, kc, vc = q.cpu(), k.cpu(), v.cpu()
+        del q, k, v
+        ref, ref_lse = oracle.attention(qc, kc, vc, causal, rows=rows, threads=THREADS)
+        _REFERENCE[key] = (rows, ref[0], ref_lse[0])
+    return _REFERENCE[key]
 
 
 @pytest.mark.parametrize("name, causal, layout, variant", CASES)
 def test_full_size_sampled_rows(name, causal, layout, variant):
+    rows, ref, ref_lse = reference(name, causal)
     w = inputs.WORKLOADS[name]
     q, k, v = inputs.workload_qkv(w)
     out, lse = ra.forward(q, k, v, w.n_ring, causal, layout, variant=variant)
     torch.cuda.synchronize()
     assert ra.get_device_status() == 0
-    rows = inputs.sample_rows(w.S, w.H, ROWS, boundary_rows(w.S, w.n_ring, layout))
     idx = torch.from_numpy(rows).cuda()
     got = torch.stack([out[0, idx[h], h].float() for h in range(w.H)]).cpu().double().numpy()
     got_lse = torch.gather(lse[0], 1, idx).cpu().double().numpy()
-    del out
-    qc, kc, vc = q.cpu(), k.cpu(), v.cpu()
-    del q, k, v
-    ref, ref_lse = oracle.attention(qc, kc, vc, causal, rows=rows, threads=THREADS)
-    err = np.abs(got - ref[0])
-    lerr = np.abs(got_lse - ref_lse[0])
+    err = np.abs(got - ref)
+    lerr = np.abs(got_lse - ref_lse)
     print(f"{name} causal={causal} {layout} {variant}: rows/head={rows.shape[1]} "
           f"max={err.max():.3e} mean={err.mean():.3e} lse={lerr.max():.3e}")
+    assert rows.shape[1] == min(ROWS, w.S)
     assert np.isfinite(got).all()
     assert err.max() <= 2e-2 and err.mean() <= 2e-3 and lerr.max() <= 1e-3
 

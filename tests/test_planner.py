@@ -156,3 +156,13 @@ def test_random_shapes_layouts_and_tiles_against_brute_force():
                             assert allowed.all() and ka.size == tile, (S, N, layout, causal, tile, i, s, qt, kt)
                         else:
                             assert allowed.any(), (S, N, layout, causal, tile, i, s, qt, kt)
+
+
+def test_plan_cache_keeps_lists_right_past_its_bound():
+    """The planner's caches hold a bounded number of shapes (least recently used dropped): a sweep
+    over more shapes than that leaves every list, recomputed or cached, as it was."""
+    first = ra.plan_items(1, 2, 4096, 4, True, "striped").copy()
+    for n in range(1, 90):  # more distinct shapes than the cache keeps
+        ra.plan_items(1, 1, 256 * n, 2, True, "contiguous")
+    again = ra.plan_items(1, 2, 4096, 4, True, "striped")
+    assert np.array_equal(first, again)
