@@ -56,7 +56,7 @@ UNIT = "TFLOP/s"
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 # DRAM bytes (read + write) per attention launch on s128k striped, from an ncu capture of the
-# 4-head case scaled by heads (profiles/attn_tc_fused_s128k_striped.md); valid only while
+# 4-head case (dram__bytes_read.sum + dram__bytes_write.sum) scaled by heads; valid only while
 # the sha256 of the TRAFFIC_SOURCES files, concatenated in that order, starts with the recorded
 # prefix -- otherwise traffic is null.
 TRAFFIC_RECORD = {"source_sha256_prefix": "19d20a87f3c3cd75", "bytes_per_launch": 3.634440e9 * 8}
@@ -260,6 +260,7 @@ def config_dict(w, args):
                     f"{args.layout} layout",
         "B": w.B, "H": w.H, "S": w.S, "D": w.D, "n_ring": w.n_ring, "causal": causal_of(args),
         "layout": args.layout, "variant": args.variant, "kernel": args.kernel,
+        **({"steps_per_launch": args.steps_per_launch} if args.variant == "per_step" else {}),
         "l2": f"inputs (3 x B*S*H*D {args.dtype}) larger than the 126 MB L2; no flush"
               if 3 * w.B * w.S * w.H * w.D * (4 if args.dtype == "fp32" else 2) > 126e6
               else "inputs smaller than the 126 MB L2 (kernel-level runs; not the headline)",
@@ -337,7 +338,7 @@ def run_ours(args, w):
 
     def step(ev=None):
         ra.forward(q, k, v, N, causal, args.layout, variant=args.variant, kernel=args.kernel, out=out,
-                   lse=lse, workspace=ws, stream=stream, events=ev)
+                   lse=lse, workspace=ws, stream=stream, events=ev, steps_per_launch=args.steps_per_launch)
 
     if args.varlen:
         lengths = varlen_lengths(S, N, w.seed)
@@ -425,7 +426,7 @@ def run_ours(args, w):
                 if st >= 2:
                     stream.wait_event(ev_free_out[b])
                 ra.forward(dq[b][0], dq[b][1], dq[b][2], N, causal, args.layout, variant=args.variant, kernel=args.kernel,
-                           out=do[b], lse=dl[b], workspace=ws, stream=stream)
+                           out=do[b], lse=dl[b], workspace=ws, stream=stream, steps_per_launch=args.steps_per_launch)
                 ev_free_in[b].record(stream)
                 ev_done[b].record(stream)
                 with torch.cuda.stream(d2h):
@@ -448,7 +449,7 @@ def run_ours(args, w):
             for dst, src in zip(dq[0], (qh, kh, vh)):
                 dst.copy_(src, non_blocking=True)
             ra.forward(dq[0][0], dq[0][1], dq[0][2], N, causal, args.layout, variant=args.variant, kernel=args.kernel,
-                       out=do[0], lse=dl[0], workspace=ws, stream=stream)
+                       out=do[0], lse=dl[0], workspace=ws, stream=stream, steps_per_launch=args.steps_per_launch)
             oh[0].copy_(do[0], non_blocking=True)
             lh[0].copy_(dl[0], non_blocking=True)
 
@@ -523,11 +524,14 @@ def run_ours(args, w):
                                     "sample": f"{min(args.cpu_rows_single, w.S)} query rows of head 0 of "
                                               f"{w.name} ({mask_word(args)}), {f1:.3e} flops in {dt1:.1f} s"}
 
-    # our kernels per step: the zigzag permute (striped and contiguous are read in place) and the
-    # attention launch(es) -- per-step: N attention launches and N - 1 merges (2 kernels each,
-    # the last one a single final merge)
-    launches_per_step = (1 if args.layout == "zigzag" else 0) + (
-        1 if args.variant in ("fused", "auto") else N + 2 * (N - 2) + 1)
+    # our kernels per step: the zigzag permute (striped and contiguous are read in place, and the
+    # CUDA-core kernel reads natural order) and the attention launch(es) -- with chunks of C ring
+    # steps per launch: ceil(N / C) attention launches and one merge after each but the first
+    # (2 kernels each, the last one a single final merge)
+    chunk = ra.steps_per_launch(S, D, N, args.layout, 0 if fp32 else 1, args.variant, args.steps_per_launch)
+    n_att = -(-N // chunk)
+    launches_per_step = (1 if args.layout == "zigzag" and args.kernel == "tc" else 0) + (
+        1 if n_att == 1 else n_att + 2 * (n_att - 2) + 1)
     if args.backward:
         # Delta, dq, dk/dv; the tensor-core kernels read zigzag from one shard-major permute launch
         tc_bwd = args.bwd_kernel == "tc" or (args.bwd_kernel == "auto" and args.dtype == "bf16" and D in (64, 128))
@@ -557,7 +561,9 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="s128k", choices=sorted(inputs.WORKLOADS))
     ap.add_argument("--layout", default="striped", choices=["contiguous", "striped", "zigzag"])
-    ap.add_argument("--variant", default="fused", choices=["fused", "per_step"])
+    ap.add_argument("--variant", default="fused", choices=["fused", "per_step", "auto"])
+    ap.add_argument("--steps-per-launch", type=int, default=0,
+                    help="per_step variant: ring steps covered by each attention launch (0 = one)")
     ap.add_argument("--heads", type=int, default=0, help="override the head count (profiling runs)")
     ap.add_argument("--kernel", default="tc", choices=["tc", "simt"],
                     help="tc: the tcgen05 kernel (the headline); simt: the fp32 CUDA-core kernel")

@@ -61,10 +61,15 @@ enum ra_dtype { RA_DTYPE_FP32 = 0, RA_DTYPE_BF16 = 1 };
 /* Kernel path for ra_forward_ex.
  *   RA_VARIANT_FUSED:    one persistent launch walks all n_ring steps per query tile and keeps the
  *                        running (m, l, O) on chip (ultralytics.com toy loop structure).
- *   RA_VARIANT_PER_STEP: one attention launch per ring step writes a partial (O_s, lse_s); an
- *                        HBM-bound merge launch folds it into the running (O, lse) with the
- *                        log-sum-exp form of the merge identities.
- *   RA_VARIANT_AUTO:     FUSED. */
+ *   RA_VARIANT_PER_STEP: each attention launch covers ra_options.steps_per_launch ring steps (0 or
+ *                        1: one step, the pages' per-device loop) and writes a partial (O_s,
+ *                        lse_s); an HBM-bound merge launch folds it into the running (O, lse) with
+ *                        the log-sum-exp form of the merge identities.
+ *   RA_VARIANT_AUTO:     FUSED while one head's keys and values (2*S*D*esize bytes) fit in 96 MB of
+ *                        the 126 MB L2; beyond that, PER_STEP with as many steps per launch as keep
+ *                        a launch's keys and values per head within 96 MB (a fused item walks every
+ *                        key/value block of its head, and CTAs running at their own pace then spread
+ *                        over more blocks than L2 holds). */
 enum ra_variant { RA_VARIANT_AUTO = 0, RA_VARIANT_FUSED = 1, RA_VARIANT_PER_STEP = 2 };
 
 /* Kernel family for ra_forward_ex.
@@ -99,6 +104,8 @@ typedef struct ra_options {
     int debug;               /* enum ra_debug */
     void* attn_events[2];    /* optional cudaEvent_t pair recorded on `stream` right before the
                                 first and right after the last attention-kernel launch */
+    int steps_per_launch;    /* RA_VARIANT_PER_STEP: ring steps per attention launch (0 = 1; values
+                                above n_ring are n_ring); ignored by the other variants; >= 0 */
 } ra_options;
 
 /* ra_forward: exact attention as described above, with the defaults of ra_options (variant AUTO,
@@ -115,9 +122,19 @@ RA_API int ra_forward_ex(const void* q, const void* k, const void* v, void* out,
                   void* stream, const ra_options* opt);
 
 /* ra_workspace_size: bytes of caller workspace ra_forward_ex needs for these arguments and the
- * given variant/kernel (enum values as in ra_options), written to *bytes.  Host only. */
+ * given variant/kernel (enum values as in ra_options), written to *bytes.  Host only.  For
+ * RA_VARIANT_PER_STEP the size covers every steps_per_launch; for RA_VARIANT_AUTO it is the size of
+ * the path AUTO takes for these arguments.  (The pages define no such call; the kernel argument
+ * and the status return with the size in *bytes let the size depend on the kernel choice and
+ * report a bad shape the same way as the other calls.) */
 RA_API int ra_workspace_size(int64_t B, int64_t H, int64_t S, int64_t D, int n_ring, int causal,
                       int layout, int dtype, int variant, int kernel, size_t* bytes);
+
+/* ra_steps_per_launch (host only): the ring steps each attention launch of ra_forward_ex covers for
+ * these arguments, variant and ra_options.steps_per_launch, written to *chunk (n_ring: one fused
+ * launch; below n_ring: ceil(n_ring / *chunk) launches with a merge after each but the first). */
+RA_API int ra_steps_per_launch(int64_t S, int64_t D, int n_ring, int layout, int dtype, int variant,
+                               int steps_per_launch, int* chunk);
 
 /* ra_permute: gather x [B, S, H, D] (natural order) into shard-major y [B, n_ring, S_loc, H, D]
  * where y[b, i, a] = x[b, g(i, a)] under `layout` (the per-shard chunks of the pages' sequence

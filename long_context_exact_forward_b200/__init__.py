@@ -63,6 +63,7 @@ class Options(ctypes.Structure):
         ("timeout_ns", ctypes.c_uint64),
         ("debug", ctypes.c_int),
         ("attn_events", ctypes.c_void_p * 2),
+        ("steps_per_launch", ctypes.c_int),
     ]
 
 
@@ -101,6 +102,7 @@ def lib():
         L.ra_ring_step_workspace_size.argtypes = [i64, i64, i64, i64, ci, ci, ci, ci,
                                                   ctypes.POINTER(ctypes.c_size_t)]
         L.ra_ring_finalize.argtypes = [vp, vp, vp, vp, i64, i64, i64, i64, ci, vp]
+        L.ra_steps_per_launch.argtypes = [i64, i64, ci, ci, ci, ci, ci, ctypes.POINTER(ctypes.c_int)]
         L.ra_layout_positions.argtypes = [i64, ci, ci, vp]
         L.ra_plan_tiles.argtypes = [i64, ci, ci, ci, ci, vp]
         L.ra_plan_items.argtypes = [i64, i64, i64, i64, ci, ci, ci, vp, i64, ctypes.POINTER(ctypes.c_int64)]
@@ -115,7 +117,7 @@ def lib():
                      "ra_unpermute", "ra_merge_partials", "ra_layout_positions", "ra_plan_tiles",
                      "ra_plan_items", "ra_get_device_status", "ra_backward", "ra_backward_ex", "ra_rope", "ra_forward_varlen",
                      "ra_forward_varlen_ex", "ra_varlen_workspace_size", "ra_ring_step",
-                     "ra_ring_step_workspace_size", "ra_ring_finalize"):
+                     "ra_ring_step_workspace_size", "ra_ring_finalize", "ra_steps_per_launch"):
             getattr(L, name).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -190,13 +192,15 @@ def workspace_size(B, H, S, D, n_ring, causal, layout, dtype_code, variant="auto
 
 
 def forward(q, k, v, n_ring, causal=True, layout="contiguous", *, variant="auto", kernel="auto",
-            out=None, lse=None, workspace=None, stream=None, events=None, timeout_ns=0, debug=0):
+            out=None, lse=None, workspace=None, stream=None, events=None, timeout_ns=0, debug=0,
+            steps_per_launch=0):
     """Exact attention of q, k, v ([B, S, H, D], CUDA, fp32 or bf16) over an n_ring virtual ring.
 
     Returns (out [B, S, H, D] in q's dtype, lse [B, H, S] fp32).  `workspace` is an optional
     uint8 CUDA tensor of at least workspace_size(...) bytes (otherwise the library allocates
     stream-ordered); `events` an optional pair of torch.cuda.Event recorded around the attention
-    kernel launches on `stream`.
+    kernel launches on `stream`.  `steps_per_launch`: ring steps per attention launch of the
+    per_step variant (0 = one).
     """
     torch = _torch()
     _check_cuda(q, k, v)
@@ -214,6 +218,7 @@ def forward(q, k, v, n_ring, causal=True, layout="contiguous", *, variant="auto"
     opt = Options()
     opt.variant = VARIANTS[variant]
     opt.kernel = KERNELS[kernel]
+    opt.steps_per_launch = int(steps_per_launch)
     if workspace is not None:
         _check_cuda(q, workspace)
         opt.workspace = workspace.data_ptr()
@@ -234,6 +239,16 @@ def forward(q, k, v, n_ring, causal=True, layout="contiguous", *, variant="auto"
                                  ctypes.byref(opt))
     _check(rc, "ra_forward_ex")
     return out, lse
+
+
+def steps_per_launch(S, D, n_ring, layout, dtype_code, variant="auto", steps=0):
+    """Ring steps each attention launch of forward() covers for these arguments (ra_steps_per_launch):
+    n_ring means one fused launch."""
+    n = ctypes.c_int(0)
+    _clear_error()
+    _check(lib().ra_steps_per_launch(S, D, int(n_ring), LAYOUTS[layout], dtype_code, VARIANTS[variant], int(steps),
+                                     ctypes.byref(n)), "ra_steps_per_launch")
+    return n.value
 
 
 def forward_noalloc(q, k, v, n_ring, causal=True, layout="contiguous", *, out=None, lse=None,

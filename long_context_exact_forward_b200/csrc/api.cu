@@ -286,10 +286,10 @@ struct FlatList {
 
 struct FlatKey {
     PlanKey plan;
-    bool per_step;
+    int chunk;  // ring steps per attention launch (N: one fused launch)
     int device;
     bool operator<(const FlatKey& o) const {
-        return std::tie(plan, per_step, device) < std::tie(o.plan, o.per_step, o.device);
+        return std::tie(plan, chunk, device) < std::tie(o.plan, o.chunk, o.device);
     }
 };
 
@@ -298,26 +298,27 @@ LruCache<FlatKey, FlatList>& flat_cache() {
     return *cache;
 }
 
-// shard >= 0: the list of that query shard for the single step s_begin (a ring step on local
-// buffers); otherwise every shard, for all steps (fused) or one list per step (per_step).
-int flat_items(int64_t B, int64_t H, const Layout& L, int64_t D, int causal, bool per_step,
+// shard >= 0: the list of that query shard for the single step `step` (a ring step on local
+// buffers); otherwise every shard, one list per launch of `chunk` ring steps (chunk = N: the single
+// list of the fused launch; the last launch takes the steps that remain).
+int flat_items(int64_t B, int64_t H, const Layout& L, int64_t D, int causal, int chunk,
                std::shared_ptr<FlatList>* out, int shard = -1, int step = 0) {
     int device = 0;
     cudaError_t e = cudaGetDevice(&device);
     if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
     const PlanKey pk = shard >= 0 ? PlanKey{B, H, L.S, (int)L.N, causal, L.kind, step, step + 1, D, shard}
                                   : PlanKey{B, H, L.S, (int)L.N, causal, L.kind, 0, (int)L.N, D, -1};
-    const FlatKey key{pk, per_step, device};
+    if (shard >= 0) chunk = 1;
+    const FlatKey key{pk, chunk, device};
     if ((*out = flat_cache().get(key))) return RA_OK;
     auto f = std::make_shared<FlatList>();
     std::vector<int4> flat;
-    const int n_lists = (per_step && shard < 0) ? (int)L.N : 1;
-    for (int s = 0; s < n_lists; ++s) {
+    const int n_lists = shard >= 0 ? 1 : (int)((L.N + chunk - 1) / chunk);
+    for (int c = 0; c < n_lists; ++c) {
         f->offsets.push_back((int)flat.size());
-        std::shared_ptr<const ItemList> items =
-            shard >= 0 ? plan_items(B, H, L, D, causal, step, step + 1, shard)
-            : per_step ? plan_items(B, H, L, D, causal, s, s + 1)
-                       : plan_items(B, H, L, D, causal, 0, (int)L.N);
+        const int s0 = c * chunk, s1 = std::min<int>((int)L.N, s0 + chunk);
+        std::shared_ptr<const ItemList> items = shard >= 0 ? plan_items(B, H, L, D, causal, step, step + 1, shard)
+                                                           : plan_items(B, H, L, D, causal, s0, s1);
         for (const PlanItem& x : *items) flat.push_back(make_int4(x.b, x.h, x.i, x.p));
     }
     f->offsets.push_back((int)flat.size());
@@ -340,24 +341,48 @@ struct Workspace {
     size_t qp = 0, kp = 0, vp = 0;  // permuted q, k, v
     size_t O_run = 0, lse_run = 0, O_step = 0, lse_step = 0;
     bool permute = false, per_step = false;
+    int chunk = 1, n_launches = 1;  // ring steps per attention launch, and the launches
     size_t total = 0;
 };
 
+// Ring steps per attention launch.  FUSED: all N in one launch.  PER_STEP: `steps_per_launch`
+// (0 means 1), at most N.  AUTO: fused while one head's keys and values fit comfortably in L2;
+// beyond that, launches of as many steps as keep a launch's keys and values per head within the
+// same budget, evened out over the N steps.  The reason: a fused work item walks every key/value
+// block of its head, and when those do not fit in L2 the CTAs running together (each on its own
+// item, at its own pace) spread over more blocks than L2 holds; a launch that covers a few steps
+// keeps the blocks its CTAs read together in L2, for the price of one merge of partial results
+// per extra launch.
+constexpr int64_t kFusedKvBudget = int64_t(96) << 20;
+
+int launch_chunk(const Layout& L, int64_t D, int dtype, int variant, int requested) {
+    const int N = (int)L.N;
+    if (variant == RA_VARIANT_FUSED) return N;
+    if (variant == RA_VARIANT_PER_STEP) return std::min(N, std::max(1, requested));
+    const int64_t esize = dtype == RA_DTYPE_BF16 ? 2 : 4;
+    const int64_t block_kv = 2 * L.S_loc * D * esize;  // one key/value block of one head
+    if (block_kv * N <= kFusedKvBudget) return N;
+    const int64_t fit = std::max<int64_t>(1, kFusedKvBudget / std::max<int64_t>(1, block_kv));
+    const int64_t launches = (N + fit - 1) / fit;
+    return (int)((N + launches - 1) / launches);
+}
+
 Workspace carve(int64_t B, int64_t H, const Layout& L, int64_t D, int causal, int dtype,
-                bool per_step, Kernel kernel) {
+                int chunk, Kernel kernel) {
     Workspace w;
     size_t off = 0;
     const size_t esize = dtype == RA_DTYPE_BF16 ? 2 : 4;
     const size_t elems = (size_t)(B * L.S * H * D);
-    w.per_step = per_step && L.N > 1;
+    w.chunk = std::max(1, std::min<int>(chunk, (int)L.N));
+    w.n_launches = (int)((L.N + w.chunk - 1) / w.chunk);
+    w.per_step = w.n_launches > 1;
     if (kernel == kTC) {
-        if (w.per_step) {
-            for (int s = 0; s < (int)L.N; ++s) w.n_items_total += plan_items(B, H, L, D, causal, s, s + 1)->size();
-        } else {
-            w.n_items_total = plan_items(B, H, L, D, causal, 0, (int)L.N)->size();
+        for (int c = 0; c < w.n_launches; ++c) {
+            const int s0 = c * w.chunk, s1 = std::min<int>((int)L.N, s0 + w.chunk);
+            w.n_items_total += plan_items(B, H, L, D, causal, s0, s1)->size();
         }
         w.counters = off;
-        w.n_counters = w.per_step ? (size_t)L.N : 1;
+        w.n_counters = (size_t)w.n_launches;
         off = align_up(off + w.n_counters * sizeof(int));
         w.items = off;
         off = align_up(off + w.n_items_total * sizeof(int4));
@@ -463,14 +488,15 @@ int run_forward(const Call& c, const ra_options& opt) {
         (reinterpret_cast<uintptr_t>(c.lse) & 3u))
         return RA_ERR_ALIGN;
     if (opt.variant < RA_VARIANT_AUTO || opt.variant > RA_VARIANT_PER_STEP) return RA_ERR_INVALID_ARG;
+    if (opt.steps_per_launch < 0) return RA_ERR_INVALID_ARG;
     DeviceInfo dev;
     if ((rc = device_info(&dev)) != RA_OK) return rc;
     Kernel kernel;
     if ((rc = select_kernel(c, opt.kernel, dev, &kernel)) != RA_OK) return rc;
 
     const Layout L = make_layout(c.S, c.n_ring, c.layout);
-    const bool per_step = (opt.variant == RA_VARIANT_PER_STEP);
-    const Workspace w = carve(c.B, c.H, L, c.D, c.causal, c.dtype, per_step, kernel);
+    const int chunk = launch_chunk(L, c.D, c.dtype, opt.variant, opt.steps_per_launch);
+    const Workspace w = carve(c.B, c.H, L, c.D, c.causal, c.dtype, chunk, kernel);
     uint8_t* ws = static_cast<uint8_t*>(opt.workspace);
     bool own_ws = false;
     if (ws) {
@@ -523,7 +549,7 @@ int run_forward(const Call& c, const ra_options& opt) {
         if ((rc = encode_qkv_map(&tc.tm_v, v, c.B, L, c.H, c.D, striped_natural)) != RA_OK) return finish(rc);
         // upload the work list(s) from the cached pinned copy
         std::shared_ptr<FlatList> fl;
-        if ((rc = flat_items(c.B, c.H, L, c.D, args.causal, w.per_step, &fl)) != RA_OK) return finish(rc);
+        if ((rc = flat_items(c.B, c.H, L, c.D, args.causal, w.chunk, &fl)) != RA_OK) return finish(rc);
         step_item_offset = fl->offsets;
         if (fl->count > 0 && (e = fl->upload(ws + w.items, 0, fl->count, c.stream)) != cudaSuccess)
             return finish(cuda_fail(e, "work list upload"));
@@ -543,7 +569,7 @@ int run_forward(const Call& c, const ra_options& opt) {
         a.lse = lse;
         if (kernel == kTC) {
             ra::TcLaunch t = tc;
-            const int list = w.per_step ? s_begin : 0;
+            const int list = s_begin / w.chunk;
             t.items = reinterpret_cast<const int4*>(ws + w.items) + step_item_offset[list];
             t.n_items = step_item_offset[list + 1] - step_item_offset[list];
             t.grid = std::max(1, std::min(t.n_items, dev.sms));
@@ -566,18 +592,21 @@ int run_forward(const Call& c, const ra_options& opt) {
         float* O_step = reinterpret_cast<float*>(ws + w.O_step);
         float* lse_step = reinterpret_cast<float*>(ws + w.lse_step);
         const int64_t rows = c.B * c.S * c.H;
-        nvtxRangePushA("ra_forward attention (ring step 0)");
-        e = attention(0, 1, ra::kOutPartial, O_run, lse_run);
+        // launch k covers ring steps [k * chunk, min(N, (k + 1) * chunk)); its partial result is
+        // merged into the running one, the last merge writing out and lse in natural order
+        nvtxRangePushA("ra_forward attention (first ring steps)");
+        e = attention(0, std::min<int>(w.chunk, (int)L.N), ra::kOutPartial, O_run, lse_run);
         nvtxRangePop();
         if (e != cudaSuccess) return finish(cuda_fail(e, "attention launch (step 0)"));
-        for (int s = 1; s < (int)L.N; ++s) {
-            nvtxRangePushA("ra_forward attention (ring step)");
-            e = attention(s, s + 1, ra::kOutPartial, O_step, lse_step);
+        for (int s = w.chunk; s < (int)L.N; s += w.chunk) {
+            const int s_end = std::min<int>((int)L.N, s + w.chunk);
+            nvtxRangePushA("ra_forward attention (ring steps)");
+            e = attention(s, s_end, ra::kOutPartial, O_step, lse_step);
             nvtxRangePop();
             if (e != cudaSuccess) return finish(cuda_fail(e, "attention launch (step)"));
             // the last merge also unpermutes: it writes out and lse in natural order
-            nvtxRangePushA(s + 1 < (int)L.N ? "ra_forward merge" : "ra_forward merge + unpermute");
-            if (s + 1 < (int)L.N)
+            nvtxRangePushA(s_end < (int)L.N ? "ra_forward merge" : "ra_forward merge + unpermute");
+            if (s_end < (int)L.N)
                 e = ra::launch_merge_inplace(O_run, lse_run, O_step, lse_step, rows, c.D, c.stream);
             else
                 e = ra::launch_merge_final(O_run, lse_run, O_step, lse_step, c.out, c.lse, c.dtype, c.B,
@@ -644,9 +673,22 @@ int ra_workspace_size(int64_t B, int64_t H, int64_t S, int64_t D, int n_ring, in
     if (variant < RA_VARIANT_AUTO || variant > RA_VARIANT_PER_STEP) return RA_ERR_INVALID_ARG;
     if (kernel < RA_KERNEL_AUTO || kernel > RA_KERNEL_SIMT) return RA_ERR_INVALID_ARG;
     // Host-only: the tensor-core layout is assumed whenever it could apply, which is never smaller.
+    // PER_STEP is sized for one step per launch, which covers any steps_per_launch (fewer
+    // launches need fewer counters and lists); AUTO is sized for the chunk it picks.
     const bool tc = (kernel != RA_KERNEL_SIMT) && dtype == RA_DTYPE_BF16 && (D == 64 || D == 128);
     const Layout L = make_layout(S, n_ring, layout);
-    *bytes = carve(B, H, L, D, causal ? 1 : 0, dtype, variant == RA_VARIANT_PER_STEP, tc ? kTC : kSIMT).total;
+    const int chunk = launch_chunk(L, D, dtype, variant, 1);
+    *bytes = carve(B, H, L, D, causal ? 1 : 0, dtype, chunk, tc ? kTC : kSIMT).total;
+    return RA_OK;
+}
+
+int ra_steps_per_launch(int64_t S, int64_t D, int n_ring, int layout, int dtype, int variant, int steps_per_launch,
+                        int* chunk) {
+    if (!chunk) return RA_ERR_INVALID_ARG;
+    const int rc = check_shape(1, 1, S, D, n_ring, layout, dtype);
+    if (rc != RA_OK) return rc;
+    if (variant < RA_VARIANT_AUTO || variant > RA_VARIANT_PER_STEP || steps_per_launch < 0) return RA_ERR_INVALID_ARG;
+    *chunk = launch_chunk(make_layout(S, n_ring, layout), D, dtype, variant, steps_per_launch);
     return RA_OK;
 }
 

@@ -163,3 +163,23 @@ def test_ring_step_workspace_covers_every_shard_and_step():
     assert n == 256 + a256(B * H * pairs * 16) + a256(rows * D * 4) + a256(rows * 4)
     simt = ra.ring_step_workspace_size(B, H, S, 40, N, True, "zigzag", 0)
     assert simt == a256(rows * 40 * 4) + a256(rows * 4)
+
+
+def test_steps_per_launch_policy():
+    # FUSED covers every step; PER_STEP takes the request (0 -> 1, clamped to n_ring)
+    assert ra.steps_per_launch(4096, 128, 8, "striped", 1, "fused") == 8
+    assert ra.steps_per_launch(4096, 128, 8, "striped", 1, "per_step", 0) == 1
+    assert ra.steps_per_launch(4096, 128, 8, "striped", 1, "per_step", 3) == 3
+    assert ra.steps_per_launch(4096, 128, 8, "striped", 1, "per_step", 99) == 8
+    # AUTO: fused while a head's K/V (2 * S * D * 2 bytes) fits 96 MB -- s128k (64 MB) stays fused;
+    # s1m (512 MB, 16 MB per block) takes launches of 6 steps (96 MB), evened out over 32 steps
+    assert ra.steps_per_launch(131072, 128, 16, "striped", 1, "auto") == 16
+    assert ra.steps_per_launch(1 << 20, 128, 32, "striped", 1, "auto") == 6
+    assert ra.steps_per_launch(262144, 128, 32, "striped", 1, "auto") == 16
+    # the workspace of AUTO follows the path it takes: none of the per-step buffers for s128k
+    fused = ra.workspace_size(1, 32, 131072, 128, 16, True, "striped", 1, variant="fused")
+    assert ra.workspace_size(1, 32, 131072, 128, 16, True, "striped", 1, variant="auto") == fused
+    per_step = ra.workspace_size(1, 4, 1 << 20, 128, 32, True, "striped", 1, variant="per_step")
+    auto = ra.workspace_size(1, 4, 1 << 20, 128, 32, True, "striped", 1, variant="auto")
+    assert auto <= per_step and auto > 2 * (1 << 20) * 4 * 128 * 4  # running and step partials
+    assert ra.lib().ra_steps_per_launch(4096, 128, 8, 1, 1, 2, -1, ctypes.byref(ctypes.c_int())) == -1

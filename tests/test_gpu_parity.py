@@ -125,6 +125,35 @@ def test_tc_planted_dominant_key():
     compare(out, lse, ref_out, ref_lse, torch.bfloat16)
 
 
+@pytest.mark.parametrize("kernel, dtype, D", [("tc", torch.bfloat16, 128), ("simt", torch.float32, 40)])
+@pytest.mark.parametrize("layout", ["contiguous", "striped", "zigzag"])
+@pytest.mark.parametrize("steps", [2, 3, 8])
+def test_per_step_launches_of_several_ring_steps(kernel, dtype, D, layout, steps):
+    """Each attention launch covers `steps` ring steps (the last one what remains of 8); partial
+    results merge into the running one after each launch but the first."""
+    B, H, S, N = 1, 2, 8 * 256, 8
+    q, k, v = inputs.make_qkv(B, S, H, D, dtype=dtype, device="cuda", seed=31 + steps)
+    out, lse = ra.forward(q, k, v, N, True, layout, variant="per_step", kernel=kernel, steps_per_launch=steps)
+    torch.cuda.synchronize()
+    assert ra.get_device_status() == 0
+    ref_out, ref_lse = oracle.attention(q.cpu(), k.cpu(), v.cpu(), True, threads=THREADS)
+    compare(out, lse, ref_out, ref_lse, dtype)
+
+
+def test_auto_takes_launches_of_several_steps_for_a_head_beyond_l2():
+    """One head of 262144 tokens: its K/V (128 MB) exceed the fused budget, so AUTO runs two
+    launches of 16 ring steps and merges them."""
+    B, H, S, D, N = 1, 1, 262144, 128, 32
+    assert ra.steps_per_launch(S, D, N, "striped", 1, "auto") == 16
+    q, k, v = inputs.make_qkv(B, S, H, D, dtype=torch.bfloat16, device="cuda", seed=41)
+    out, lse = ra.forward(q, k, v, N, True, "striped")
+    torch.cuda.synchronize()
+    assert ra.get_device_status() == 0
+    rows = inputs.sample_rows(S, H, 256, [0, S - 1, S // 2])
+    ref_out, ref_lse = oracle.attention(q.cpu(), k.cpu(), v.cpu(), True, rows=rows, threads=THREADS)
+    compare(out, lse, ref_out, ref_lse, torch.bfloat16, rows=rows)
+
+
 # ---------------------------------------------------------------- s4k: all rows
 @pytest.mark.parametrize("variant", ["fused", "per_step"])
 def test_s4k_all_rows(variant):
