@@ -340,6 +340,7 @@ struct Workspace {
     size_t items = 0, n_items_total = 0;
     size_t qp = 0, kp = 0, vp = 0;  // permuted q, k, v
     size_t O_run = 0, lse_run = 0, O_step = 0, lse_step = 0;
+    size_t kmax = 0;  // largest query and key norm per (b, h), the score bound of the frozen max
     bool permute = false, per_step = false;
     int chunk = 1, n_launches = 1;  // ring steps per attention launch, and the launches
     size_t total = 0;
@@ -386,6 +387,8 @@ Workspace carve(int64_t B, int64_t H, const Layout& L, int64_t D, int causal, in
         off = align_up(off + w.n_counters * sizeof(int));
         w.items = off;
         off = align_up(off + w.n_items_total * sizeof(int4));
+        w.kmax = off;
+        off = align_up(off + (size_t)(2 * B * H) * sizeof(float));
         // striped is read in place through a strided tensor map; zigzag is gathered shard-major
         w.permute = (L.kind == RA_LAYOUT_ZIGZAG);
         if (w.permute) {
@@ -555,6 +558,15 @@ int run_forward(const Call& c, const ra_options& opt) {
             return finish(cuda_fail(e, "work list upload"));
         if ((e = cudaMemsetAsync(ws + w.counters, 0, w.n_counters * sizeof(int), c.stream)) != cudaSuccess)
             return finish(cuda_fail(e, "work counter reset"));
+        if (ra::key_norm_max_applies(c.B, c.H, c.D)) {  // the score bound of every query row (frozen max)
+            float* nmax = reinterpret_cast<float*>(ws + w.kmax);
+            nvtxRangePushA("ra_forward query and key norms");
+            e = ra::launch_norm_max(c.q, c.k, nmax, c.B, c.S, c.H, c.D, dev.sms, c.stream);
+            nvtxRangePop();
+            if (e != cudaSuccess) return finish(cuda_fail(e, "norm launch"));
+            args.qmax = nmax;
+            args.kmax = nmax + c.B * c.H;
+        }
         tc.timeout_ns = opt.timeout_ns ? opt.timeout_ns : 2000000000ull;
         tc.debug = opt.debug;
         tc.status = dev.status;
@@ -793,7 +805,7 @@ int ra_plan_items(int64_t B, int64_t H, int64_t S, int64_t D, int n_ring, int ca
 namespace {
 
 struct RingWorkspace {
-    size_t counter = 0, items = 0, O_s = 0, lse_s = 0, total = 0;
+    size_t counter = 0, items = 0, kmax = 0, O_s = 0, lse_s = 0, total = 0;
     size_t n_items = 0;
 };
 
@@ -807,6 +819,8 @@ RingWorkspace ring_carve(int64_t B, int64_t H, const Layout& L, int64_t D, int c
         off = align_up(off + sizeof(int));
         w.items = off;
         off = align_up(off + w.n_items * sizeof(int4));
+        w.kmax = off;
+        off = align_up(off + (size_t)(2 * B * H) * sizeof(float));
     }
     const size_t rows = (size_t)(B * L.S_loc * H);
     w.O_s = off;
@@ -843,7 +857,8 @@ int ra_ring_step_workspace_size(int64_t B, int64_t H, int64_t S, int64_t D, int 
     const Layout L = make_layout(S, n_ring, layout);
     const int64_t pairs = (L.S_loc + kTcPairRows - 1) / kTcPairRows;
     size_t off = 0;
-    if (tc) off = align_up(sizeof(int)) + align_up((size_t)(B * H * pairs) * sizeof(int4));
+    if (tc) off = align_up(sizeof(int)) + align_up((size_t)(B * H * pairs) * sizeof(int4)) +
+                  align_up((size_t)(2 * B * H) * sizeof(float));
     const size_t rows = (size_t)(B * L.S_loc * H);
     off = align_up(off + rows * (size_t)D * 4);
     off = align_up(off + rows * 4);
@@ -925,6 +940,13 @@ int ra_ring_step(const void* q_i, const void* k_j, const void* v_j, float* O_acc
             return nvtx_pop(finish(cuda_fail(e, "work list upload")));
         if ((e = cudaMemsetAsync(ws + w.counter, 0, sizeof(int), stream)) != cudaSuccess)
             return nvtx_pop(finish(cuda_fail(e, "work counter reset")));
+        if (ra::key_norm_max_applies(B, H, D)) {  // the score bound over query shard i and key block j
+            float* nmax = reinterpret_cast<float*>(ws + w.kmax);
+            if ((e = ra::launch_norm_max(q_i, k_j, nmax, B, L.S_loc, H, D, dev.sms, stream)) != cudaSuccess)
+                return nvtx_pop(finish(cuda_fail(e, "norm launch")));
+            a.qmax = nmax;
+            a.kmax = nmax + B * H;
+        }
         t.items = reinterpret_cast<const int4*>(ws + w.items);
         t.n_items = (int)fl->count;
         t.counter = reinterpret_cast<int*>(ws + w.counter);

@@ -39,6 +39,8 @@
 // status word, lets its own copies and MMAs drain (again bounded), frees TMEM and exits.
 #include <cuda_bf16.h>
 
+#include <type_traits>
+
 #include "ra.h"
 #include "ra_internal.cuh"
 #include "sm100.cuh"
@@ -65,6 +67,11 @@ constexpr int kLoadWarp = 8;
 constexpr int kMmaWarp = 9;
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleLog2 = 8.0f;  // lazy-rescale threshold (log2 units)
+// Frozen max: when the head's score bound (qmax * kmax * scale, log2 units) lies within kFreezeLog2
+// of every row's max after the first tile of an item, a warp keeps its rows' max fixed for the rest
+// of the item: no later weight exceeds 2^kFreezeLog2, so no max and no rescale is needed.
+constexpr float kFreezeLog2 = 32.0f;
+constexpr float kBoundSlack = 1.0f + 1.0f / 256.0f;  // covers fp32 rounding of the norms and of S
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr uint32_t kNegInfBits = 0xff800000u;
@@ -448,13 +455,70 @@ struct Roles {
             const int a = G.a0[q] + row;
             float m_run = -INFINITY, l = 0.f;
             int n_act = 0;
+            bool frozen = false;  // the row max of this warp's rows stays fixed (see kFreezeLog2)
             for (int s = A.s_begin; s < A.s_end && ok; ++s) {
                 const int j = ring_block32(G.i, s, G.L.N);
                 const int nt = tiles_for(G.L, A.causal, G, q, j);
                 if (nt == 0) continue;
                 const int cnt = visible_keys(G.L, A.causal, G.i, a, j);
-                for (int kt = 0; kt < nt; ++kt) {
-                    if (!wait_all(&sm.s_full[q], s_cnt & 1)) break;
+                // One key tile.  Compiled twice: with the row max and the lazy rescale, and -- once the
+                // warp's max is frozen -- without them, so that each copy keeps its own registers.
+                auto tile = [&](auto frozen_tag, int kt) -> bool {
+                    constexpr bool kFrozen = decltype(frozen_tag)::value;
+                    if constexpr (kFrozen) {
+                        // Frozen max: no row max and no rescale, so S need not be held whole.  It is
+                        // read from TMEM 32 columns at a time, each read issued while the previous
+                        // chunk's exponentials run; P of chunk c goes to columns [16c, 16c + 16), which
+                        // only chunks already read occupied.
+                        if (!wait_all(&sm.s_full[q], s_cnt & 1)) return false;
+                        ++s_cnt;
+                        const int valid = cnt - kt * kN;
+                        const uint64_t scale2 = f32x2(sl2, sl2), neg_m2 = f32x2(-m_run, -m_run);
+                        uint64_t lsum[4] = {0, 0, 0, 0};
+                        uint32_t ca[32], cb[32];
+                        tmem_ld32(tS, ca);
+#pragma unroll
+                        for (int c4 = 0; c4 < 4; ++c4) {
+                            uint32_t(&cur)[32] = (c4 & 1) ? cb : ca;
+                            uint32_t(&nxt)[32] = (c4 & 1) ? ca : cb;
+                            tmem_wait_ld_regs(cur);
+                            if (c4 < 3) tmem_ld32(tS + (c4 + 1) * 32, nxt);
+                            if (valid < (c4 + 1) * 32) {
+#pragma unroll
+                                for (int x = 0; x < 32; ++x)
+                                    if (c4 * 32 + x >= valid) cur[x] = kNegInfBits;
+                            }
+                            uint32_t pk[16];
+#pragma unroll
+                            for (int x = 0; x < 16; ++x) {
+                                const uint64_t t2 = fma_f32x2(f32x2(__uint_as_float(cur[2 * x]), __uint_as_float(cur[2 * x + 1])),
+                                                              scale2, neg_m2);
+                                float t0, t1;
+                                split_f32x2(t2, t0, t1);
+                                const uint64_t p2 = f32x2(ex2(t0), ex2(t1));
+                                lsum[x & 3] = add_f32x2(lsum[x & 3], p2);
+                                float p0, p1;
+                                split_f32x2(p2, p0, p1);
+                                pk[x] = pack_bf16x2(p0, p1);
+                            }
+                            tmem_st16(tS + c4 * 16, pk);
+                            if (c4 == 1) {  // P of keys 0..63 visible to the MMA
+                                tmem_wait_st();
+                                tc_fence_before();
+                                __syncwarp();
+                                if ((threadIdx.x & 31) == 0) mbar_arrive(&sm.p_half[q]);
+                            }
+                        }
+                        float a0, a1;
+                        split_f32x2(add_f32x2(add_f32x2(lsum[0], lsum[1]), add_f32x2(lsum[2], lsum[3])), a0, a1);
+                        l += a0 + a1;
+                        tmem_wait_st();
+                        tc_fence_before();
+                        __syncwarp();
+                        if ((threadIdx.x & 31) == 0) mbar_arrive(&sm.p_full[q]);
+                        return true;
+                    } else {
+                    if (!wait_all(&sm.s_full[q], s_cnt & 1)) return false;
                     ++s_cnt;
                     uint32_t r[128];
 #pragma unroll
@@ -470,7 +534,9 @@ struct Roles {
                             if (c >= valid) r[c] = kNegInfBits;
                     }
 #define SF(c) __uint_as_float(r[(c)])
-                    // row max: 8 independent chains of three-input max
+                    // row max, 8 chains of three-input max (not computed once the warp's max is frozen)
+                    float m_new = m_run;
+                    if (!kFrozen) {
                     float mc[8];
 #pragma unroll
                     for (int k = 0; k < 8; ++k) mc[k] = fmax3(SF(k), SF(k + 8), SF(k + 16));
@@ -482,7 +548,8 @@ struct Roles {
                     for (int k = 0; k < 8; ++k) mc[k] = fmaxf(mc[k], SF(120 + k));
                     const float mx = fmax3(fmax3(mc[0], mc[1], mc[2]), fmax3(mc[3], mc[4], mc[5]),
                                            fmaxf(mc[6], mc[7]));
-                    const float m_new = fmaxf(m_run, mx * sl2);
+                    m_new = fmaxf(m_run, mx * sl2);
+                    }
                     bool rescale = false;
                     float alpha = 1.f;
                     if (n_act == 0) {
@@ -495,7 +562,7 @@ struct Roles {
                     }
                     // rescale O before any P V of this tile accumulates into it (P_q V of the
                     // previous tile is complete: S_q of this tile was issued after it)
-                    if (__any_sync(0xffffffffu, rescale)) {
+                    if (!kFrozen && __any_sync(0xffffffffu, rescale)) {
                         const uint64_t alpha2 = f32x2(alpha, alpha);
 #pragma unroll 1
                         for (int c = 0; c < kD / 32; ++c) {
@@ -557,6 +624,20 @@ struct Roles {
                     tc_fence_before();
                     __syncwarp();
                     if ((threadIdx.x & 31) == 0) mbar_arrive(&sm.p_full[q]);
+                    return true;
+                    }
+                };
+                for (int kt = 0; kt < nt && ok; ++kt) {
+                    const bool done = frozen ? tile(std::true_type{}, kt) : tile(std::false_type{}, kt);
+                    if (!done) break;
+                    if (n_act == 0 && A.kmax) {
+                        // after the first tile: the score bound of every row of this head, log2 units
+                        // (Cauchy-Schwarz with the head's largest query and key norms), against the
+                        // max each row has now
+                        const int bh = kVarlen ? G.h : G.b * (int)A.H + G.h;
+                        const float bound = __ldg(A.qmax + bh) * __ldg(A.kmax + bh) * sl2 * kBoundSlack;
+                        frozen = __all_sync(0xffffffffu, bound - m_run <= kFreezeLog2);
+                    }
                     ++n_act;
                 }
             }

@@ -15,7 +15,7 @@
 // Rules of use.
 //   * The first call on a device, with that device current, looks up the array's device address
 //     (cudaGetSymbolAddress) and loads every kernel this entry point launches (both head-dim
-//     instantiations of the attention kernel, the permute kernels and the list builder), so that
+//     instantiations of the attention kernel, the permute and key-norm kernels and the list builder), so that
 //     no later call loads module code.  Make that first call before any stream capture.
 //   * Every call on a device shares the one array and leaves its contents behind.  The one part
 //     that must start at zero, the kernel's work counter, is cleared by each call on its stream
@@ -68,6 +68,7 @@ int scratch_address(unsigned char** out) {
             return ra::host_cuda_fail(e, "loading the work-list builder");
         if ((e = ra::preload_attn_tc()) != cudaSuccess) return ra::host_cuda_fail(e, "loading the attention kernel");
         if ((e = ra::preload_permute()) != cudaSuccess) return ra::host_cuda_fail(e, "loading the permute kernel");
+        if ((e = ra::preload_key_norm()) != cudaSuccess) return ra::host_cuda_fail(e, "loading the key norm kernel");
         it = addr.emplace(dev, static_cast<unsigned char*>(p)).first;
     }
     *out = it->second;
@@ -155,7 +156,8 @@ extern "C" int ra_forward_noalloc(const void* q, const void* k, const void* v, v
     const bool permute = (layout == RA_LAYOUT_ZIGZAG);  // striped is read in place
     const size_t counter_bytes = 256;  // the persistent kernel's work counter, zeroed every call
     const size_t items_bytes = align256((size_t)n_items * sizeof(int4));
-    const size_t need = counter_bytes + items_bytes + (permute ? 3 * align256(tensor_bytes) : 0);
+    const size_t kmax_bytes = align256((size_t)(2 * B * H) * sizeof(float));
+    const size_t need = counter_bytes + items_bytes + kmax_bytes + (permute ? 3 * align256(tensor_bytes) : 0);
     const size_t builder_smem = (size_t)(per_head + L.N) * sizeof(int);
     if (builder_smem > kBuilderSmemBytes) {
         ra::host_set_error("ra_forward_noalloc: too many work items per head for the device list "
@@ -182,7 +184,7 @@ extern "C" int ra_forward_noalloc(const void* q, const void* k, const void* v, v
 
     const void *qs = q, *ks = k, *vs = v;
     if (permute) {
-        unsigned char* base = scratch + counter_bytes + items_bytes;
+        unsigned char* base = scratch + counter_bytes + items_bytes + kmax_bytes;
         void* dst[3] = {base, base + align256(tensor_bytes), base + 2 * align256(tensor_bytes)};
         const void* src[3] = {q, k, v};
         if ((e = ra::launch_permute(src, dst, 3, B, L, H, D, 2, false, stream)) != cudaSuccess)
@@ -217,6 +219,13 @@ extern "C" int ra_forward_noalloc(const void* q, const void* k, const void* v, v
     a.out = out;
     a.lse = lse;
     a.scale = (float)(1.0 / sqrt((double)D));
+    if (ra::key_norm_max_applies(B, H, D)) {  // the score bound of every query row (frozen max)
+        float* nmax = reinterpret_cast<float*>(scratch + counter_bytes + items_bytes);
+        if ((e = ra::launch_norm_max(q, k, nmax, B, S, H, D, sms, stream)) != cudaSuccess)
+            return ra::host_cuda_fail(e, "norm launch");
+        a.qmax = nmax;
+        a.kmax = nmax + B * H;
+    }
     if ((e = ra::launch_attn_tc(a, t, stream)) != cudaSuccess) return ra::host_cuda_fail(e, "attention launch");
     return RA_OK;
 }

@@ -35,7 +35,23 @@ struct AttnArgs {
     // shard 0 of a one-shard buffer, and the partial rows are local, ((b * S_loc + a) * H + h).
     int local;
     int q_shard;
+    // Largest query and key norm per (b, h) -- batch mode -- or per h -- packed sequences -- over
+    // every query row and key the launch reads (launch_norm_max).  Null: every tile computes its
+    // row max (no freezing).
+    const float* qmax;
+    const float* kmax;
 };
+
+// norms.cu: nmax[b * H + h] = max over the `rows` tokens of ||q[b, token, h, :]||_2 and
+// nmax[B * H + b * H + h] the same for k (bf16 q, k of [B, rows, H, D] in any token order, D a
+// multiple of 8 up to 128); zeroes nmax first.  Needs H <= kKeyNormMaxHeads and B <= 65535
+// (key_norm_max_applies).
+constexpr int64_t kKeyNormMaxHeads = 2048;
+inline bool key_norm_max_applies(int64_t B, int64_t H, int64_t D) {
+    return H <= kKeyNormMaxHeads && B <= 65535 && D % 8 == 0 && D <= 128;
+}
+cudaError_t launch_norm_max(const void* q, const void* k, float* nmax, int64_t B, int64_t rows, int64_t H,
+                            int64_t D, int sms, cudaStream_t stream);
 
 // permute.cu
 cudaError_t launch_permute(const void* const* src, void* const* dst, int n_tensors, int64_t B,
@@ -73,6 +89,7 @@ size_t tc_smem_bytes(int64_t D);
 // never triggers lazy module loading.
 cudaError_t preload_attn_tc();
 cudaError_t preload_permute();
+cudaError_t preload_key_norm();
 
 // api.cu: host helpers shared by the entry points.
 int host_check_shape(int64_t B, int64_t H, int64_t S, int64_t D, int n_ring, int layout, int dtype);

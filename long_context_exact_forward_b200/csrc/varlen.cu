@@ -98,11 +98,11 @@ int check_packed(const int64_t* cu_seqlens, int n_seqs, int64_t H, int64_t D, in
 }
 
 // Scratch of one call, in this order: work counter (256 B), sequence table {length, first token},
-// work list (int4 per item), and for zigzag the shard-major copies of q, k, v; every part 256-byte
-// aligned.  The item count is known before the list is built: per non-empty sequence,
+// work list (int4 per item), the largest query and key norm of every head (2 floats per head), and for zigzag the
+// shard-major copies of q, k, v; every part 256-byte aligned.  The item count is known before the list is built: per non-empty sequence,
 // H * N * ceil(S_loc / 256) items.
 struct Scratch {
-    size_t off_seqs, off_items, off_perm, tensor_bytes, bytes;
+    size_t off_seqs, off_items, off_kmax, off_perm, tensor_bytes, bytes;
     int64_t n_items;
 };
 
@@ -116,7 +116,8 @@ Scratch scratch_layout(const int64_t* cu_seqlens, int n_seqs, int64_t H, int64_t
     w.tensor_bytes = align256((size_t)S_total * (size_t)H * (size_t)D * 2);
     w.off_seqs = 256;
     w.off_items = w.off_seqs + align256((size_t)n_seqs * sizeof(int2));
-    w.off_perm = w.off_items + align256((size_t)w.n_items * sizeof(int4));
+    w.off_kmax = w.off_items + align256((size_t)w.n_items * sizeof(int4));
+    w.off_perm = w.off_kmax + align256((size_t)(2 * H) * sizeof(float));
     w.bytes = w.off_perm + (layout == RA_LAYOUT_ZIGZAG ? 3 * w.tensor_bytes : 0);
     return w;
 }
@@ -248,6 +249,13 @@ int varlen_forward(const void* q, const void* k, const void* v, void* out, float
     a.scale = (float)(1.0 / std::sqrt((double)D));
     a.seqs = reinterpret_cast<const int2*>(ws + w.off_seqs);
     a.varlen_striped = striped ? 1 : 0;
+    if (ra::key_norm_max_applies(1, H, D)) {  // the score bound of every query row (frozen max)
+        float* nmax = reinterpret_cast<float*>(ws + w.off_kmax);
+        if ((e = ra::launch_norm_max(q, k, nmax, 1, S_total, H, D, sms, stream)) != cudaSuccess)
+            return finish(ra::host_cuda_fail(e, "norm launch"));
+        a.qmax = nmax;
+        a.kmax = nmax + H;
+    }
     if (ev0 && (e = cudaEventRecord(ev0, stream)) != cudaSuccess) return finish(ra::host_cuda_fail(e, "cudaEventRecord"));
     if ((e = ra::launch_attn_tc(a, t, stream)) != cudaSuccess) return finish(ra::host_cuda_fail(e, "attention launch"));
     if (ev1 && (e = cudaEventRecord(ev1, stream)) != cudaSuccess) return finish(ra::host_cuda_fail(e, "cudaEventRecord"));

@@ -114,7 +114,7 @@ def test_varlen_workspace_size_and_options_validate_on_the_host():
     H, D, N = 3, 128, 8
     a256 = lambda x: -(-x // 256) * 256
     items = sum(H * N * -(-(n // N) // 256) for n in lengths)
-    base = 256 + a256(len(lengths) * 8) + a256(items * 16)
+    base = 256 + a256(len(lengths) * 8) + a256(items * 16) + a256(2 * H * 4)  # ..., norms per head
     assert ra.varlen_workspace_size(cu, H, D, N, "contiguous") == base
     assert ra.varlen_workspace_size(cu, H, D, N, "striped") == base
     assert ra.varlen_workspace_size(cu, H, D, N, "zigzag") == base + 3 * a256(int(cu[-1]) * H * D * 2)
@@ -160,7 +160,7 @@ def test_ring_step_workspace_covers_every_shard_and_step():
     a256 = lambda x: -(-x // 256) * 256
     rows = B * (S // N) * H
     pairs = -(-(S // N) // 256)
-    assert n == 256 + a256(B * H * pairs * 16) + a256(rows * D * 4) + a256(rows * 4)
+    assert n == 256 + a256(B * H * pairs * 16) + a256(2 * B * H * 4) + a256(rows * D * 4) + a256(rows * 4)
     simt = ra.ring_step_workspace_size(B, H, S, 40, N, True, "zigzag", 0)
     assert simt == a256(rows * 40 * 4) + a256(rows * 4)
 
