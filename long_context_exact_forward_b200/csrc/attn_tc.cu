@@ -219,6 +219,14 @@ __device__ __forceinline__ void give_up(volatile int* abort, int* status) {
 }
 
 // Order uses of r[] after the asynchronous TMEM load has landed.
+__device__ __forceinline__ void tmem_wait_ld_regs16(uint32_t (&r)[16]) {
+    asm volatile("tcgen05.wait::ld.sync.aligned;"
+                 : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]),
+                   "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]),
+                   "+r"(r[14]), "+r"(r[15])
+                 :
+                 : "memory");
+}
 __device__ __forceinline__ void tmem_wait_ld_regs(uint32_t (&r)[32]) {
     asm volatile("tcgen05.wait::ld.sync.aligned;"
                  : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]),
@@ -565,18 +573,18 @@ struct Roles {
                     if (!kFrozen && __any_sync(0xffffffffu, rescale)) {
                         const uint64_t alpha2 = f32x2(alpha, alpha);
 #pragma unroll 1
-                        for (int c = 0; c < kD / 32; ++c) {
-                            uint32_t o[32];
-                            tmem_ld32(tO + c * 32, o);
-                            tmem_wait_ld_regs(o);
+                        for (int c = 0; c < kD / 16; ++c) {  // 16 columns at a time: all of S is still live
+                            uint32_t o[16];
+                            tmem_ld16(tO + c * 16, o);
+                            tmem_wait_ld_regs16(o);
 #pragma unroll
-                            for (int x = 0; x < 16; ++x) {
+                            for (int x = 0; x < 8; ++x) {
                                 float v0, v1;
                                 split_f32x2(mul_f32x2(f32x2(__uint_as_float(o[2 * x]), __uint_as_float(o[2 * x + 1])), alpha2), v0, v1);
                                 o[2 * x] = __float_as_uint(v0);
                                 o[2 * x + 1] = __float_as_uint(v1);
                             }
-                            tmem_st32(tO + c * 32, o);
+                            tmem_st16(tO + c * 16, o);
                         }
                     }
                     const float m_use = (m_run == -INFINITY) ? 0.f : m_run;

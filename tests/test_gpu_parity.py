@@ -154,6 +154,25 @@ def test_auto_takes_launches_of_several_steps_for_a_head_beyond_l2():
     compare(out, lse, ref_out, ref_lse, torch.bfloat16, rows=rows)
 
 
+def test_tc_frozen_max_with_a_late_dominant_key():
+    """Norms of about 16 keep the head's score bound (qmax * kmax / sqrt(D)) within 2^32 of the first
+    tile's max, so the kernel freezes each row's max after that tile.  Keys planted parallel to some
+    query rows and visited only in the last ring step then score up to the bound itself -- about 25
+    (log2) above the frozen max -- and those rows must still come out as the exact softmax."""
+    B, H, S, D, N = 1, 2, 4 * 512, 128, 4
+    q, k, v = inputs.make_qkv(B, S, H, D, dtype=torch.float32, device="cuda", seed=17)
+    q, k = q * 1.4, k * 1.4
+XX
+        for h in range(H):
+            k[0, late, h] = q[0, r, h] * (k[0, late, h].norm() / q[0, r, h].norm())
+    q, k, v = (t.to(torch.bfloat16) for t in (q, k, v))
+    out, lse = ra.forward(q, k, v, N, True, "striped", kernel="tc")
+    torch.cuda.synchronize()
+    assert ra.get_device_status() == 0
+    ref_out, ref_lse = oracle.attention(q.cpu(), k.cpu(), v.cpu(), True, threads=THREADS)
+    compare(out, lse, ref_out, ref_lse, torch.bfloat16)
+
+
 # ---------------------------------------------------------------- s4k: all rows
 @pytest.mark.parametrize("variant", ["fused", "per_step"])
 def test_s4k_all_rows(variant):
