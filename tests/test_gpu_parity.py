@@ -162,7 +162,7 @@ def test_tc_frozen_max_with_a_late_dominant_key():
     B, H, S, D, N = 1, 2, 4 * 512, 128, 4
     q, k, v = inputs.make_qkv(B, S, H, D, dtype=torch.float32, device="cuda", seed=17)
     q, k = q * 1.4, k * 1.4
-XX
+    for r, late in ((2000, 1001), (1500, 1397), (2043, 2)):  # striped: key `late` is met after row r's first tile
         for h in range(H):
             k[0, late, h] = q[0, r, h] * (k[0, late, h].norm() / q[0, r, h].norm())
     q, k, v = (t.to(torch.bfloat16) for t in (q, k, v))
