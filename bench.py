@@ -528,9 +528,11 @@ def run_ours(args, w):
     # CUDA-core kernel reads natural order) and the attention launch(es) -- with chunks of C ring
     # steps per launch: ceil(N / C) attention launches and one merge after each but the first
     # (2 kernels each, the last one a single final merge)
+    # the tensor-core path also launches the query/key norm pre-pass (one kernel per call)
     chunk = ra.steps_per_launch(S, D, N, args.layout, 0 if fp32 else 1, args.variant, args.steps_per_launch)
     n_att = -(-N // chunk)
-    launches_per_step = (1 if args.layout == "zigzag" and args.kernel == "tc" else 0) + (
+    tc = args.kernel == "tc"
+    launches_per_step = (1 if args.layout == "zigzag" and tc else 0) + (1 if tc else 0) + (
         1 if n_att == 1 else n_att + 2 * (n_att - 2) + 1)
     if args.backward:
         # Delta, dq, dk/dv; the tensor-core kernels read zigzag from one shard-major permute launch

@@ -157,7 +157,7 @@ def test_auto_takes_launches_of_several_steps_for_a_head_beyond_l2():
 def test_tc_frozen_max_with_a_late_dominant_key():
     """Norms of about 16 keep the head's score bound (qmax * kmax / sqrt(D)) within 2^32 of the first
     tile's max, so the kernel freezes each row's max after that tile.  Keys planted parallel to some
-    query rows and visited only in the last ring step then score up to the bound itself -- about 25
+    query rows and met only in a later ring step then score up to the bound itself -- about 25
     (log2) above the frozen max -- and those rows must still come out as the exact softmax."""
     B, H, S, D, N = 1, 2, 4 * 512, 128, 4
     q, k, v = inputs.make_qkv(B, S, H, D, dtype=torch.float32, device="cuda", seed=17)
