@@ -260,6 +260,7 @@ def config_dict(w, args):
                     f"{args.layout} layout",
         "B": w.B, "H": w.H, "S": w.S, "D": w.D, "n_ring": w.n_ring, "causal": causal_of(args),
         "layout": args.layout, "variant": args.variant, "kernel": args.kernel,
+        **({"workspace": "allocated by every call"} if getattr(args, "no_workspace", False) else {}),
         **({"steps_per_launch": args.steps_per_launch} if args.variant == "per_step" else {}),
         "l2": f"inputs (3 x B*S*H*D {args.dtype}) larger than the 126 MB L2; no flush"
               if 3 * w.B * w.S * w.H * w.D * (4 if args.dtype == "fp32" else 2) > 126e6
@@ -335,6 +336,9 @@ def run_ours(args, w):
                                        variant=args.variant, kernel=args.kernel),
                      dtype=torch.uint8, device=dev)
     flops = attention_flops(B, H, S, D, causal)
+
+    if args.no_workspace:  # every call allocates and frees its own scratch (the library's pool)
+        ws = None
 
     def step(ev=None):
         ra.forward(q, k, v, N, causal, args.layout, variant=args.variant, kernel=args.kernel, out=out,
@@ -579,6 +583,8 @@ def main():
                          "tokens (needs --no-e2e --no-cpu-baseline; not the headline)")
     ap.add_argument("--backward", action="store_true",
                     help="time ra_backward (needs --no-e2e and --no-cpu-baseline; not the headline)")
+    ap.add_argument("--no-workspace", action="store_true",
+                    help="call ra_forward without a caller workspace, so that every call allocates its scratch")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-hbm-kernels", action="store_true")

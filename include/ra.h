@@ -97,8 +97,10 @@ typedef struct ra_options {
     int variant;             /* enum ra_variant */
     int kernel;              /* enum ra_kernel */
     void* workspace;         /* device buffer of >= ra_workspace_size bytes, 256-byte aligned;
-                                NULL: the call allocates stream-ordered (cudaMallocAsync) and frees
-                                it the same way on `stream` */
+                                NULL: the call allocates stream-ordered on `stream` from a pool the
+                                library keeps per device, and frees it the same way; freed memory
+                                stays reserved in that pool for later calls until the process exits
+                                (a stream being captured allocates from the default pool) */
     size_t workspace_bytes;
     uint64_t timeout_ns;     /* limit for every in-kernel wait; 0 = 2 s */
     int debug;               /* enum ra_debug */
@@ -218,7 +220,7 @@ RA_API int ra_forward_noalloc(const void* q, const void* k, const void* v, void*
  *   D <= 128 (RA_ERR_UNSUPPORTED otherwise); pointers aligned to their element size.
  *   The caller owns every buffer; scratch (B*H*S fp32 for Delta, plus shard-major copies for
  *   zigzag on the tensor-core path) is allocated and freed stream-ordered on `stream`
- *   (cudaMallocAsync / cudaFreeAsync).  Asynchronous on `stream`.
+ *   (from the library's pool, as ra_options.workspace = NULL describes).  Asynchronous on `stream`.
  * Returns RA_OK or a negative status (validation errors before anything is enqueued). */
 RA_API int ra_backward(const void* q, const void* k, const void* v, const void* out, const float* lse,
                        const void* dout, void* dq, void* dk, void* dv, int64_t B, int64_t H, int64_t S,

@@ -506,8 +506,8 @@ int run_forward(const Call& c, const ra_options& opt) {
         if (opt.workspace_bytes < w.total) return RA_ERR_NO_WORKSPACE;
         if (reinterpret_cast<uintptr_t>(ws) % kAlign) return RA_ERR_ALIGN;
     } else {
-        cudaError_t e = cudaMallocAsync(reinterpret_cast<void**>(&ws), w.total, c.stream);
-        if (e != cudaSuccess) return cuda_fail(e, "cudaMallocAsync(workspace)");
+        cudaError_t e = ra::scratch_alloc(reinterpret_cast<void**>(&ws), w.total, c.stream);
+        if (e != cudaSuccess) return cuda_fail(e, "stream-ordered allocation (workspace)");
         own_ws = true;
     }
     auto finish = [&](int status) {
@@ -896,8 +896,8 @@ int ra_ring_step(const void* q_i, const void* k_j, const void* v_j, float* O_acc
         if (workspace_bytes < w.total) return RA_ERR_NO_WORKSPACE;
         if (reinterpret_cast<uintptr_t>(ws) % kAlign) return RA_ERR_ALIGN;
     } else {
-        cudaError_t e = cudaMallocAsync(reinterpret_cast<void**>(&ws), w.total, stream);
-        if (e != cudaSuccess) return cuda_fail(e, "cudaMallocAsync(ring step workspace)");
+        cudaError_t e = ra::scratch_alloc(reinterpret_cast<void**>(&ws), w.total, stream);
+        if (e != cudaSuccess) return cuda_fail(e, "stream-ordered allocation (ring step workspace)");
         own_ws = true;
     }
     auto finish = [&](int status) {

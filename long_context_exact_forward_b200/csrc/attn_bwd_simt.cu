@@ -432,9 +432,9 @@ extern "C" int ra_backward_ex(const void* q, const void* k, const void* v, const
     const size_t copy_bytes = ((size_t)(B * S * H * D) * 2 + 255) / 256 * 256;
     const bool copies = use_tc && layout == RA_LAYOUT_ZIGZAG;
     uint8_t* scratch = nullptr;
-    cudaError_t e = cudaMallocAsync(reinterpret_cast<void**>(&scratch), delta_bytes + (copies ? 4 * copy_bytes : 0),
-                                    stream);
-    if (e != cudaSuccess) return ra::host_cuda_fail(e, "cudaMallocAsync(backward scratch)");
+    cudaError_t e = ra::scratch_alloc(reinterpret_cast<void**>(&scratch), delta_bytes + (copies ? 4 * copy_bytes : 0),
+                                      stream);
+    if (e != cudaSuccess) return ra::host_cuda_fail(e, "stream-ordered allocation (backward scratch)");
     float* delta = reinterpret_cast<float*>(scratch);
     ra::BwdArgs A{};
     A.L = ra::Layout{S, (int64_t)n_ring, S / n_ring, layout};

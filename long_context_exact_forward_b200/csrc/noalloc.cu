@@ -2,7 +2,7 @@
 //
 // Who needs this.  ra_forward needs scratch memory (the work list of the persistent kernel and,
 // for the zigzag layout, shard-major copies of q, k and v) and, unless the caller
-// hands it a workspace, gets it with cudaMallocAsync.  Some callers cannot let a library
+// hands it a workspace, allocates it stream-ordered.  Some callers cannot let a library
 // allocate device memory at all: code recording a CUDA graph (an allocation inside stream capture
 // either fails or becomes part of the graph), engines that own every byte of the GPU through
 // their own allocator and budget, and latency-critical loops where an allocator call may stall.

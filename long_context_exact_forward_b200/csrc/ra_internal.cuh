@@ -53,6 +53,10 @@ inline bool key_norm_max_applies(int64_t B, int64_t H, int64_t D) {
 cudaError_t launch_norm_max(const void* q, const void* k, float* nmax, int64_t B, int64_t rows, int64_t H,
                             int64_t D, int sms, cudaStream_t stream);
 
+// pool.cu: stream-ordered scratch of the allocating entry points, from a library-owned pool per
+// device that keeps freed memory reserved (the default pool when the stream is capturing).
+cudaError_t scratch_alloc(void** ptr, size_t bytes, cudaStream_t stream);
+
 // permute.cu
 cudaError_t launch_permute(const void* const* src, void* const* dst, int n_tensors, int64_t B,
                            const Layout& L, int64_t H, int64_t D, int esize, bool inverse,

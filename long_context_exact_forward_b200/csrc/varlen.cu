@@ -180,8 +180,8 @@ int varlen_forward(const void* q, const void* k, const void* v, void* out, float
     uint8_t* ws = ws_given;
     cudaError_t e = cudaSuccess;
     if (!ws_given) {
-        e = cudaMallocAsync(reinterpret_cast<void**>(&ws), w.bytes, stream);
-        if (e != cudaSuccess) return ra::host_cuda_fail(e, "cudaMallocAsync(varlen scratch)");
+        e = ra::scratch_alloc(reinterpret_cast<void**>(&ws), w.bytes, stream);
+        if (e != cudaSuccess) return ra::host_cuda_fail(e, "stream-ordered allocation (varlen scratch)");
     }
     auto finish = [&](int r) {
         if (ws_given) return r;
