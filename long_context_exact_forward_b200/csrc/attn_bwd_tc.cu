@@ -515,16 +515,30 @@ __global__ void __launch_bounds__(kThreads, 1)
                     uint32_t sv[32], pk[16];
                     tmem_ld32(lane_base + kST + 32 * c, sv);
                     wait_ld_tied(sv);
+                    const float4* l4 = reinterpret_cast<const float4*>(&sm.col_lse2[st][32 * c]);
+                    // every query of this chunk sees the key: no per-element check (the common case)
+                    const bool all_vis = q0 + 32 * c >= a_min && q0 + 32 * c + 31 < L.S_loc;
+                    if (all_vis) {
 #pragma unroll
-                    for (int x = 0; x < 16; ++x) {
-                        float p[2];
-#pragma unroll
-                        for (int e = 0; e < 2; ++e) {
-                            const int col = 32 * c + 2 * x + e, a = q0 + col;
-                            const bool vis = a >= a_min && a < L.S_loc;
-                            p[e] = vis ? ex2(fmaf(__uint_as_float(sv[2 * x + e]), sl2, -sm.col_lse2[st][col])) : 0.f;
+                        for (int x = 0; x < 8; ++x) {
+                            const float4 lv = l4[x];  // 4 columns' lse per shared-memory load
+                            pk[2 * x] = pack_bf16x2(ex2(fmaf(__uint_as_float(sv[4 * x]), sl2, -lv.x)),
+                                                    ex2(fmaf(__uint_as_float(sv[4 * x + 1]), sl2, -lv.y)));
+                            pk[2 * x + 1] = pack_bf16x2(ex2(fmaf(__uint_as_float(sv[4 * x + 2]), sl2, -lv.z)),
+                                                        ex2(fmaf(__uint_as_float(sv[4 * x + 3]), sl2, -lv.w)));
                         }
-                        pk[x] = pack_bf16x2(p[0], p[1]);
+                    } else {
+#pragma unroll
+                        for (int x = 0; x < 16; ++x) {
+                            float p[2];
+#pragma unroll
+                            for (int e = 0; e < 2; ++e) {
+                                const int col = 32 * c + 2 * x + e, a = q0 + col;
+                                const bool vis = a >= a_min && a < L.S_loc;
+                                p[e] = vis ? ex2(fmaf(__uint_as_float(sv[2 * x + e]), sl2, -sm.col_lse2[st][col])) : 0.f;
+                            }
+                            pk[x] = pack_bf16x2(p[0], p[1]);
+                        }
                     }
                     tmem_st16(lane_base + kST + 16 * c, pk);
                 }
@@ -539,13 +553,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tmem_ld16(lane_base + kST + 16 * c, pb);
                     wait_ld_tied(pv);
                     wait_ld_tied(pb);
+                    const float4* d4 = reinterpret_cast<const float4*>(&sm.col_delta[st][32 * c]);
 #pragma unroll
-                    for (int x = 0; x < 16; ++x) {
-                        const float p0 = __uint_as_float(pb[x] << 16), p1 = __uint_as_float(pb[x] & 0xffff0000u);
-                        const int col = 32 * c + 2 * x;
-                        const float d0 = p0 * (__uint_as_float(pv[2 * x]) - sm.col_delta[st][col]);
-                        const float d1 = p1 * (__uint_as_float(pv[2 * x + 1]) - sm.col_delta[st][col + 1]);
-                        dk16[x] = pack_bf16x2(d0, d1);
+                    for (int x = 0; x < 8; ++x) {
+                        const float4 dv = d4[x];  // 4 columns' Delta per shared-memory load
+                        const uint32_t b0 = pb[2 * x], b1 = pb[2 * x + 1];
+                        dk16[2 * x] = pack_bf16x2(__uint_as_float(b0 << 16) * (__uint_as_float(pv[4 * x]) - dv.x),
+                                                  __uint_as_float(b0 & 0xffff0000u) * (__uint_as_float(pv[4 * x + 1]) - dv.y));
+                        dk16[2 * x + 1] = pack_bf16x2(__uint_as_float(b1 << 16) * (__uint_as_float(pv[4 * x + 2]) - dv.z),
+                                                      __uint_as_float(b1 & 0xffff0000u) * (__uint_as_float(pv[4 * x + 3]) - dv.w));
                     }
                     tmem_st16(lane_base + kdPT + 16 * c, dk16);
                 }
