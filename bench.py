@@ -39,6 +39,13 @@ METRIC_BWD = "ring-attn bwd TFLOP/s (causal; 2.5x forward flops)"
 METRIC_VARLEN = "ring-attn fwd TFLOP/s over packed variable-length sequences (bf16, causal)"
 
 
+def ring_word(args):
+    """How the attention launches walk the ring steps, for the roofline's kernel name."""
+    if args.variant != "per_step":
+        return "fused ring" if args.varlen or args.variant == "fused" else "ring, variant auto"
+    return f"{args.steps_per_launch or 1} ring step(s) per launch"
+
+
 def varlen_lengths(S, n_ring, seed):
     """A seeded mix of sequence lengths that fills S tokens: multiples of 128 * n_ring between
     S / 64 and S / 4 (the last one takes what is left)."""
@@ -350,11 +357,13 @@ def run_ours(args, w):
         for n in lengths:
             cu.append(cu[-1] + n)
         lse_v = torch.empty((H, S), dtype=torch.float32, device=dev)
-        ws_v = torch.empty(ra.varlen_workspace_size(cu, H, D, N, args.layout), dtype=torch.uint8, device=dev)
+        ws_v = torch.empty(ra.varlen_workspace_size(cu, H, D, N, args.layout, 0 if fp32 else 1, args.variant,
+                                                    args.kernel), dtype=torch.uint8, device=dev)
         flops = sum(attention_flops(1, H, n, D, causal) for n in lengths)
 
-        def step(ev=None):  # ev: recorded by the library around the attention launch
-            ra.forward_varlen(q[0], k[0], v[0], cu, N, causal, args.layout, out=out[0], lse=lse_v, workspace=ws_v,
+        def step(ev=None):  # ev: recorded by the library around the attention launches
+            ra.forward_varlen(q[0], k[0], v[0], cu, N, causal, args.layout, variant=args.variant, kernel=args.kernel,
+                              steps_per_launch=args.steps_per_launch, out=out[0], lse=lse_v, workspace=ws_v,
                               stream=stream, events=ev)
 
     if args.backward:
@@ -508,8 +517,8 @@ def run_ours(args, w):
             "frac_of_burst_peak": achieved / peaks["bf16_tflops"],
             "kernel": ("bwd_dq_tc_kernel + bwd_dkv_tc_kernel (tcgen05), timed as one ra_backward call"
                        if args.backward else
-                       "attn_tc_kernel<128, varlen> (fused ring, tcgen05)"
-                       if args.varlen else "attn_tc_kernel<128> (fused ring, tcgen05)"),
+                       f"attn_tc_kernel<128, varlen> ({ring_word(args)}, tcgen05)"
+                       if args.varlen else f"attn_tc_kernel<128> ({ring_word(args)}, tcgen05)"),
             "kernel_ms": k_ms,
             "algorithmic_flops_per_launch": flops,
         }
@@ -534,6 +543,8 @@ def run_ours(args, w):
     # (2 kernels each, the last one a single final merge)
     # the tensor-core path also launches the query/key norm pre-pass (one kernel per call)
     chunk = ra.steps_per_launch(S, D, N, args.layout, 0 if fp32 else 1, args.variant, args.steps_per_launch)
+    if args.varlen:  # packed sequences: one launch unless per-step launches are asked for
+        chunk = min(N, args.steps_per_launch or 1) if args.variant == "per_step" else N
     n_att = -(-N // chunk)
     tc = args.kernel == "tc"
     launches_per_step = (1 if args.layout == "zigzag" and tc else 0) + (1 if tc else 0) + (

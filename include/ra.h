@@ -248,36 +248,46 @@ RA_API int ra_backward_ex(const void* q, const void* k, const void* v, const voi
  * axis -- each query attends only to the keys of its own sequence (and, when `causal`, to those at or
  * before its position inside that sequence).  troisinh.com "Ring Attention", "Trade-off thuc te",
  * names load balancing with sequences of different lengths as the challenge; every sequence is split
- * into n_ring shards with `layout` and all their work items join one longest-first list for the
- * fused tensor-core kernel.
- *   q, k, v, out: [S_total, H, D] bf16 (batch 1), natural order; lse: [H, S_total] fp32, natural log.
+ * into n_ring shards with `layout` and all their work items join one longest-first list.
+ *   q, k, v, out: [S_total, H, D] in dtype (batch 1), natural order; lse: [H, S_total] fp32, natural
+ *     log.
  *   cu_seqlens: HOST array of n_seqs + 1 int64 offsets, cu[0] = 0, non-decreasing, cu[n_seqs] =
  *     S_total; every length a multiple of n_ring, of 2 n_ring for zigzag (RA_ERR_SHAPE otherwise);
- *     empty sequences allowed.
- *   layout: contiguous, striped or zigzag, applied inside each sequence; D in {64, 128}; sm_100;
- *   q, k, v, out 16-byte aligned.  Scratch (work list, sequence table, counter; for zigzag also
- *   shard-major copies of q, k, v, 3 x S_total*H*D bf16) is allocated stream-ordered.
- *   Asynchronous on `stream`; bounded waits report through ra_get_device_status. */
+ *     empty sequences allowed.  S_total < 2^31, H <= 65535, 1 <= D <= 256.
+ *   layout: contiguous, striped or zigzag, applied inside each sequence; dtype RA_DTYPE_FP32 or
+ *   RA_DTYPE_BF16; q, k, v, out 16-byte aligned.  The defaults of ra_options apply: the tcgen05
+ *   kernel (sm_100) for bf16 with D in {64, 128}, all ring steps in one persistent launch; the
+ *   CUDA-core kernel with fp32 arithmetic otherwise.  Scratch (work list, sequence table, counter;
+ *   for zigzag on the tensor cores also shard-major copies of q, k, v, 3 x S_total*H*D bf16) is
+ *   allocated stream-ordered.  Asynchronous on `stream`; bounded waits report through
+ *   ra_get_device_status. */
 RA_API int ra_forward_varlen(const void* q, const void* k, const void* v, void* out, float* lse,
                              const int64_t* cu_seqlens, int n_seqs, int64_t H, int64_t D, int n_ring,
-                             int causal, int layout, void* stream);
+                             int causal, int layout, int dtype, void* stream);
 
 /* ra_forward_varlen_ex: ra_forward_varlen with options (opt may be NULL for the defaults).
- *   workspace / workspace_bytes: caller scratch of at least ra_varlen_workspace_size bytes, 256-byte
- *     aligned (RA_ERR_ALIGN otherwise; RA_ERR_NO_WORKSPACE if smaller); NULL: allocated and freed
- *     stream-ordered as ra_forward_varlen does.  A caller that keeps the buffer between calls saves
- *     the allocation, which for zigzag holds the 3 x S_total*H*D bf16 shard-major copies.
- *   timeout_ns, debug: as for ra_forward_ex.  attn_events: recorded right before and right after the
- *     attention launch (after the zigzag gather).
- *   variant must be AUTO or FUSED and kernel AUTO or TC (RA_ERR_UNSUPPORTED otherwise). */
+ *   variant: AUTO and FUSED walk every ring step in one attention launch; PER_STEP walks
+ *     opt->steps_per_launch steps per launch (0 = 1) and folds each launch's partial result, kept
+ *     in fp32 in natural packed rows, into the running one with the log-sum-exp merge.
+ *   kernel: AUTO (tensor cores where they apply, see ra_forward_varlen), TC (bf16 with D in {64, 128}
+ *     on sm_100, RA_ERR_UNSUPPORTED otherwise) or SIMT (CUDA cores, fp32 arithmetic, any dtype).
+ *   workspace / workspace_bytes: caller scratch of at least ra_varlen_workspace_size bytes (for the
+ *     same variant and kernel), 256-byte aligned (RA_ERR_ALIGN otherwise; RA_ERR_NO_WORKSPACE if
+ *     smaller); NULL: allocated and freed stream-ordered as ra_forward_varlen does.  A caller that
+ *     keeps the buffer between calls saves the allocation, which for zigzag on the tensor cores
+ *     holds the 3 x S_total*H*D bf16 shard-major copies and, with more than one launch, the fp32
+ *     running and partial results (2 x S_total*H*(D + 1) floats).
+ *   timeout_ns, debug: as for ra_forward_ex (the tensor-core kernel's waits).  attn_events: recorded
+ *     right before the first and right after the last attention launch (after the zigzag gather). */
 RA_API int ra_forward_varlen_ex(const void* q, const void* k, const void* v, void* out, float* lse,
                                 const int64_t* cu_seqlens, int n_seqs, int64_t H, int64_t D, int n_ring,
-                                int causal, int layout, void* stream, const ra_options* opt);
+                                int causal, int layout, int dtype, void* stream, const ra_options* opt);
 
 /* ra_varlen_workspace_size: scratch bytes ra_forward_varlen_ex needs for these packed sequences,
- * written to *bytes.  Host only; the arguments are validated as for ra_forward_varlen. */
+ * dtype, variant and kernel (enum values as in ra_options), written to *bytes; for PER_STEP the size
+ * covers every steps_per_launch.  Host only; the arguments are validated as for ra_forward_varlen. */
 RA_API int ra_varlen_workspace_size(const int64_t* cu_seqlens, int n_seqs, int64_t H, int64_t D, int n_ring,
-                                    int layout, size_t* bytes);
+                                    int layout, int dtype, int variant, int kernel, size_t* bytes);
 
 /* ra_rope: rotary position embedding with global token positions (troisinh.com "Ring Attention",
  * "RoPE va Position Embedding": a token must be rotated by the angle m theta of its own position m

@@ -90,10 +90,11 @@ def lib():
         L.ra_forward_noalloc.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i64, ci, ci, ci, vp]
         L.ra_backward.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i64, i64, i64, i64, ci, ci, ci,
                                   ci, vp]
-        L.ra_forward_varlen.argtypes = [vp, vp, vp, vp, vp, vp, ci, i64, i64, ci, ci, ci, vp]
-        L.ra_forward_varlen_ex.argtypes = [vp, vp, vp, vp, vp, vp, ci, i64, i64, ci, ci, ci, vp,
+        L.ra_forward_varlen.argtypes = [vp, vp, vp, vp, vp, vp, ci, i64, i64, ci, ci, ci, ci, vp]
+        L.ra_forward_varlen_ex.argtypes = [vp, vp, vp, vp, vp, vp, ci, i64, i64, ci, ci, ci, ci, vp,
                                            ctypes.POINTER(Options)]
-        L.ra_varlen_workspace_size.argtypes = [vp, ci, i64, i64, ci, ci, ctypes.POINTER(ctypes.c_size_t)]
+        L.ra_varlen_workspace_size.argtypes = [vp, ci, i64, i64, ci, ci, ci, ci, ci,
+                                               ctypes.POINTER(ctypes.c_size_t)]
         L.ra_rope.argtypes = [vp, vp, i64, i64, i64, i64, i64, ctypes.c_double, ci, vp]
         L.ra_backward_ex.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i64, i64, i64, i64, ci, ci, ci,
                                      ci, ci, ctypes.c_uint64, ci, vp]
@@ -315,32 +316,38 @@ def _cu_array(cu_seqlens):
     return cu
 
 
-def varlen_workspace_size(cu_seqlens, H, D, n_ring, layout="contiguous"):
+def varlen_workspace_size(cu_seqlens, H, D, n_ring, layout="contiguous", dtype_code=1, variant="auto",
+                          kernel="auto"):
     """Bytes of scratch forward_varlen needs for these packed sequences (ra_varlen_workspace_size)."""
     cu = _cu_array(cu_seqlens)
     n = ctypes.c_size_t(0)
     _clear_error()
     _check(lib().ra_varlen_workspace_size(cu.ctypes.data, int(cu.size - 1), H, D, int(n_ring), LAYOUTS[layout],
-                                          ctypes.byref(n)), "ra_varlen_workspace_size")
+                                          int(dtype_code), VARIANTS[variant], KERNELS[kernel], ctypes.byref(n)),
+           "ra_varlen_workspace_size")
     return n.value
 
 
-def forward_varlen(q, k, v, cu_seqlens, n_ring, causal=True, layout="contiguous", *, out=None, lse=None,
-                   workspace=None, stream=None, events=None, timeout_ns=0, debug=0):
+def forward_varlen(q, k, v, cu_seqlens, n_ring, causal=True, layout="contiguous", *, variant="auto",
+                   kernel="auto", steps_per_launch=0, out=None, lse=None, workspace=None, stream=None,
+                   events=None, timeout_ns=0, debug=0):
     """ra_forward_varlen_ex: attention over sequences packed on the token axis of q, k, v [S_total, H, D]
-    (bf16); cu_seqlens: n_seqs + 1 offsets (a host sequence of ints); layout "contiguous", "striped"
-    or "zigzag" inside each sequence.  Returns (out [S_total, H, D], lse [H, S_total]).
+    (fp32 or bf16); cu_seqlens: n_seqs + 1 offsets (a host sequence of ints); layout "contiguous",
+    "striped" or "zigzag" inside each sequence; variant "auto", "fused" or "per_step" (with
+    `steps_per_launch` ring steps per launch); kernel "auto", "tc" or "simt".  Returns
+    (out [S_total, H, D] in q's dtype, lse [H, S_total]).
 
     `workspace` is an optional uint8 CUDA tensor of at least varlen_workspace_size(...) bytes; without
     it the scratch comes from torch's caching allocator on the call's stream, so repeated calls do
     not allocate device memory anew.  `events`: an optional pair of torch.cuda.Event recorded around
-    the attention launch."""
+    the attention launches."""
     torch = _torch()
     _check_cuda(q, k, v)
     if q.dim() != 3 or q.shape != k.shape or q.shape != v.shape:
         raise ValueError("q, k, v must all be [S_total, H, D]")
-    if q.dtype != torch.bfloat16 or k.dtype != q.dtype or v.dtype != q.dtype:
-        raise TypeError("forward_varlen takes bf16 q, k, v")
+    dtype_code = _dtype_code(q)
+    if k.dtype != q.dtype or v.dtype != q.dtype:
+        raise TypeError("q, k, v must share one dtype")
     S, H, D = q.shape
     cu = _cu_array(cu_seqlens)
     if cu[-1] != S:
@@ -350,13 +357,16 @@ def forward_varlen(q, k, v, cu_seqlens, n_ring, causal=True, layout="contiguous"
     _check_out(out, q.shape, q.dtype, "out", q)
     _check_out(lse, (H, S), torch.float32, "lse", q)
     if workspace is None:
-        n = varlen_workspace_size(cu, H, D, n_ring, layout)
+        n = varlen_workspace_size(cu, H, D, n_ring, layout, dtype_code, variant, kernel)
         with torch.cuda.device(q.device):
             workspace = torch.empty(n, dtype=torch.uint8, device=q.device)
         if stream is not None:  # the scratch must outlive the work enqueued on `stream`
             workspace.record_stream(stream)
     _check_cuda(q, workspace)
     opt = Options()
+    opt.variant = VARIANTS[variant]
+    opt.kernel = KERNELS[kernel]
+    opt.steps_per_launch = int(steps_per_launch)
     opt.workspace = workspace.data_ptr()
     opt.workspace_bytes = workspace.numel() * workspace.element_size()
     opt.timeout_ns = int(timeout_ns)
@@ -371,7 +381,7 @@ def forward_varlen(q, k, v, cu_seqlens, n_ring, causal=True, layout="contiguous"
     with torch.cuda.device(q.device):
         rc = lib().ra_forward_varlen_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
                                         cu.ctypes.data, int(cu.size - 1), H, D, int(n_ring), int(bool(causal)),
-                                        LAYOUTS[layout], _stream_handle(stream), ctypes.byref(opt))
+                                        LAYOUTS[layout], dtype_code, _stream_handle(stream), ctypes.byref(opt))
     _check(rc, "ra_forward_varlen_ex")
     return out, lse
 

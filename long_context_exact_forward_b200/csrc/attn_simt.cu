@@ -18,6 +18,11 @@
 // consecutive bytes of V, so the float4 loads are free of bank conflicts).  Two CTAs share an SM.  Row maxima and sums are reduced over
 // the 16 threads of a row group with shuffles.  Keys and values are gathered straight from natural
 // order with the layout map, so no permute is needed.
+//
+// Packed sequences (several sequences one after another on the token axis, batch 1): block x takes
+// the work item items[x] = {sequence, shard, 64-row query tile} and block z the head; the sequence's
+// own layout map (its length split into N shards) places every row, offset by the sequence's first
+// token, so a query only meets the keys of its own sequence.
 #include <cuda_bf16.h>
 
 #include "ra_internal.cuh"
@@ -43,23 +48,25 @@ __device__ __forceinline__ float from_float<float>(float x) { return x; }
 template <>
 __device__ __forceinline__ __nv_bfloat16 from_float<__nv_bfloat16>(float x) { return __float2bfloat16_rn(x); }
 
+// Token row of local token a of shard `shard`: natural order through the layout map (after the
+// first token `base` of a packed sequence), or, for a ring step on local buffers, row a of the
+// one-shard buffer.
+__device__ __forceinline__ int64_t token_row(const Layout& L, int local, int64_t b, int64_t base, int64_t shard,
+                                             int64_t a) {
+    return local ? b * L.S_loc + a : b * L.S + base + global_position(L, shard, a);
+}
+
 // Gather `kB` token rows of shard `shard` from local row a0 (natural order through the layout map)
 // as fp32 into shared memory, transposed: dst[d * kB + r].  Rows past the shard end and columns
 // d >= D read as zero.  Thread t takes row t % kB and 4 consecutive columns at a time, so
 // consecutive threads write consecutive words and each thread reads whole sectors of its row.
-// Token row of local token a of shard `shard`: natural order through the layout map, or, for a
-// ring step on local buffers, row a of the one-shard buffer.
-__device__ __forceinline__ int64_t token_row(const Layout& L, int local, int64_t b, int64_t shard, int64_t a) {
-    return local ? b * L.S_loc + a : b * L.S + global_position(L, shard, a);
-}
-
 template <typename T, int kDMax, int kB>
 __device__ void load_transposed(float* dst, const T* __restrict__ src, const Layout& L, int local, int64_t b,
-                                int64_t h, int64_t H, int64_t D, int64_t shard, int64_t a0) {
+                                int64_t base, int64_t h, int64_t H, int64_t D, int64_t shard, int64_t a0) {
     const int r = threadIdx.x % kB;
     const int64_t a = a0 + r;
     const T* row = nullptr;
-    if (a < L.S_loc) row = src + (token_row(L, local, b, shard, a) * H + h) * D;
+    if (a < L.S_loc) row = src + (token_row(L, local, b, base, shard, a) * H + h) * D;
     for (int d4 = 4 * (threadIdx.x / kB); d4 < kDMax; d4 += 4 * (kThreads / kB)) {
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
@@ -72,13 +79,13 @@ __device__ void load_transposed(float* dst, const T* __restrict__ src, const Lay
 // Same rows, row-major: dst[r * kDMax + d].  Consecutive threads take consecutive columns.
 template <typename T, int kDMax, int kB>
 __device__ void load_rowmajor(float* dst, const T* __restrict__ src, const Layout& L, int local, int64_t b,
-                              int64_t h, int64_t H, int64_t D, int64_t shard, int64_t a0) {
+                              int64_t base, int64_t h, int64_t H, int64_t D, int64_t shard, int64_t a0) {
     for (int idx = threadIdx.x; idx < kB * kDMax; idx += kThreads) {
         const int r = idx / kDMax, d = idx % kDMax;
         const int64_t a = a0 + r;
         float x = 0.f;
         if (a < L.S_loc && d < D)
-            x = to_float<T>(src[(token_row(L, local, b, shard, a) * H + h) * D + d]);
+            x = to_float<T>(src[(token_row(L, local, b, base, shard, a) * H + h) * D + d]);
         dst[idx] = x;
     }
 }
@@ -93,7 +100,7 @@ __device__ __forceinline__ int pt_index(int key, int row4) {
 template <typename T, int kDMax>
 __global__ void __launch_bounds__(kThreads, kDMax <= 128 ? 2 : 1)
     attn_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
-                     AttnArgs args) {
+                     AttnArgs args, const int4* __restrict__ items) {
     constexpr int kOC = kDMax / 16;  // output columns per thread
     static_assert(kOC % 4 == 0, "kDMax is a multiple of 64");
     extern __shared__ __align__(16) float smem[];
@@ -102,18 +109,31 @@ __global__ void __launch_bounds__(kThreads, kDMax <= 128 ? 2 : 1)
     float* Vs = Kt + kDMax * kBK;     // [kBK][kDMax]
     float* Pt = Vs + kBK * kDMax;     // [kBK][kBQ], swizzled (pt_index)
 
-    const Layout L = args.L;
     const int64_t D = args.D, H = args.H;
-    // heaviest shards first: under the causal mask with the contiguous layout shard i meets i + 1
-    // live blocks, so the CTAs of the last shards are launched first (a longest-first order)
-    const int64_t i = args.local ? args.q_shard : L.N - 1 - blockIdx.y;
-    const int64_t bh = blockIdx.z;
-    const int64_t b = bh / H, h = bh % H;
-    const int64_t a0 = (int64_t)blockIdx.x * kBQ;
+    const int64_t S_axis = args.L.S;  // token axis of out and lse (the packed length for packed sequences)
+    Layout L = args.L;
+    int64_t i, b, h, a0, base = 0;
+    if (items) {  // packed sequences: this block's item, the sequence's own layout
+        const int4 it = items[blockIdx.x];
+        const int2 sd = args.seqs[it.x];
+        L = Layout{sd.x, args.L.N, sd.x / args.L.N, args.L.kind};
+        base = sd.y;
+        i = it.y;
+        a0 = (int64_t)it.z * kBQ;
+        b = 0;
+        h = blockIdx.z;
+    } else {
+        // heaviest shards first: under the causal mask with the contiguous layout shard i meets
+        // i + 1 live blocks, so the CTAs of the last shards are launched first (a longest-first order)
+        i = args.local ? args.q_shard : L.N - 1 - blockIdx.y;
+        b = blockIdx.z / H;
+        h = blockIdx.z % H;
+        a0 = (int64_t)blockIdx.x * kBQ;
+    }
     const int ty = threadIdx.x >> 4, tx = threadIdx.x & 15;
     const int64_t a_last = (a0 + kBQ - 1 < L.S_loc - 1) ? a0 + kBQ - 1 : L.S_loc - 1;
 
-    load_transposed<T, kDMax, kBQ>(Qt, q, L, args.local, b, h, H, D, i, a0);
+    load_transposed<T, kDMax, kBQ>(Qt, q, L, args.local, b, base, h, H, D, i, a0);
 
     float m[4], l[4], o[4][kOC];
 #pragma unroll
@@ -135,8 +155,8 @@ __global__ void __launch_bounds__(kThreads, kDMax <= 128 ? 2 : 1)
         const int64_t n_vis_cta = visible_keys(L, args.causal, i, a_last, j);  // the CTA's widest
         for (int64_t b0 = 0; b0 < n_vis_cta; b0 += kBK) {
             __syncthreads();  // previous tile consumed (and Q loaded on the first pass)
-            load_transposed<T, kDMax, kBK>(Kt, k, L, args.local, b, h, H, D, j, b0);
-            load_rowmajor<T, kDMax, kBK>(Vs, v, L, args.local, b, h, H, D, j, b0);
+            load_transposed<T, kDMax, kBK>(Kt, k, L, args.local, b, base, h, H, D, j, b0);
+            load_rowmajor<T, kDMax, kBK>(Vs, v, L, args.local, b, base, h, H, D, j, b0);
             __syncthreads();
 
             // S block: rows 4ty + r, keys 4tx + c
@@ -218,16 +238,20 @@ __global__ void __launch_bounds__(kThreads, kDMax <= 128 ? 2 : 1)
         const float inv_l = (l[r] > 0.f) ? 1.f / l[r] : 0.f;
         const float lse = (l[r] > 0.f) ? m[r] + logf(l[r]) : -INFINITY;
         if (args.out_mode == kOutFinal) {
-            const int64_t g = global_position(L, i, a);
-            T* dst = static_cast<T*>(args.out) + ((b * L.S + g) * H + h) * D;
+            const int64_t g = base + global_position(L, i, a);
+            T* dst = static_cast<T*>(args.out) + ((b * S_axis + g) * H + h) * D;
 #pragma unroll
             for (int c = 0; c < kOC; ++c) {
                 const int d = 4 * tx + 64 * (c / 4) + c % 4;
                 if (d < D) dst[d] = from_float<T>(o[r][c] * inv_l);
             }
-            if (tx == 0) args.lse[(b * H + h) * L.S + g] = lse;
+            if (tx == 0) args.lse[(b * H + h) * S_axis + g] = lse;
         } else {
-            const int64_t row = args.local ? (b * L.S_loc + a) * H + h : ((b * L.N + i) * L.S_loc + a) * H + h;
+            // partial rows: packed sequences in natural packed order, batch mode shard-major (or
+            // local rows for a ring step on local buffers)
+            const int64_t row = items ? (base + global_position(L, i, a)) * H + h
+                                : args.local ? (b * L.S_loc + a) * H + h
+                                             : ((b * L.N + i) * L.S_loc + a) * H + h;
             float* dst = static_cast<float*>(args.out) + row * D;
 #pragma unroll
             for (int c = 0; c < kOC; ++c) {
@@ -240,24 +264,26 @@ __global__ void __launch_bounds__(kThreads, kDMax <= 128 ? 2 : 1)
 }
 
 template <typename T, int kDMax>
-cudaError_t launch_typed(const void* q, const void* k, const void* v, const AttnArgs& a,
-                         cudaStream_t stream) {
+cudaError_t launch_typed(const void* q, const void* k, const void* v, const AttnArgs& a, const int4* items,
+                         int n_items, cudaStream_t stream) {
     const size_t smem = sizeof(float) * ((size_t)kDMax * kBQ + 2 * (size_t)kDMax * kBK + (size_t)kBK * kBQ);
     auto kern = attn_simt_kernel<T, kDMax>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    dim3 grid((unsigned)((a.L.S_loc + kBQ - 1) / kBQ), a.local ? 1u : (unsigned)a.L.N, (unsigned)(a.B * a.H));
+    const dim3 grid = items ? dim3((unsigned)n_items, 1u, (unsigned)a.H)
+                            : dim3((unsigned)((a.L.S_loc + kBQ - 1) / kBQ), a.local ? 1u : (unsigned)a.L.N,
+                                   (unsigned)(a.B * a.H));
     kern<<<grid, kThreads, smem, stream>>>(static_cast<const T*>(q), static_cast<const T*>(k),
-                                           static_cast<const T*>(v), a);
+                                           static_cast<const T*>(v), a, items);
     return cudaGetLastError();
 }
 
 template <typename T>
-cudaError_t launch_dispatch(const void* q, const void* k, const void* v, const AttnArgs& a,
-                            cudaStream_t stream) {
-    if (a.D <= 64) return launch_typed<T, 64>(q, k, v, a, stream);
-    if (a.D <= 128) return launch_typed<T, 128>(q, k, v, a, stream);
-    return launch_typed<T, 256>(q, k, v, a, stream);
+cudaError_t launch_dispatch(const void* q, const void* k, const void* v, const AttnArgs& a, const int4* items,
+                            int n_items, cudaStream_t stream) {
+    if (a.D <= 64) return launch_typed<T, 64>(q, k, v, a, items, n_items, stream);
+    if (a.D <= 128) return launch_typed<T, 128>(q, k, v, a, items, n_items, stream);
+    return launch_typed<T, 256>(q, k, v, a, items, n_items, stream);
 }
 
 }  // namespace
@@ -265,8 +291,15 @@ cudaError_t launch_dispatch(const void* q, const void* k, const void* v, const A
 cudaError_t launch_attn_simt(const void* q, const void* k, const void* v, const AttnArgs& a,
                              cudaStream_t stream) {
     if (a.B * a.H * a.L.S == 0) return cudaSuccess;
-    if (a.dtype == 0) return launch_dispatch<float>(q, k, v, a, stream);
-    return launch_dispatch<__nv_bfloat16>(q, k, v, a, stream);
+    if (a.dtype == 0) return launch_dispatch<float>(q, k, v, a, nullptr, 0, stream);
+    return launch_dispatch<__nv_bfloat16>(q, k, v, a, nullptr, 0, stream);
+}
+
+cudaError_t launch_attn_simt_packed(const void* q, const void* k, const void* v, const AttnArgs& a,
+                                    const int4* items, int n_items, cudaStream_t stream) {
+    if (n_items == 0 || a.H == 0) return cudaSuccess;
+    if (a.dtype == 0) return launch_dispatch<float>(q, k, v, a, items, n_items, stream);
+    return launch_dispatch<__nv_bfloat16>(q, k, v, a, items, n_items, stream);
 }
 
 }  // namespace ra

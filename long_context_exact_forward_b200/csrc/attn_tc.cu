@@ -670,8 +670,11 @@ struct Roles {
             row_dst = static_cast<uint8_t*>(A.out) + (((G.b * S + g) * H + G.h) * kD) * 2;
             lse_dst = A.lse + (G.b * H + G.h) * S + g;
         } else {
-            const int64_t rr = A.local ? ((int64_t)G.b * G.L.S_loc + a) * H + G.h
-                                       : (((int64_t)G.b * G.L.N + G.i) * G.L.S_loc + a) * H + G.h;
+            // packed sequences: natural packed rows; batch mode: shard-major (local rows for a ring
+            // step on local buffers)
+            const int64_t rr = kVarlen ? (G.base + (row_ok ? global_position(G.L, G.i, a) : 0)) * H + G.h
+                               : A.local ? ((int64_t)G.b * G.L.S_loc + a) * H + G.h
+                                         : (((int64_t)G.b * G.L.N + G.i) * G.L.S_loc + a) * H + G.h;
             row_dst = static_cast<uint8_t*>(A.out) + rr * kD * 4;
             lse_dst = A.lse + rr;
         }

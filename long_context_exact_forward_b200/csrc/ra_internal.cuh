@@ -24,9 +24,10 @@ struct AttnArgs {
     void* out;            // kOutFinal: [B, S, H, D] dtype; kOutPartial: fp32 [rows, D]
     float* lse;           // kOutFinal: [B, H, S]; kOutPartial: [rows]
     float scale;          // 1 / sqrt(D)
-    // Packed sequences (tensor-core kernel, fused, B = 1): work item x indexes `seqs`, each entry
-    // {S_k, first token of sequence k}; L then describes the whole packed axis (S = S_total) and
-    // every sequence is split into L.N shards with L.kind.  Null: batch mode (item x = batch b).
+    // Packed sequences (B = 1): work item x indexes `seqs`, each entry {S_k, first token of
+    // sequence k}; L then describes the whole packed axis (S = S_total) and every sequence is split
+    // into L.N shards with L.kind.  kOutPartial rows are then natural packed rows (token * H + h).
+    // Null: batch mode (item x = batch b).
     const int2* seqs;
     int varlen_striped;   // packed sequences with the striped layout inside each sequence
     // One ring step on one device's local buffers (kOutPartial only): q holds query shard
@@ -74,6 +75,11 @@ cudaError_t launch_merge_final(const float* O_r, const float* lse_r, const float
 // attn_simt.cu: CUDA-core attention over natural-order q, k, v (any layout, D <= 256).
 cudaError_t launch_attn_simt(const void* q, const void* k, const void* v, const AttnArgs& a,
                              cudaStream_t stream);
+// Packed sequences (a.seqs set, B = 1, a.L.S the packed length): block x takes items[x] =
+// {sequence, shard, 64-row query tile}, block z the head; kOutPartial rows are natural packed rows
+// (token * H + h).
+cudaError_t launch_attn_simt_packed(const void* q, const void* k, const void* v, const AttnArgs& a,
+                                    const int4* items, int n_items, cudaStream_t stream);
 
 // attn_tc.cu: tcgen05 attention over shard-major bf16 q, k, v (D in {64, 128}).
 struct TcLaunch {

@@ -35,6 +35,7 @@ The per-step compute and the final write are pluggable (`step_fn`, `finalize_fn`
 they are the library's ra_ring_step and ra_ring_finalize on the tensor's CUDA device.
 """
 import datetime
+import time
 
 import torch
 import torch.distributed as dist
@@ -82,15 +83,21 @@ class P2PExchange:
                 w.wait(timeout)
 
 
-def _abort_reason(store):
+def _abort_reason(store, wait_s=0.0):
+    """The reason a failed rank published, or None.  wait_s > 0 polls that long: after a transfer
+    failed, the peer that caused it may still be writing its reason."""
     if store is None:
         return None
-    try:
-        if store.check([ABORT_KEY]):
-            return store.get(ABORT_KEY).decode(errors="replace")
-    except Exception:  # a store that is itself gone tells us nothing more
-        return None
-    return None
+    deadline = time.monotonic() + wait_s
+    while True:
+        try:
+            if store.check([ABORT_KEY]):
+                return store.get(ABORT_KEY).decode(errors="replace")
+        except Exception:  # a store that is itself gone tells us nothing more
+            return None
+        if time.monotonic() >= deadline:
+            return None
+        time.sleep(0.05)
 
 
 def _publish_abort(store, rank, exc):
@@ -168,7 +175,12 @@ def ring_attention(q, k, v, causal=True, layout="striped", *, group=None, store=
         cur, nb = s % 2, (s + 1) % 2
         works = None
         if s + 1 < n:  # post the next block's transfer before this step's compute
-            works = exchange.start(bufs[cur], tags[cur], bufs[nb], tags[nb], nxt, prv, group)
+            try:
+                works = exchange.start(bufs[cur], tags[cur], bufs[nb], tags[nb], nxt, prv, group)
+            except Exception as exc:  # e.g. a peer that failed and closed its connections
+                reason = _abort_reason(store, wait_s=2.0)
+                raise RingError(f"rank {rank}: the transfer for step {s + 1} could not start"
+                                + (f" ({reason})" if reason else f" ({exc})")) from exc
         try:
             step_fn(q, bufs[cur][0], bufs[cur][1], O_acc, lse_acc, n, rank, s)
         except Exception as exc:
@@ -179,7 +191,7 @@ def ring_attention(q, k, v, causal=True, layout="striped", *, group=None, store=
         try:
             exchange.finish(works, timeout)
         except Exception as exc:
-            reason = _abort_reason(store)
+            reason = _abort_reason(store, wait_s=2.0)
             raise RingError(f"rank {rank}: block for step {s + 1} from rank {prv} did not arrive"
                             + (f" ({reason})" if reason else f" ({exc})")) from exc
         if check_now:

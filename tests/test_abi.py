@@ -96,43 +96,68 @@ def test_backward_rope_and_varlen_validate_before_any_cuda_call():
     assert lib.ra_rope(FAKE + 2, FAKE, 1, 4, 1, 4, 0, 10000.0, 0, None) == -3
     assert lib.ra_rope(FAKE, FAKE, 1, 4, 1 << 21, 256, 0, 10000.0, 0, None) == -2  # H * D above 2^28
     # ra_forward_varlen: a length not divisible by n_ring; under zigzag one not divisible by 2 n_ring;
-    # an unknown layout; cu[0] != 0
+    # an unknown layout; cu[0] != 0; an unknown dtype; a head dim above 256
     cu = np.array([0, 50, 100], dtype=np.int64)
-    assert lib.ra_forward_varlen(FAKE, FAKE, FAKE, FAKE, FAKE, cu.ctypes.data, 2, 1, 128, 4, 1, 0, None) == -2
+    assert lib.ra_forward_varlen(FAKE, FAKE, FAKE, FAKE, FAKE, cu.ctypes.data, 2, 1, 128, 4, 1, 0, 1, None) == -2
     cu = np.array([0, 64, 132], dtype=np.int64)
-    assert lib.ra_forward_varlen(FAKE, FAKE, FAKE, FAKE, FAKE, cu.ctypes.data, 2, 1, 128, 4, 1, 2, None) == -2
+    assert lib.ra_forward_varlen(FAKE, FAKE, FAKE, FAKE, FAKE, cu.ctypes.data, 2, 1, 128, 4, 1, 2, 1, None) == -2
     cu = np.array([0, 64, 128], dtype=np.int64)
-    assert lib.ra_forward_varlen(FAKE, FAKE, FAKE, FAKE, FAKE, cu.ctypes.data, 2, 1, 128, 4, 1, 3, None) == -1
+    assert lib.ra_forward_varlen(FAKE, FAKE, FAKE, FAKE, FAKE, cu.ctypes.data, 2, 1, 128, 4, 1, 3, 1, None) == -1
     cu = np.array([4, 64, 128], dtype=np.int64)
-    assert lib.ra_forward_varlen(FAKE, FAKE, FAKE, FAKE, FAKE, cu.ctypes.data, 2, 1, 128, 4, 1, 0, None) == -1
+    assert lib.ra_forward_varlen(FAKE, FAKE, FAKE, FAKE, FAKE, cu.ctypes.data, 2, 1, 128, 4, 1, 0, 1, None) == -1
+    cu = np.array([0, 64, 128], dtype=np.int64)
+    assert lib.ra_forward_varlen(FAKE, FAKE, FAKE, FAKE, FAKE, cu.ctypes.data, 2, 1, 128, 4, 1, 0, 2, None) == -1
+    assert lib.ra_forward_varlen(FAKE, FAKE, FAKE, FAKE, FAKE, cu.ctypes.data, 2, 1, 264, 4, 1, 0, 0, None) == -2
 
 
 def test_varlen_workspace_size_and_options_validate_on_the_host():
     lib = ra.lib()
     lengths = [1024, 0, 600 * 8, 48, 4096]
     cu = np.concatenate([[0], np.cumsum(lengths)]).astype(np.int64)
+    S = int(cu[-1])
     H, D, N = 3, 128, 8
     a256 = lambda x: -(-x // 256) * 256
-    items = sum(H * N * -(-(n // N) // 256) for n in lengths)
-    base = 256 + a256(len(lengths) * 8) + a256(items * 16) + a256(2 * H * 4)  # ..., norms per head
+    # one launch: counter, sequence table, work list, (tensor cores) norms per head
+    tc_items = sum(H * N * -(-(n // N) // 256) for n in lengths)
+    base = 256 + a256(len(lengths) * 8) + a256(tc_items * 16) + a256(2 * H * 4)
     assert ra.varlen_workspace_size(cu, H, D, N, "contiguous") == base
     assert ra.varlen_workspace_size(cu, H, D, N, "striped") == base
-    assert ra.varlen_workspace_size(cu, H, D, N, "zigzag") == base + 3 * a256(int(cu[-1]) * H * D * 2)
+    assert ra.varlen_workspace_size(cu, H, D, N, "zigzag") == base + 3 * a256(S * H * D * 2)
+    # per step: one counter per launch (N of them at one step per launch) and the fp32 running and
+    # partial results
+    acc = 2 * (a256(S * H * D * 4) + a256(S * H * 4))
+    assert ra.varlen_workspace_size(cu, H, D, N, "striped", 1, "per_step") == base + acc
+    assert ra.varlen_workspace_size(cu, H, D, 1, "striped", 1, "per_step") == \
+        256 + a256(len(lengths) * 8) + a256(sum(H * -(-n // 256) for n in lengths) * 16) + a256(2 * H * 4)
+    # CUDA cores: 64-row items over every head, no norms, no shard-major copies
+    simt_items = sum(N * -(-(n // N) // 64) for n in lengths)
+    simt = 256 + a256(len(lengths) * 8) + a256(simt_items * 16)
+    for layout in ("contiguous", "zigzag"):
+        assert ra.varlen_workspace_size(cu, H, D, N, layout, 1, "auto", "simt") == simt
+        assert ra.varlen_workspace_size(cu, H, D, N, layout, 0) == simt  # fp32: CUDA cores
+        assert ra.varlen_workspace_size(cu, H, 96, N, layout, 1) == simt  # D outside {64, 128}
+        assert ra.varlen_workspace_size(cu, H, D, N, layout, 0, "per_step") == simt + acc
     with pytest.raises(ra.RAError):  # 600 * 8 + 4 is not a multiple of 2N
         ra.varlen_workspace_size([0, 600 * 8 + 4], H, D, N, "zigzag")
+    with pytest.raises(ra.RAError):  # the tensor cores take bf16 only
+        ra.varlen_workspace_size(cu, H, D, N, "zigzag", 0, "auto", "tc")
 
-    def ex(variant=0, kernel=0, ws=None, nbytes=0, debug=0):
+    def ex(variant=0, kernel=0, ws=None, nbytes=0, debug=0, dtype=1, spl=0):
         opt = ra.Options()
-        opt.variant, opt.kernel, opt.debug = variant, kernel, debug
+        opt.variant, opt.kernel, opt.debug, opt.steps_per_launch = variant, kernel, debug, spl
         opt.workspace, opt.workspace_bytes = ws, nbytes
         return lib.ra_forward_varlen_ex(FAKE, FAKE, FAKE, FAKE, FAKE, cu.ctypes.data, len(lengths), H, D, N, 1, 2,
-                                        None, ctypes.byref(opt))
-    assert ex(variant=2) == -4                        # per-step variant not offered
-    assert ex(kernel=2) == -4                         # CUDA-core kernel not offered
+                                        dtype, None, ctypes.byref(opt))
+    assert ex(variant=3) == -1                        # unknown variant
+    assert ex(kernel=3) == -1                         # unknown kernel
+    assert ex(kernel=1, dtype=0) == -4                # tensor cores on fp32
+    assert ex(spl=-1, variant=2) == -1
     assert ex(debug=9) == -1
     need = ra.varlen_workspace_size(cu, H, D, N, "zigzag")
     assert ex(ws=FAKE + 16, nbytes=need) == -3        # workspace not 256-byte aligned
     assert ex(ws=FAKE, nbytes=need - 1) == -5         # workspace too small
+    need = ra.varlen_workspace_size(cu, H, D, N, "zigzag", 1, "per_step")
+    assert ex(variant=2, spl=3, ws=FAKE, nbytes=need - acc) == -5  # 3 launches need the results
 
 
 def test_ring_step_validates_before_any_cuda_call():

@@ -260,7 +260,9 @@ def test_caller_outputs_of_the_wrong_size_are_refused_before_launch():
         ra.backward(q, k, v, q, torch.zeros((B, H, S), device="cuda"), q, N, True, "striped", dq=short)
     with pytest.raises(ValueError):
         ra.rope(q, out=short)
-    with pytest.raises(TypeError):
-        ra.forward_varlen(q[0].float(), k[0].float(), v[0].float(), [0, S], N)
+    with pytest.raises(TypeError):  # fp16 is not a supported dtype
+        ra.forward_varlen(q[0].half(), k[0].half(), v[0].half(), [0, S], N)
+    with pytest.raises(TypeError):  # mixed dtypes
+        ra.forward_varlen(q[0], k[0].float(), v[0], [0, S], N)
     torch.cuda.synchronize()
     assert ra.get_device_status() == 0

@@ -100,6 +100,7 @@ class DroppingExchange:
 
 def _worker(rank, world, port, cfg, results):
     code = 0
+    store = None
     try:
         sys.path.insert(0, ROOT)
         import torch.distributed as dist
@@ -139,6 +140,15 @@ def _worker(rank, world, port, cfg, results):
     finally:
         results.close()
         results.join_thread()
+        if store is not None:  # rank 0 hosts the store: keep it up until every rank has reported
+            try:
+                store.add("ring_test/done", 1)
+                if rank == 0:
+                    deadline = time.time() + 15
+                    while store.add("ring_test/done", 0) < world and time.time() < deadline:
+                        time.sleep(0.05)
+            except Exception:
+                pass
         os._exit(code)  # pending gloo requests of a failed ring must not hold the process
 
 
