@@ -80,6 +80,23 @@ def test_simt_fp32(shape, layout, causal, variant):
     run_case(B, H, S, D, N, causal, layout, torch.float32, variant, kernel="simt", seed=S + D)
 
 
+# several 64-key tiles per ring step and a ragged last tile: the pipelined CUDA-core form (rows of
+# whole 16-byte vectors) prefetches the next tile across tile and step boundaries; D = 200 takes its
+# single-stage form, D = 20 (fp32) and D = 36 (bf16) the synchronous form
+SIMT_MULTI_TILE = [(1, 2, 4 * 300, 64, 4, torch.float32), (1, 1, 2 * 200, 128, 2, torch.float32),
+                   (1, 1, 2 * 160, 200, 2, torch.float32), (1, 2, 4 * 200, 64, 4, torch.bfloat16),
+                   (1, 1, 2 * 264, 128, 2, torch.bfloat16), (1, 1, 2 * 150, 20, 2, torch.float32),
+                   (1, 1, 2 * 150, 36, 2, torch.bfloat16)]
+
+
+@pytest.mark.parametrize("shape", SIMT_MULTI_TILE)
+@pytest.mark.parametrize("layout", ["contiguous", "striped", "zigzag"])
+@pytest.mark.parametrize("causal", [False, True])
+def test_simt_multi_tile(shape, layout, causal):
+    B, H, S, D, N, dtype = shape
+    run_case(B, H, S, D, N, causal, layout, dtype, "fused", kernel="simt", seed=S + 3 * D)
+
+
 @pytest.mark.parametrize("layout", ["contiguous", "striped", "zigzag"])
 @pytest.mark.parametrize("variant", ["fused", "per_step"])
 def test_simt_bf16_odd_head_dim(layout, variant):
