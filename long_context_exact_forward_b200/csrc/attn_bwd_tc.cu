@@ -24,9 +24,10 @@
 //                    the elementwise warps write P^T over S^T and dS^T over dP^T (bf16), then
 //                    dV += P^T dO and dK += dS^T Q (TS, dO and Q as MN-major operands).
 //
-// Roles (192 threads): warp 0 TMA producer (lane 0 issues), warp 1 MMA issuer (converged warp,
-// elect.sync picks the issuing lane) and TMEM owner, warps 2-5 elementwise (warp w reads TMEM lanes
-// 32 (w mod 4) .. +31).  The streamed tiles go through two shared-memory stages.  Every wait is
+// Roles (320 threads): warp 0 TMA producer (lane 0 issues), warp 1 MMA issuer (converged warp,
+// elect.sync picks the issuing lane) and TMEM owner, warps 2-9 elementwise: warp w reads TMEM lanes
+// 32 (w mod 4) .. +31, warps 2-5 the columns 0..63 of every tile and warps 6-9 the columns 64..127
+// (the elementwise steps have no row reductions, so the two halves never meet).  The streamed tiles go through two shared-memory stages.  Every wait is
 // bounded; on give-up the CTA records RA_ERR_DEVICE_TIMEOUT, lets its copies and MMAs drain, frees
 // TMEM and exits.
 #include <cuda_bf16.h>
@@ -40,7 +41,8 @@ namespace {
 using namespace sm100;
 
 constexpr int kTile = 128;
-constexpr int kThreads = 192;
+constexpr int kThreads = 320;
+constexpr int kEwWarps = 8;  // elementwise warps: two per TMEM lane quadrant, one per 64-column half
 constexpr int kProducerWarp = 0, kMmaWarp = 1;
 constexpr uint32_t kTmemCols = 512;
 constexpr float kLog2e = 1.4426950408889634f;
@@ -116,15 +118,22 @@ __device__ __forceinline__ void mma_tile_ss(uint32_t d_tmem, const uint8_t* a, c
     }
 }
 
-// D[tmem] (+)= A[tmem, bf16, 128 x 128] B, B an MN-major 128 x kD tile in shared memory (TS, N = kD)
+// Packed bf16 A operands of the TS products (dS in the dq kernel; P^T and dS^T in the dk/dv kernel)
+// are written over the fp32 tile they are computed from.  The 32 columns of chunk c (c = 0..3) go to
+// TMEM columns 64 (c / 2) + 16 (c mod 2) .. +15: each of the two warps of a lane quadrant, which take
+// columns 0..63 and 64..127, then overwrites only columns it has already read itself.
+__device__ __forceinline__ uint32_t packed_col(int c) { return 64u * (uint32_t)(c >> 1) + 16u * (uint32_t)(c & 1); }
+
+// D[tmem] (+)= A[tmem, bf16, 128 x 128, packed as above] B, B an MN-major 128 x kD tile in shared
+// memory (TS, N = kD); K-step kk (16 columns of A = 8 TMEM columns) sits at 64 (kk / 4) + 8 (kk mod 4)
 template <int kD>
 __device__ __forceinline__ void mma_tile_ts(uint32_t d_tmem, uint32_t a_tmem, const uint8_t* b, bool accumulate) {
     constexpr uint32_t idesc = idesc_bf16_f32(kTile, kD, 0, 1);
     const uint32_t ba = smem_addr(b);
 #pragma unroll
     for (int kk = 0; kk < kTile / 16; ++kk)
-        warp_mma_ts(d_tmem, a_tmem + kk * 8, smem_desc_sw128(ba + kk * 16 * 128, kColBlockBytes, 1024), idesc,
-                    (kk > 0 || accumulate) ? 1u : 0u);
+        warp_mma_ts(d_tmem, a_tmem + 64u * (kk >> 2) + 8u * (kk & 3),
+                    smem_desc_sw128(ba + kk * 16 * 128, kColBlockBytes, 1024), idesc, (kk > 0 || accumulate) ? 1u : 0u);
 }
 
 // Number of live 128-key tiles of block j for the query tile at a0 of shard i.
@@ -183,7 +192,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         mbar_init(&sm.s_full, 1);
         mbar_init(&sm.dp_full, 1);
-        mbar_init(&sm.ds_full, 4);
+        mbar_init(&sm.ds_full, kEwWarps);
         mbar_init(&sm.acc_full, 1);
         mbar_init(&sm.drain, 1);
         sm.abort = 0;
@@ -272,7 +281,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_wait(&sm.drain, 0, timeout, nullptr);
         }
     } else {
-        // elementwise: row r of the query tile
+        // elementwise: row r of the query tile, columns 64 half .. 64 half + 63 of each key tile
+        const int half = (warp - 2) >> 2;
         const int r = 32 * (warp & 3) + lane;
         const int a = a0 + r;
         const bool row_ok = a < L.S_loc;
@@ -300,7 +310,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int valid = cnt - kt * kTile;
                 const uint32_t kS = 128 * (it & 1);
 #pragma unroll 1
-                for (int c = 0; c < kTile / 32; ++c) {
+                for (int c = 2 * half; c < 2 * half + 2; ++c) {
                     uint32_t sv[32], pv[32], pk[16];
                     tmem_ld32(lane_base + kS + 32 * c, sv);
                     tmem_ld32(lane_base + kdP + 32 * c, pv);
@@ -317,8 +327,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                         }
                         pk[x] = pack_bf16x2(ds[0], ds[1]);
                     }
-                    // dS of columns 32c..32c+31 -> TMEM columns 16c..16c+15 (already read)
-                    tmem_st16(lane_base + kS + 16 * c, pk);
+                    // dS of columns 32c..32c+31 -> TMEM columns packed_col(c)..+15 (already read)
+                    tmem_st16(lane_base + kS + packed_col(c), pk);
                 }
                 tmem_wait_st();
                 tc_fence_before();
@@ -326,11 +336,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (lane == 0) mbar_arrive(&sm.ds_full);
             }
         }
+        // each warp of a quadrant stores its half of the head dims
         if (ok && any) {
             if (wait_all(&sm.acc_full, 0)) {
                 __nv_bfloat16* dst = A.dq + (((size_t)b * L.S + g) * A.H + h) * A.D;
 #pragma unroll 1
-                for (int c = 0; c < kD / 32; ++c) {
+                for (int c = half * (kD / 64); c < (half + 1) * (kD / 64); ++c) {
                     uint32_t v[32];
                     tmem_ld32(lane_base + kdQ + 32 * c, v);
                     wait_ld_tied(v);
@@ -339,7 +350,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         } else if (ok && row_ok) {  // no visible key at all: the gradient is zero
             __nv_bfloat16* dst = A.dq + (((size_t)b * L.S + g) * A.H + h) * A.D;
-            for (int d = 0; d < kD; ++d) dst[d] = __float2bfloat16_rn(0.f);
+            for (int d = half * (kD / 2); d < (half + 1) * (kD / 2); ++d) dst[d] = __float2bfloat16_rn(0.f);
         }
         if (!ok && lane == 0) give_up(abort, A.status);
     }
@@ -377,7 +388,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         mbar_init(&sm.s_full, 1);
         mbar_init(&sm.dp_full, 1);
-        mbar_init(&sm.ds_full, 4);
+        mbar_init(&sm.ds_full, kEwWarps);
         mbar_init(&sm.acc_full, 1);
         mbar_init(&sm.drain, 1);
         sm.abort = 0;
@@ -483,7 +494,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_wait(&sm.drain, 0, timeout, nullptr);
         }
     } else {
-        // elementwise: row r = key c0 + r of this tile, columns = the 128 query rows of a tile
+        // elementwise: row r = key c0 + r of this tile, columns = the query rows 64 half .. 64 half + 63
+        // of a query tile
+        const int half = (warp - 2) >> 2;
         const int r = 32 * (warp & 3) + lane;
         const int key = c0 + r;
         const bool row_ok = key < L.S_loc;
@@ -508,10 +521,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (!wait_all(&sm.s_full, it & 1)) break;
                 if (!wait_all(&sm.stage_full[st], (it >> 1) & 1)) break;  // the query statistics
                 any = true;
-                // phase 1 (S^T ready): P^T = exp(S^T / sqrt(D) - lse), bf16, over the first 64
-                // columns of S^T (chunk c writes columns 16c.., already read)
+                // phase 1 (S^T ready): P^T = exp(S^T / sqrt(D) - lse), bf16, written over S^T
+                // (chunk c writes columns packed_col(c).., already read by this warp)
 #pragma unroll 1
-                for (int c = 0; c < kTile / 32; ++c) {
+                for (int c = 2 * half; c < 2 * half + 2; ++c) {
                     uint32_t sv[32], pk[16];
                     tmem_ld32(lane_base + kST + 32 * c, sv);
                     wait_ld_tied(sv);
@@ -540,17 +553,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                             pk[x] = pack_bf16x2(p[0], p[1]);
                         }
                     }
-                    tmem_st16(lane_base + kST + 16 * c, pk);
+                    tmem_st16(lane_base + kST + packed_col(c), pk);
                 }
-                // phase 2 (dP^T ready): dS^T = P^T (dP^T - Delta) from the stored bf16 P^T, over the
-                // first 64 columns of dP^T
+                // phase 2 (dP^T ready): dS^T = P^T (dP^T - Delta) from the stored bf16 P^T, written
+                // over dP^T in the same packed columns
                 tmem_wait_st();
                 if (!wait_all(&sm.dp_full, it & 1)) break;
 #pragma unroll 1
-                for (int c = 0; c < kTile / 32; ++c) {
+                for (int c = 2 * half; c < 2 * half + 2; ++c) {
                     uint32_t pv[32], pb[16], dk16[16];
                     tmem_ld32(lane_base + kdPT + 32 * c, pv);
-                    tmem_ld16(lane_base + kST + 16 * c, pb);
+                    tmem_ld16(lane_base + kST + packed_col(c), pb);
                     wait_ld_tied(pv);
                     wait_ld_tied(pb);
                     const float4* d4 = reinterpret_cast<const float4*>(&sm.col_delta[st][32 * c]);
@@ -563,7 +576,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         dk16[2 * x + 1] = pack_bf16x2(__uint_as_float(b1 << 16) * (__uint_as_float(pv[4 * x + 2]) - dv.z),
                                                       __uint_as_float(b1 & 0xffff0000u) * (__uint_as_float(pv[4 * x + 3]) - dv.w));
                     }
-                    tmem_st16(lane_base + kdPT + 16 * c, dk16);
+                    tmem_st16(lane_base + kdPT + packed_col(c), dk16);
                 }
                 tmem_wait_st();
                 tc_fence_before();
@@ -574,10 +587,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         __nv_bfloat16* dkr = A.dk + (((size_t)b * L.S + gk) * A.H + h) * A.D;
         __nv_bfloat16* dvr = A.dv + (((size_t)b * L.S + gk) * A.H + h) * A.D;
+        // each warp of a quadrant stores its half of the head dims
         if (ok && any) {
             if (wait_all(&sm.acc_full, 0)) {
 #pragma unroll 1
-                for (int c = 0; c < kD / 32; ++c) {
+                for (int c = half * (kD / 64); c < (half + 1) * (kD / 64); ++c) {
                     uint32_t v[32];
                     tmem_ld32(lane_base + kdV + 32 * c, v);
                     wait_ld_tied(v);
@@ -588,7 +602,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
             }
         } else if (ok && row_ok) {  // no query sees these keys: the gradients are zero
-            for (int d = 0; d < kD; ++d) {
+            for (int d = half * (kD / 2); d < (half + 1) * (kD / 2); ++d) {
                 dkr[d] = __float2bfloat16_rn(0.f);
                 dvr[d] = __float2bfloat16_rn(0.f);
             }
