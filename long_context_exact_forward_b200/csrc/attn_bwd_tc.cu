@@ -418,6 +418,20 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (!query_tile_live(L, A.causal, i, q0, j, c0)) continue;
                 const uint32_t st = it & 1;
                 if (A.debug == RA_DEBUG_STALL_LOADS) break;  // consumers must time out
+                // lse (log2 units) and Delta of the tile's query rows, for the elementwise warps: read
+                // before the stage frees, so that the gather's latency overlaps the wait
+                float l2[kTile / 32], dl[kTile / 32];
+#pragma unroll
+                for (int e = 0; e < kTile / 32; ++e) {
+                    const int a = q0 + lane * (kTile / 32) + e;
+                    l2[e] = 0.f;
+                    dl[e] = 0.f;
+                    if (a < L.S_loc) {
+                        const size_t ix = ((size_t)b * A.H + h) * L.S + global_position(L, i, a);
+                        l2[e] = __ldg(A.lse + ix) * kLog2e;
+                        dl[e] = __ldg(A.delta + ix);
+                    }
+                }
                 ok = __all_sync(0xffffffffu, mbar_wait(&sm.stage_empty[st], ((it >> 1) & 1) ^ 1, timeout, abort));
                 if (!ok) break;
                 if (lane == 0) {
@@ -425,18 +439,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tma_tile(sm.stream[st][0], &tm_q, &sm.stage_full[st], kD, h, q0, i, b);
                     tma_tile(sm.stream[st][1], &tm_do, &sm.stage_full[st], kD, h, q0, i, b);
                 }
-                // lse (log2 units) and Delta of the tile's query rows, for the elementwise warps
 #pragma unroll
                 for (int e = 0; e < kTile / 32; ++e) {
-                    const int r = lane * (kTile / 32) + e, a = q0 + r;
-                    float l2 = 0.f, dl = 0.f;
-                    if (a < L.S_loc) {
-                        const size_t ix = ((size_t)b * A.H + h) * L.S + global_position(L, i, a);
-                        l2 = A.lse[ix] * kLog2e;
-                        dl = A.delta[ix];
-                    }
-                    sm.col_lse2[st][r] = l2;
-                    sm.col_delta[st][r] = dl;
+                    const int r = lane * (kTile / 32) + e;
+                    sm.col_lse2[st][r] = l2[e];
+                    sm.col_delta[st][r] = dl[e];
                 }
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&sm.stage_full[st]);
