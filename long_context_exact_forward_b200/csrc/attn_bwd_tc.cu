@@ -94,6 +94,18 @@ __device__ __forceinline__ void wait_ld_tied(uint32_t (&r)[N]) {
 #pragma unroll
     for (int x = 0; x < N; ++x) asm volatile("" : "+r"(r[x]));
 }
+// Tie more registers to the wait just made (the wait covers every load issued before it).
+template <int N>
+__device__ __forceinline__ void tie_regs(uint32_t (&r)[N]) {
+#pragma unroll
+    for (int x = 0; x < N; ++x) asm volatile("" : "+r"(r[x]));
+}
+
+// mbar_wait preceded by a non-blocking probe: a phase that has already completed (the common case
+// for the barriers the elementwise warps check second) costs one test instead of a try_wait.
+__device__ __forceinline__ bool bar_wait(uint64_t* bar, uint32_t parity, uint64_t timeout, volatile int* abort) {
+    return mbar_test_wait(bar, parity) || mbar_wait(bar, parity, timeout, abort);
+}
 
 __device__ __forceinline__ void give_up(volatile int* abort, int* status) {
     *abort = 1;
@@ -244,7 +256,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         bool ok = true;
         auto wait = [&](uint64_t* bar, uint32_t parity) {
             if (!ok) return false;
-            ok = __all_sync(0xffffffffu, mbar_wait(bar, parity, timeout, abort));
+            ok = __all_sync(0xffffffffu, bar_wait(bar, parity, timeout, abort));
             if (ok) tc_fence_after();
             return ok;
         };
@@ -294,7 +306,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float sl2 = A.scale * kLog2e;
         bool ok = true;
         auto wait_all = [&](uint64_t* bar, uint32_t parity) {
-            ok = __all_sync(0xffffffffu, mbar_wait(bar, parity, timeout, abort));
+            ok = __all_sync(0xffffffffu, bar_wait(bar, parity, timeout, abort));
             if (ok) tc_fence_after();
             return ok;
         };
@@ -460,7 +472,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         bool ok = true;
         auto wait = [&](uint64_t* bar, uint32_t parity) {
             if (!ok) return false;
-            ok = __all_sync(0xffffffffu, mbar_wait(bar, parity, timeout, abort));
+            ok = __all_sync(0xffffffffu, bar_wait(bar, parity, timeout, abort));
             if (ok) tc_fence_after();
             return ok;
         };
@@ -512,7 +524,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int gk = row_ok ? global_position(L, j, key) : 0;
         bool ok = true;
         auto wait_all = [&](uint64_t* bar, uint32_t parity) {
-            ok = __all_sync(0xffffffffu, mbar_wait(bar, parity, timeout, abort));
+            ok = __all_sync(0xffffffffu, bar_wait(bar, parity, timeout, abort));
             if (ok) tc_fence_after();
             return ok;
         };
@@ -529,12 +541,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (!wait_all(&sm.stage_full[st], (it >> 1) & 1)) break;  // the query statistics
                 any = true;
                 // phase 1 (S^T ready): P^T = exp(S^T / sqrt(D) - lse), bf16, written over S^T
-                // (chunk c writes columns packed_col(c).., already read by this warp)
-#pragma unroll 1
-                for (int c = 2 * half; c < 2 * half + 2; ++c) {
-                    uint32_t sv[32], pk[16];
-                    tmem_ld32(lane_base + kST + 32 * c, sv);
-                    wait_ld_tied(sv);
+                // (chunk c writes columns packed_col(c).., already read by this warp).  Both of the
+                // warp's chunks are loaded at once, so that one TMEM round trip serves them.
+                auto phase1 = [&](int c, const uint32_t (&sv)[32]) {
+                    uint32_t pk[16];
                     const float4* l4 = reinterpret_cast<const float4*>(&sm.col_lse2[st][32 * c]);
                     // every query of this chunk sees the key: no per-element check (the common case)
                     const bool all_vis = q0 + 32 * c >= a_min && q0 + 32 * c + 31 < L.S_loc;
@@ -561,18 +571,23 @@ __global__ void __launch_bounds__(kThreads, 1)
                         }
                     }
                     tmem_st16(lane_base + kST + packed_col(c), pk);
+                };
+                {
+                    const int c0 = 2 * half;
+                    uint32_t sv0[32], sv1[32];
+                    tmem_ld32(lane_base + kST + 32 * c0, sv0);
+                    tmem_ld32(lane_base + kST + 32 * (c0 + 1), sv1);
+                    wait_ld_tied(sv0);
+                    tie_regs(sv1);
+                    phase1(c0, sv0);
+                    phase1(c0 + 1, sv1);
                 }
                 // phase 2 (dP^T ready): dS^T = P^T (dP^T - Delta) from the stored bf16 P^T, written
                 // over dP^T in the same packed columns
                 tmem_wait_st();
                 if (!wait_all(&sm.dp_full, it & 1)) break;
-#pragma unroll 1
-                for (int c = 2 * half; c < 2 * half + 2; ++c) {
-                    uint32_t pv[32], pb[16], dk16[16];
-                    tmem_ld32(lane_base + kdPT + 32 * c, pv);
-                    tmem_ld16(lane_base + kST + packed_col(c), pb);
-                    wait_ld_tied(pv);
-                    wait_ld_tied(pb);
+                auto phase2 = [&](int c, const uint32_t (&pv)[32], const uint32_t (&pb)[16]) {
+                    uint32_t dk16[16];
                     const float4* d4 = reinterpret_cast<const float4*>(&sm.col_delta[st][32 * c]);
 #pragma unroll
                     for (int x = 0; x < 8; ++x) {
@@ -584,6 +599,20 @@ __global__ void __launch_bounds__(kThreads, 1)
                                                       __uint_as_float(b1 & 0xffff0000u) * (__uint_as_float(pv[4 * x + 3]) - dv.w));
                     }
                     tmem_st16(lane_base + kdPT + packed_col(c), dk16);
+                };
+                {  // both chunks' loads at once, as in phase 1
+                    const int c0 = 2 * half;
+                    uint32_t pv0[32], pb0[16], pv1[32], pb1[16];
+                    tmem_ld32(lane_base + kdPT + 32 * c0, pv0);
+                    tmem_ld16(lane_base + kST + packed_col(c0), pb0);
+                    tmem_ld32(lane_base + kdPT + 32 * (c0 + 1), pv1);
+                    tmem_ld16(lane_base + kST + packed_col(c0 + 1), pb1);
+                    wait_ld_tied(pv0);
+                    tie_regs(pb0);
+                    tie_regs(pv1);
+                    tie_regs(pb1);
+                    phase2(c0, pv0, pb0);
+                    phase2(c0 + 1, pv1, pb1);
                 }
                 tmem_wait_st();
                 tc_fence_before();
