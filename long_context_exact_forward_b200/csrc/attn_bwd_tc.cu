@@ -322,12 +322,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int valid = cnt - kt * kTile;
                 const uint32_t kS = 128 * (it & 1);
 #pragma unroll 1
-                for (int c = 2 * half; c < 2 * half + 2; ++c) {
-                    uint32_t sv[32], pv[32], pk[16];
-                    tmem_ld32(lane_base + kS + 32 * c, sv);
-                    tmem_ld32(lane_base + kdP + 32 * c, pv);
-                    wait_ld_tied(sv);
-                    wait_ld_tied(pv);
+                auto chunk = [&](int c, const uint32_t (&sv)[32], const uint32_t (&pv)[32]) {
+                    uint32_t pk[16];
 #pragma unroll
                     for (int x = 0; x < 16; ++x) {
                         float ds[2];
@@ -341,6 +337,20 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     // dS of columns 32c..32c+31 -> TMEM columns packed_col(c)..+15 (already read)
                     tmem_st16(lane_base + kS + packed_col(c), pk);
+                };
+                {  // the second chunk's loads run while the first is computed
+                    const int c0 = 2 * half;
+                    uint32_t sv0[32], pv0[32], sv1[32], pv1[32];
+                    tmem_ld32(lane_base + kS + 32 * c0, sv0);
+                    tmem_ld32(lane_base + kdP + 32 * c0, pv0);
+                    wait_ld_tied(sv0);
+                    tie_regs(pv0);
+                    tmem_ld32(lane_base + kS + 32 * (c0 + 1), sv1);
+                    tmem_ld32(lane_base + kdP + 32 * (c0 + 1), pv1);
+                    chunk(c0, sv0, pv0);
+                    wait_ld_tied(sv1);
+                    tie_regs(pv1);
+                    chunk(c0 + 1, sv1, pv1);
                 }
                 tmem_wait_st();
                 tc_fence_before();
