@@ -547,8 +547,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int q0 = 0; q0 < L.S_loc && ok; q0 += kTile) {
                 if (!query_tile_live(L, A.causal, i, q0, j, c0)) continue;
                 const uint32_t st = it & 1;
+                // the query statistics first: they land with the tile's copies, well before S^T, so
+                // this check overlaps the wait for S^T instead of following it (no TMEM access
+                // depends on it, hence no tcgen05 fence)
+                ok = __all_sync(0xffffffffu, bar_wait(&sm.stage_full[st], (it >> 1) & 1, timeout, abort));
+                if (!ok) break;
                 if (!wait_all(&sm.s_full, it & 1)) break;
-                if (!wait_all(&sm.stage_full[st], (it >> 1) & 1)) break;  // the query statistics
                 any = true;
                 // phase 1 (S^T ready): P^T = exp(S^T / sqrt(D) - lse), bf16, written over S^T
                 // (chunk c writes columns packed_col(c).., already read by this warp).  Both of the
