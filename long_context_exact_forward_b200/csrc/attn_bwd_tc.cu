@@ -614,18 +614,18 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     tmem_st16(lane_base + kdPT + packed_col(c), dk16);
                 };
-                {  // both chunks' loads at once, as in phase 1
+                {  // the second chunk's loads run while the first chunk is computed
                     const int c0 = 2 * half;
                     uint32_t pv0[32], pb0[16], pv1[32], pb1[16];
                     tmem_ld32(lane_base + kdPT + 32 * c0, pv0);
                     tmem_ld16(lane_base + kST + packed_col(c0), pb0);
-                    tmem_ld32(lane_base + kdPT + 32 * (c0 + 1), pv1);
-                    tmem_ld16(lane_base + kST + packed_col(c0 + 1), pb1);
                     wait_ld_tied(pv0);
                     tie_regs(pb0);
-                    tie_regs(pv1);
-                    tie_regs(pb1);
+                    tmem_ld32(lane_base + kdPT + 32 * (c0 + 1), pv1);
+                    tmem_ld16(lane_base + kST + packed_col(c0 + 1), pb1);
                     phase2(c0, pv0, pb0);
+                    wait_ld_tied(pv1);
+                    tie_regs(pb1);
                     phase2(c0 + 1, pv1, pb1);
                 }
                 tmem_wait_st();

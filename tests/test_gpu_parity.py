@@ -81,12 +81,13 @@ def test_simt_fp32(shape, layout, causal, variant):
 
 
 # several 64-key tiles per ring step and a ragged last tile: the pipelined CUDA-core form (rows of
-# whole 16-byte vectors) prefetches the next tile across tile and step boundaries; D = 200 takes its
-# single-stage form, D = 20 (fp32) and D = 36 (bf16) the synchronous form
+# whole 16-byte vectors) prefetches the next tile across tile and step boundaries; D = 200 (fp32)
+# takes its single-stage form, D = 256 (bf16) two stages at 210 KB of shared memory, D = 20 (fp32)
+# and D = 36 (bf16) the synchronous form
 SIMT_MULTI_TILE = [(1, 2, 4 * 300, 64, 4, torch.float32), (1, 1, 2 * 200, 128, 2, torch.float32),
                    (1, 1, 2 * 160, 200, 2, torch.float32), (1, 2, 4 * 200, 64, 4, torch.bfloat16),
-                   (1, 1, 2 * 264, 128, 2, torch.bfloat16), (1, 1, 2 * 150, 20, 2, torch.float32),
-                   (1, 1, 2 * 150, 36, 2, torch.bfloat16)]
+                   (1, 1, 2 * 264, 128, 2, torch.bfloat16), (1, 1, 2 * 160, 256, 2, torch.bfloat16),
+                   (1, 1, 2 * 150, 20, 2, torch.float32), (1, 1, 2 * 150, 36, 2, torch.bfloat16)]
 
 
 @pytest.mark.parametrize("shape", SIMT_MULTI_TILE)
