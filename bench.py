@@ -541,13 +541,17 @@ def run_ours(args, w):
     # CUDA-core kernel reads natural order) and the attention launch(es) -- with chunks of C ring
     # steps per launch: ceil(N / C) attention launches and one merge after each but the first
     # (2 kernels each, the last one a single final merge)
-    # the tensor-core path also launches the query/key norm pre-pass (one kernel per call)
+    # the tensor-core path also launches the query/key norm pre-pass (one kernel per call) when it pays
     chunk = ra.steps_per_launch(S, D, N, args.layout, 0 if fp32 else 1, args.variant, args.steps_per_launch)
     if args.varlen:  # packed sequences: one launch unless per-step launches are asked for
         chunk = min(N, args.steps_per_launch or 1) if args.variant == "per_step" else N
     n_att = -(-N // chunk)
     tc = args.kernel == "tc"
-    launches_per_step = (1 if args.layout == "zigzag" and tc else 0) + (1 if tc else 0) + (
+    # the score-bound pre-pass runs when each query row meets >= 65536 keys per launch (RA_DEBUG_FROZEN_MAX
+    # in include/ra.h): chunk x S/N keys, or for packed sequences sum(len^2) / S of them per ring pass
+    keys_per_row = (sum(n * n for n in varlen_lengths(S, N, w.seed)) / S if args.varlen else S) * chunk / N
+    norms = 1 if tc and keys_per_row >= 65536 else 0
+    launches_per_step = (1 if args.layout == "zigzag" and tc else 0) + norms + (
         1 if n_att == 1 else n_att + 2 * (n_att - 2) + 1)
     if args.backward:
         # Delta, dq, dk/dv; the tensor-core kernels read zigzag from one shard-major permute launch

@@ -38,6 +38,7 @@ LAYOUTS = {"contiguous": 0, "striped": 1, "zigzag": 2}
 VARIANTS = {"auto": 0, "fused": 1, "per_step": 2}
 KERNELS = {"auto": 0, "tc": 1, "simt": 2}
 DEBUG_STALL_LOADS = 1
+DEBUG_FROZEN_MAX = 2   # score-bound pre-pass and frozen row max at any size (tests)
 
 RA_OK = 0
 STATUS = {

@@ -558,7 +558,9 @@ int run_forward(const Call& c, const ra_options& opt) {
             return finish(cuda_fail(e, "work list upload"));
         if ((e = cudaMemsetAsync(ws + w.counters, 0, w.n_counters * sizeof(int), c.stream)) != cudaSuccess)
             return finish(cuda_fail(e, "work counter reset"));
-        if (ra::key_norm_max_applies(c.B, c.H, c.D)) {  // the score bound of every query row (frozen max)
+        if (ra::key_norm_max_applies(c.B, c.H, c.D) &&
+            ra::frozen_max_pays((int64_t)w.chunk * L.S_loc, opt.debug == RA_DEBUG_FROZEN_MAX)) {
+            // the score bound of every query row (frozen max)
             float* nmax = reinterpret_cast<float*>(ws + w.kmax);
             nvtxRangePushA("ra_forward query and key norms");
             e = ra::launch_norm_max(c.q, c.k, nmax, c.B, c.S, c.H, c.D, dev.sms, c.stream);
@@ -940,7 +942,8 @@ int ra_ring_step(const void* q_i, const void* k_j, const void* v_j, float* O_acc
             return nvtx_pop(finish(cuda_fail(e, "work list upload")));
         if ((e = cudaMemsetAsync(ws + w.counter, 0, sizeof(int), stream)) != cudaSuccess)
             return nvtx_pop(finish(cuda_fail(e, "work counter reset")));
-        if (ra::key_norm_max_applies(B, H, D)) {  // the score bound over query shard i and key block j
+        if (ra::key_norm_max_applies(B, H, D) && ra::frozen_max_pays(L.S_loc, false)) {
+            // the score bound over query shard i and key block j
             float* nmax = reinterpret_cast<float*>(ws + w.kmax);
             if ((e = ra::launch_norm_max(q_i, k_j, nmax, B, L.S_loc, H, D, dev.sms, stream)) != cudaSuccess)
                 return nvtx_pop(finish(cuda_fail(e, "norm launch")));

@@ -219,7 +219,8 @@ extern "C" int ra_forward_noalloc(const void* q, const void* k, const void* v, v
     a.out = out;
     a.lse = lse;
     a.scale = (float)(1.0 / sqrt((double)D));
-    if (ra::key_norm_max_applies(B, H, D)) {  // the score bound of every query row (frozen max)
+    if (ra::key_norm_max_applies(B, H, D) && ra::frozen_max_pays(S, false)) {
+        // the score bound of every query row (frozen max)
         float* nmax = reinterpret_cast<float*>(scratch + counter_bytes + items_bytes);
         if ((e = ra::launch_norm_max(q, k, nmax, B, S, H, D, sms, stream)) != cudaSuccess)
             return ra::host_cuda_fail(e, "norm launch");

@@ -53,6 +53,11 @@ inline bool key_norm_max_applies(int64_t B, int64_t H, int64_t D) {
 }
 cudaError_t launch_norm_max(const void* q, const void* k, float* nmax, int64_t B, int64_t rows, int64_t H,
                             int64_t D, int sms, cudaStream_t stream);
+// The pre-pass and the frozen row max it enables pay when each query row of a launch meets many keys
+// (the row maxima saved grow with them, the pre-pass's read of q and k does not); `force` is
+// RA_DEBUG_FROZEN_MAX.
+constexpr int64_t kFrozenMaxMinKeys = 65536;
+inline bool frozen_max_pays(int64_t keys_per_row, bool force) { return force || keys_per_row >= kFrozenMaxMinKeys; }
 
 // pool.cu: stream-ordered scratch of the allocating entry points, from a library-owned pool per
 // device that keeps freed memory reserved (the default pool when the stream is capturing).

@@ -305,7 +305,16 @@ int varlen_forward(const void* q, const void* k, const void* v, void* out, float
         t.debug = debug;
         t.status = status;
         a.varlen_striped = striped ? 1 : 0;
-        if (ra::key_norm_max_applies(1, H, D)) {  // the score bound of every query row (frozen max)
+        // keys a query row meets per launch, on average over the packed tokens: sum len^2 / S_total
+        // for a whole ring pass, a share chunk / N of it per launch
+        double sq = 0.0;
+        for (int q_ = 0; q_ < n_seqs; ++q_) {
+            const double len = (double)(cu_seqlens[q_ + 1] - cu_seqlens[q_]);
+            sq += len * len;
+        }
+        const int64_t keys_per_row = (int64_t)(sq / (double)S_total * plan.chunk / n_ring);
+        if (ra::key_norm_max_applies(1, H, D) && ra::frozen_max_pays(keys_per_row, debug == RA_DEBUG_FROZEN_MAX)) {
+            // the score bound of every query row (frozen max)
             float* nmax = reinterpret_cast<float*>(ws + w.off_kmax);
             if ((e = ra::launch_norm_max(q, k, nmax, 1, S_total, H, D, sms, stream)) != cudaSuccess)
                 return finish(ra::host_cuda_fail(e, "norm launch"));
@@ -371,7 +380,8 @@ extern "C" int ra_forward_varlen_ex(const void* q, const void* k, const void* v,
                                     int causal, int layout, int dtype, void* stream_handle, const ra_options* opt) {
     ra_options o{};
     if (opt) o = *opt;
-    if (o.debug != RA_DEBUG_NONE && o.debug != RA_DEBUG_STALL_LOADS) return RA_ERR_INVALID_ARG;
+    if (o.debug != RA_DEBUG_NONE && o.debug != RA_DEBUG_STALL_LOADS && o.debug != RA_DEBUG_FROZEN_MAX)
+        return RA_ERR_INVALID_ARG;
     return varlen_forward(q, k, v, out, lse, cu_seqlens, n_seqs, H, D, n_ring, causal, layout, dtype, o.variant,
                           o.kernel, o.steps_per_launch, static_cast<cudaStream_t>(stream_handle),
                           static_cast<uint8_t*>(o.workspace), o.workspace_bytes, o.timeout_ns, o.debug,

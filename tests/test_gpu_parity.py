@@ -173,7 +173,8 @@ def test_auto_takes_launches_of_several_steps_for_a_head_beyond_l2():
 
 
 def test_tc_frozen_max_with_a_late_dominant_key():
-    """Norms of about 16 keep the head's score bound (qmax * kmax / sqrt(D)) within 2^32 of the first
+    """(RA_DEBUG_FROZEN_MAX: the pre-pass and the frozen max at a size that would not take them.)
+    Norms of about 16 keep the head's score bound (qmax * kmax / sqrt(D)) within 2^32 of the first
     tile's max, so the kernel freezes each row's max after that tile.  Keys planted parallel to some
     query rows and met only in a later ring step then score up to the bound itself -- about 25
     (log2) above the frozen max -- and those rows must still come out as the exact softmax."""
@@ -184,11 +185,16 @@ def test_tc_frozen_max_with_a_late_dominant_key():
         for h in range(H):
             k[0, late, h] = q[0, r, h] * (k[0, late, h].norm() / q[0, r, h].norm())
     q, k, v = (t.to(torch.bfloat16) for t in (q, k, v))
-    out, lse = ra.forward(q, k, v, N, True, "striped", kernel="tc")
+    # a sequence this short takes the frozen max only on request
+    out, lse = ra.forward(q, k, v, N, True, "striped", kernel="tc", debug=ra.DEBUG_FROZEN_MAX)
     torch.cuda.synchronize()
     assert ra.get_device_status() == 0
     ref_out, ref_lse = oracle.attention(q.cpu(), k.cpu(), v.cpu(), True, threads=THREADS)
     compare(out, lse, ref_out, ref_lse, torch.bfloat16)
+    # and without the request (no pre-pass, the exact row max on every tile) the same bars hold
+    out2, lse2 = ra.forward(q, k, v, N, True, "striped", kernel="tc")
+    torch.cuda.synchronize()
+    compare(out2, lse2, ref_out, ref_lse, torch.bfloat16)
 
 
 # ---------------------------------------------------------------- s4k: all rows

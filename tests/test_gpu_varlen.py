@@ -139,3 +139,19 @@ def test_caller_workspace_per_step_and_reuse():
     with pytest.raises(ra.RAError):  # per-step launches need the running result: too small
         ra.forward_varlen(q, k, v, cu, 4, True, "zigzag", variant="per_step",
                           workspace=ws[:ra.varlen_workspace_size(cu, 2, 128, 4, "zigzag")])
+
+
+def test_frozen_max_on_request_for_packed_sequences():
+    """Packed sequences this short skip the score-bound pre-pass; on request they take it (and the
+    frozen row max), with the same bars."""
+    lengths = [1024, 256, 0, 2048, 512]
+    cu = np.concatenate([[0], np.cumsum(lengths)]).astype(np.int64)
+    q, k, v = (x[0] for x in inputs.make_qkv(1, int(cu[-1]), 2, 128, dtype=torch.bfloat16, device="cuda", seed=16))
+    a, la = ra.forward_varlen(q, k, v, cu, 4, True, "striped", debug=ra.DEBUG_FROZEN_MAX)
+    torch.cuda.synchronize()
+    assert ra.get_device_status() == 0
+    ref, ref_lse = oracle.attention_varlen(q[None].cpu(), k[None].cpu(), v[None].cpu(), cu, True, threads=16)
+    err = np.abs(a.float().cpu().double().numpy() - ref)
+    assert err.max() <= 2e-2 and err.mean() <= 2e-3
+    assert np.abs(la.cpu().double().numpy() - ref_lse).max() <= 1e-3
+
