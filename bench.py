@@ -66,7 +66,7 @@ PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # 4-head case (dram__bytes_read.sum + dram__bytes_write.sum) scaled by heads; valid only while
 # the sha256 of the TRAFFIC_SOURCES files, concatenated in that order, starts with the recorded
 # prefix -- otherwise traffic is null.
-TRAFFIC_RECORD = {"source_sha256_prefix": "395392999f316e0e", "bytes_per_launch": (3.552965e9 + 0.138803e9) * 8}
+TRAFFIC_RECORD = {"source_sha256_prefix": "489c96f8d0891039", "bytes_per_launch": (3.463295e9 + 0.140089e9) * 8}
 # the files whose concatenation the record's hash covers: the kernel, the helpers it inlines and
 # the host code that decides the layout it reads
 TRAFFIC_SOURCES = ("attn_tc.cu", "sm100.cuh", "layout.cuh", "api.cu")
@@ -547,10 +547,10 @@ def run_ours(args, w):
         chunk = min(N, args.steps_per_launch or 1) if args.variant == "per_step" else N
     n_att = -(-N // chunk)
     tc = args.kernel == "tc"
-    # the score-bound pre-pass runs when each query row meets >= 65536 keys per launch (RA_DEBUG_FROZEN_MAX
+    # the score-bound pre-pass runs when each query row meets >= 32768 keys per launch (RA_DEBUG_FROZEN_MAX
     # in include/ra.h): chunk x S/N keys, or for packed sequences sum(len^2) / S of them per ring pass
     keys_per_row = (sum(n * n for n in varlen_lengths(S, N, w.seed)) / S if args.varlen else S) * chunk / N
-    norms = 1 if tc and keys_per_row >= 65536 else 0
+    norms = 1 if tc and keys_per_row >= 32768 else 0
     launches_per_step = (1 if args.layout == "zigzag" and tc else 0) + norms + (
         1 if n_att == 1 else n_att + 2 * (n_att - 2) + 1)
     if args.backward:

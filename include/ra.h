@@ -93,9 +93,9 @@ enum ra_status {
  * issue no copies, so every consumer wait runs out: a test of the bounded-wait give-up path.
  * RA_DEBUG_FROZEN_MAX runs the forward kernel's score-bound pre-pass (the largest query and key norm
  * per head) and lets it freeze row maxima at any size.  Without it that happens only when a launch's
- * query rows each meet at least 65536 keys (n_ring steps x S/n_ring keys per launch, or the mean
- * sequence length for packed sequences): below that, the pre-pass's read of q and k costs more than
- * the row maxima it saves.  Results are exact either way. */
+ * query rows each meet at least 32768 keys (steps per launch x S/n_ring keys, or the mean sequence
+ * length for packed sequences): below that, the pre-pass's read of q and k costs more than the row
+ * maxima it saves.  Results are exact either way. */
 enum ra_debug { RA_DEBUG_NONE = 0, RA_DEBUG_STALL_LOADS = 1, RA_DEBUG_FROZEN_MAX = 2 };
 
 typedef struct ra_options {

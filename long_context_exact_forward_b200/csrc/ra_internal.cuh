@@ -56,7 +56,7 @@ cudaError_t launch_norm_max(const void* q, const void* k, float* nmax, int64_t B
 // The pre-pass and the frozen row max it enables pay when each query row of a launch meets many keys
 // (the row maxima saved grow with them, the pre-pass's read of q and k does not); `force` is
 // RA_DEBUG_FROZEN_MAX.
-constexpr int64_t kFrozenMaxMinKeys = 65536;
+constexpr int64_t kFrozenMaxMinKeys = 32768;
 inline bool frozen_max_pays(int64_t keys_per_row, bool force) { return force || keys_per_row >= kFrozenMaxMinKeys; }
 
 // pool.cu: stream-ordered scratch of the allocating entry points, from a library-owned pool per
