@@ -5,7 +5,8 @@
 //     P = exp(S / sqrt(D) - lse),  dP = dO V^T,  dS = P (dP - Delta),  Delta = rowsum(dO * O)
 //     dQ = dS K / sqrt(D),  dK = dS^T Q / sqrt(D),  dV = P^T dO
 // with the four products of a 128 x 128 tile on the tensor cores (bf16 operands, fp32 accumulators
-// in TMEM) and the elementwise step on 128 threads, one TMEM lane (tile row) each.
+// in TMEM) and the elementwise step on 256 threads, two per TMEM lane (tile row), each on half of
+// the tile's columns.
 //
 // Inputs are read through 5-D TMA maps: in place for the contiguous and striped layouts, from
 // shard-major copies for zigzag.
@@ -13,7 +14,7 @@
 // bwd_dq_tc_kernel   one CTA per 128-row query tile of shard i; key tiles of the blocks
 //                    j = (i - s) mod N in ring order.  TMEM: S of even / odd tiles [0,128) /
 //                    [128,256), dP [256,384), dQ [384,512).  Per key tile t: S = Q K^T and dP = dO V^T
-//                    (SS), the elementwise warps write dS (bf16) over the first 64 columns of S_t,
+//                    (SS), the elementwise warps write dS (bf16) over S_t (packed_col below),
 //                    then dQ += dS K (TS, K as the MN-major operand, like V in the forward P V).
 //                    S of tile t + 1 is computed while the elementwise warps work on tile t, and
 //                    dP of tile t + 1 goes before dQ of tile t, so the elementwise warps wait only
@@ -27,9 +28,9 @@
 // Roles (320 threads): warp 0 TMA producer (lane 0 issues), warp 1 MMA issuer (converged warp,
 // elect.sync picks the issuing lane) and TMEM owner, warps 2-9 elementwise: warp w reads TMEM lanes
 // 32 (w mod 4) .. +31, warps 2-5 the columns 0..63 of every tile and warps 6-9 the columns 64..127
-// (the elementwise steps have no row reductions, so the two halves never meet).  The streamed tiles go through two shared-memory stages.  Every wait is
-// bounded; on give-up the CTA records RA_ERR_DEVICE_TIMEOUT, lets its copies and MMAs drain, frees
-// TMEM and exits.
+// (the elementwise steps have no row reductions, so the two halves never meet).  The streamed tiles
+// go through two shared-memory stages.  Every wait is bounded; on give-up the CTA records
+// RA_ERR_DEVICE_TIMEOUT, lets its copies and MMAs drain, frees TMEM and exits.
 #include <cuda_bf16.h>
 
 #include "ra.h"
